@@ -1,0 +1,236 @@
+"""ctypes front end of the CSA2 CPU oracle (test infrastructure only).
+
+Every array crosses as a numpy array; raw bit patterns travel as uint16 (bf16) or
+uint8 (E4M3, packed E2M1). The arithmetic lives in csa2_oracle.c; this file only
+marshals arguments and composes the per-query steps in the order the pages describe
+them (score -> Top-K / pool -> gather -> attention).
+"""
+import ctypes as C
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+BF16, E4M3 = 0, 1
+POOL_BLOCK = 8
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        d, u8, u16, i32, i64, f32 = (C.c_double, C.c_uint8, C.c_uint16, C.c_int32,
+                                     C.c_int64, C.c_float)
+        P = C.c_void_p
+        L.orc_bf16_value.restype = d
+        L.orc_bf16_value.argtypes = [u16]
+        L.orc_e2m1_value.restype = d
+        L.orc_e2m1_value.argtypes = [C.c_uint]
+        L.orc_e4m3_value.restype = d
+        L.orc_e4m3_value.argtypes = [u8]
+        L.orc_e4m3_encode.restype = u8
+        L.orc_e4m3_encode.argtypes = [d]
+        L.orc_e2m1_encode.restype = C.c_uint
+        L.orc_e2m1_encode.argtypes = [d]
+        L.orc_fp4_scale_code.restype = u8
+        L.orc_fp4_scale_code.argtypes = [d]
+        L.orc_fp4_code.restype = C.c_uint
+        L.orc_fp4_code.argtypes = [d, d]
+        for nm in ("orc_fp4_scale_codes_many", "orc_e4m3_encode_many"):
+            getattr(L, nm).restype = None
+            getattr(L, nm).argtypes = [P, i64, P]
+        L.orc_fp4_codes_many.restype = None
+        L.orc_fp4_codes_many.argtypes = [P, P, i64, P]
+        L.orc_quantize_block16.restype = None
+        L.orc_quantize_block16.argtypes = [P, P, P]
+        L.orc_quantize_entries.restype = None
+        L.orc_quantize_entries.argtypes = [P, i64, i64, C.c_int, P, P]
+        L.orc_dequant_entry.restype = None
+        L.orc_dequant_entry.argtypes = [P, P, C.c_int, P]
+        L.orc_index_scores.restype = None
+        L.orc_index_scores.argtypes = [C.c_int, C.c_int, C.c_int, P, P, P, P, i64, P]
+        L.orc_topk.restype = i64
+        L.orc_topk.argtypes = [P, P, i64, i64, P]
+        L.orc_pool.restype = i64
+        L.orc_pool.argtypes = [P, i64, i64, C.c_int, P]
+        L.orc_attention.restype = None
+        L.orc_attention.argtypes = [C.c_int, C.c_int, P, P, i64, d, P]
+        L.orc_main_entry_bytes.restype = C.c_int
+        L.orc_main_entry_bytes.argtypes = [C.c_int]
+        L.orc_kv_bytes_per_token.restype = d
+        L.orc_kv_bytes_per_token.argtypes = [C.c_int, d, C.c_int, C.c_int, C.c_int, C.c_int]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(C.c_void_p) if a is not None else None
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---- formats -------------------------------------------------------------------------
+
+def bf16_value(bits):
+    return lib().orc_bf16_value(int(bits))
+
+
+def e2m1_value(code):
+    return lib().orc_e2m1_value(int(code))
+
+
+def e4m3_value(code):
+    return lib().orc_e4m3_value(int(code))
+
+
+def e4m3_encode(v):
+    return int(lib().orc_e4m3_encode(float(v)))
+
+
+def e2m1_encode(v):
+    return int(lib().orc_e2m1_encode(float(v)))
+
+
+def bf16_array_to_f64(bits):
+    bits = _c(bits, np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def e4m3_array_to_f64(codes):
+    table = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+    return table[_c(codes, np.uint8)]
+
+
+def e4m3_encode_many(v):
+    v = _c(v, np.float64)
+    out = np.zeros(v.shape[0], np.uint8)
+    lib().orc_e4m3_encode_many(_p(v), v.shape[0], _p(out))
+    return out
+
+
+def fp4_scale_codes(amax):
+    """Scale code step of the block quantiser for many block maxima."""
+    a = _c(amax, np.float64)
+    out = np.zeros(a.shape[0], np.uint8)
+    lib().orc_fp4_scale_codes_many(_p(a), a.shape[0], _p(out))
+    return out
+
+
+def fp4_codes(x, s):
+    """Element code step of the block quantiser for many (x, decoded scale) pairs."""
+    x = _c(x, np.float64)
+    s = _c(s, np.float64)
+    out = np.zeros(x.shape[0], np.uint8)
+    lib().orc_fp4_codes_many(_p(x), _p(s), x.shape[0], _p(out))
+    return out
+
+
+def quantize_block16(x):
+    x = _c(x, np.float64)
+    codes = np.zeros(16, np.uint8)
+    sc = np.zeros(1, np.uint8)
+    lib().orc_quantize_block16(_p(x), _p(codes), _p(sc))
+    return codes, int(sc[0])
+
+
+def quantize_entries(kv_bits, D=512):
+    """kv_bits: uint16 [n, D] bf16 patterns -> (codes uint8 [n, D/2], scales uint8 [n, D/16])."""
+    kv_bits = _c(kv_bits, np.uint16).reshape(-1, D)
+    n = kv_bits.shape[0]
+    codes = np.zeros((n, D // 2), np.uint8)
+    scales = np.zeros((n, D // 16), np.uint8)
+    lib().orc_quantize_entries(_p(kv_bits), n, D, D, _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequant_entries(codes, scales, D=512):
+    codes = _c(codes, np.uint8).reshape(-1, D // 2)
+    scales = _c(scales, np.uint8).reshape(-1, D // 16)
+    out = np.zeros((codes.shape[0], D), np.float64)
+    for i in range(codes.shape[0]):
+        row = out[i]
+        lib().orc_dequant_entry(_p(codes[i]), _p(scales[i]), D, _p(row))
+    return out
+
+
+# ---- indexer / selection ---------------------------------------------------------------
+
+def index_scores(q, w, k, dtype, rows=None):
+    """q: [H, Di] raw (uint16 bf16 or uint8 E4M3); w: float32 [H]; k: [n_all, Di] raw.
+    rows: optional int32 positions; returns float64 scores for rows (or all rows)."""
+    npdt = np.uint16 if dtype == BF16 else np.uint8
+    q = _c(q, npdt)
+    k = _c(k, npdt)
+    w = _c(w, np.float32)
+    H, Di = q.shape
+    if rows is None:
+        n = k.shape[0]
+        r = None
+    else:
+        r = _c(rows, np.int32)
+        n = r.shape[0]
+    s = np.zeros(n, np.float64)
+    lib().orc_index_scores(H, Di, dtype, _p(q), _p(w), _p(k), _p(r), n, _p(s))
+    return s
+
+
+def topk(scores, K, ids=None):
+    s = _c(scores, np.float64)
+    i = _c(ids, np.int32) if ids is not None else None
+    out = np.zeros(K, np.int32)
+    lib().orc_topk(_p(s), _p(i), s.shape[0], K, _p(out))
+    return out
+
+
+def pool(scores, nblk, blk=POOL_BLOCK):
+    s = _c(scores, np.float64)
+    out = np.zeros(nblk * blk, np.int32)
+    lib().orc_pool(_p(s), s.shape[0], nblk, blk, _p(out))
+    return out
+
+
+# ---- attention ---------------------------------------------------------------------
+
+def attention(q, rows, tau):
+    """q: float64 [H, D]; rows: float64 [n, D] -> float64 [H, D]."""
+    q = _c(q, np.float64)
+    rows = _c(rows, np.float64).reshape(-1, q.shape[1])
+    H, D = q.shape
+    out = np.zeros((H, D), np.float64)
+    lib().orc_attention(H, D, _p(q), _p(rows), rows.shape[0], float(tau), _p(out))
+    return out
+
+
+def gather_rows(codes, scales, idx, D=512):
+    """Dequantised main-KV rows for the indices != -1, in the order given."""
+    sel = [int(i) for i in idx if i >= 0]
+    if not sel:
+        return np.zeros((0, D), np.float64)
+    return dequant_entries(codes[sel], scales[sel], D)
+
+
+def attention_decode_query(q_bits, codes, scales, idx, swa_codes, tau, swa_valid=None, D=512):
+    """One decode query: q bf16 bits [H, D]; idx [K]; swa E4M3 [W, D] (last swa_valid
+    rows valid when given). Returns float64 [H, D]."""
+    q = bf16_array_to_f64(q_bits).reshape(-1, D)
+    sel = gather_rows(codes, scales, idx, D)
+    W = swa_codes.shape[0]
+    v = W if swa_valid is None else int(swa_valid)
+    swa = e4m3_array_to_f64(swa_codes[W - v:]).reshape(-1, D)
+    rows = np.concatenate([sel, swa], axis=0)
+    return attention(q, rows, tau)
+
+
+def bytes_per_token(D=512, indexer_entry_bytes=68.0, enc_full=3, enc_ratio=2, dec_full=1,
+                    dec_ratio=1):
+    return lib().orc_kv_bytes_per_token(D, float(indexer_entry_bytes), enc_full, enc_ratio,
+                                        dec_full, dec_ratio)
+
+
+def main_entry_bytes(D=512):
+    return lib().orc_main_entry_bytes(D)
