@@ -1,0 +1,477 @@
+"""CSA2 decode benchmark on B200: queries/s and HBM GB/s of the whole hot path.
+
+One step = one pass of the CSA2 path over one batch of synthetic, seeded inputs:
+FP4 quantize-on-write of the new entries, indexer scoring + exact Top-K (and the candidate
+pool / Reindex / Reuse layers the workload has), then the fused gather + dequant + sparse /
+sliding-window attention of every layer. Everything runs in libcsa2's kernels.
+
+Default workload: Full-mode decode, batch 32, 65,536-token context at compression ratio 2
+(32,768 compressed entries per sequence), FP8 indexer keys with 64 heads, Top-512, 64 query
+heads of 512 channels, 128-row FP8 window.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+For N > 1 launch under torchrun: every rank runs its own batch (weak scaling, no collective
+on the data path); the time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp4_compressed_sparse_quantize_b200 import csa2, synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "decode_full_b32_ctx64k_r2"
+L2_FLUSH_BYTES = 256 << 20
+SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csrc", "indexer.cu")
+
+# DRAM traffic of one indexer-scan launch, from `ncu --metrics dram__bytes_read.sum,
+# dram__bytes_write.sum` (summary in profiles/), valid only for the indexer.cu it was taken
+# on: {workload: (sha1 of indexer.cu, bytes per launch)}.
+SCAN_TRAFFIC = {}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---- clocks sampler ------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- workload ----------------------------------------------------------------------------
+
+class Decode:
+    """Device-resident state of one decode workload plus its per-step inputs."""
+
+    def __init__(self, w, seed, dev):
+        self.w = w
+        self.dev = dev
+        self.seed = seed
+        B, N, cap = w.B, w.N, w.cap
+        self.tau = 1.0 / math.sqrt(synth.D_MAIN)
+        # layers' query-side inputs; planted keys follow the layers' indexer queries
+        self.layers = [synth.layer_inputs(w, li, seed, dev) for li in range(len(w.layers))]
+        dirs = None
+        if w.planted:
+            dirs = synth.planted_direction([L["q_I"] for L, m in zip(self.layers, w.layers)
+                                            if m in ("full", "reindex")])
+        self.k_I, self.planted = synth.indexer_keys(w, seed, dev, planted_dirs=dirs)
+        # FP4 cache built once by the library's own quantize-on-write
+        self.codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
+        chunk = max(1, (1 << 28) // (cap * 1024))
+        for b0 in range(0, B, chunk):
+            b1 = min(B, b0 + chunk)
+            src = torch.empty((b1 - b0, cap, synth.D_MAIN), dtype=torch.bfloat16, device=dev)
+            for b in range(b0, b1):
+                src[b - b0] = _main_rows(w, seed, b, dev)
+            csa2.quantize_kv(src, torch.zeros(b1 - b0, dtype=torch.int32, device=dev),
+                             self.codes[b0:b1], self.scales[b0:b1])
+            del src
+        self.n_vis = synth.decode_positions(w, dev)
+        self.dst = (self.n_vis - 1).contiguous()
+        # the newest entry is re-quantised every step from its bf16 row
+        self.kv_new = torch.stack([_main_rows(w, seed, b, dev)[N - 1:N] for b in range(B)])
+        self.idx = [torch.empty((B, 1, w.K), dtype=torch.int32, device=dev) for _ in w.layers]
+        self.out = [torch.empty((B, w.H, synth.D_MAIN), dtype=torch.float32, device=dev)
+                    for _ in w.layers]
+        self.pool = None
+        if w.pool:
+            self.pool = torch.empty((B, 1, synth.POOL_BLOCKS * synth.POOL_BLOCK),
+                                    dtype=torch.int32, device=dev)
+        P = synth.POOL_BLOCKS * synth.POOL_BLOCK
+        ws_i = max(csa2.workspace_bytes(0, B, 1, w.H_I, cap, w.K,
+                                        synth.POOL_BLOCKS if w.pool else 0),
+                   csa2.workspace_bytes(0, B, 1, w.H_I, P, w.K))
+        self.ws_idx = csa2.new_workspace(ws_i)
+        self.ws_attn = csa2.new_workspace(csa2.workspace_bytes(1, B, 1, w.H, cap, w.K))
+        torch.cuda.synchronize()
+
+    def step(self, scan_events=None, stream=None):
+        w = self.w
+        csa2.quantize_kv(self.kv_new, self.dst, self.codes, self.scales,
+                         status=self.ws_idx[:4].view(torch.int32), stream=stream)
+        cur = None
+        for li, mode in enumerate(w.layers):
+            L = self.layers[li]
+            if mode == "full":
+                if scan_events is not None:
+                    csa2.set_stage_events(*scan_events)
+                    scan_events = None
+                csa2.index_score_topk("full", L["q_I"], L["w"], self.k_I, w.K, self.idx[li],
+                                      self.ws_idx, n_vis0=self.n_vis, pool_out=self.pool,
+                                      pool_blocks=synth.POOL_BLOCKS if w.pool else 0,
+                                      stream=stream)
+                cur = self.idx[li]
+            elif mode == "reindex":
+                csa2.index_score_topk("reindex", L["q_I"], L["w"], self.k_I, w.K, self.idx[li],
+                                      self.ws_idx, n_vis0=self.n_vis, pool_in=self.pool,
+                                      stream=stream)
+                cur = self.idx[li]
+            else:
+                csa2.index_score_topk("reuse", L["q_I"], L["w"], self.k_I, w.K, cur,
+                                      self.ws_idx, n_vis0=self.n_vis, stream=stream)
+            csa2.sparse_attn_decode(mode, L["q"], self.codes, self.scales, cur.view(w.B, w.K),
+                                    L["swa"], self.out[li], self.ws_attn, scale=self.tau,
+                                    stream=stream)
+
+    def launches_per_step(self):
+        n = 1  # quantize
+        for m in self.w.layers:
+            if m == "full":
+                n += 4 + (2 if self.w.pool else 0)   # prep, scan, collect, finalize (+ pool)
+            elif m == "reindex":
+                n += 4
+            n += 1 + (1 if csa2_attn_splits(self.w) > 1 else 0)
+        return n
+
+    def step_inputs(self):
+        """Per-step host->device inputs: every layer's queries and window rows, the new row."""
+        t = [self.kv_new]
+        for L in self.layers:
+            t += [L["q_I"], L["w"], L["q"], L["swa"]]
+        return t
+
+    def step_outputs(self):
+        return self.out
+
+    def algorithmic_bytes(self):
+        w = self.w
+        B, N, K, H, W = w.B, w.N, w.K, w.H, synth.WINDOW
+        ek = 2 if w.idx_dtype == "bf16" else 1
+        tot = B * (512 * 2 + 288)                         # quantize-on-write
+        scan = 0
+        for m in w.layers:
+            if m in ("full", "reindex"):
+                rows = N if m == "full" else synth.POOL_BLOCKS * synth.POOL_BLOCK
+                b = B * (rows * 128 * ek + w.H_I * 128 * ek + w.H_I * 4 + K * 4)
+                if m == "full":
+                    scan = B * (N * 128 * ek + w.H_I * 128 * ek + w.H_I * 4)
+                if m == "reindex":
+                    b += B * rows * 4
+                if m == "full" and w.pool:
+                    b += B * synth.POOL_BLOCKS * synth.POOL_BLOCK * 4
+                tot += b
+            tot += B * (K * 4 + K * 288 + W * 512 + H * 512 * 2 + H * 512 * 4)
+        return tot, scan
+
+
+def csa2_attn_splits(w):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    nch = (w.K + synth.WINDOW + 63) // 64
+    ns = min(nch, (2 * sms + w.B - 1) // w.B)
+    cps = (nch + ns - 1) // ns
+    return (nch + cps - 1) // cps
+
+
+def _main_rows(w, seed, b, dev):
+    """bf16 [cap, 512] main-KV source rows of sequence b (drawn per sequence, exactly as
+    synth.main_kv_source draws them)."""
+    g = synth._gen(seed, 1, b, dev)
+    x = torch.randn((w.cap, synth.D_MAIN), generator=g, device=dev, dtype=torch.float32)
+    if w.lognormal_channels:
+        s = torch.exp(torch.randn((synth.D_MAIN,), generator=synth._gen(seed, 2, b, dev),
+                                  device=dev, dtype=torch.float32))
+        x = x * s
+    return x.to(torch.bfloat16)
+
+
+# ---- CPU baseline / reference arm (the oracle as it stands) --------------------------------------
+
+def oracle_queries(state, budget_s):
+    """Run the oracle over whole decode queries of this workload until ~budget_s of CPU work;
+    returns (queries done, seconds, cores)."""
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as O
+    w = state.w
+    ek = O.BF16 if w.idx_dtype == "bf16" else O.E4M3
+    done, t_total = 0, 0.0
+    b = 0
+    while t_total < budget_s and b < w.B:
+        # inputs of sequence b (copied out of device memory before the clock starts)
+        k_raw = state.k_I[b, :w.N].contiguous().cpu().view(torch.uint8 if ek == O.E4M3 else torch.int16).numpy()
+        if ek == O.BF16:
+            k_raw = k_raw.view(np.uint16)
+        src = _main_rows(w, state.seed, b, state.dev)[: w.N].cpu().view(torch.int16).numpy().view(np.uint16)
+        lay = []
+        for L in state.layers:
+            qi = L["q_I"][b, 0].contiguous().cpu().view(torch.uint8 if ek == O.E4M3 else torch.int16).numpy()
+            if ek == O.BF16:
+                qi = qi.view(np.uint16)
+            lay.append((qi, L["w"][b, 0].cpu().numpy(), L["q"][b].cpu().view(torch.int16).numpy().view(np.uint16),
+                        L["swa"][b].cpu().view(torch.uint8).numpy()))
+        t0 = time.perf_counter()
+        O.quantize_entries(src[w.N - 1:w.N])              # quantize-on-write of the new entry
+        cur = None
+        pool = None
+        for (qi, wt, qb, swa), mode in zip(lay, w.layers):
+            if mode == "full":
+                s = O.index_scores(qi, wt, k_raw, ek)
+                cur = O.topk(s, w.K)
+                if w.pool:
+                    pool = O.pool(s, synth.POOL_BLOCKS)
+            elif mode == "reindex":
+                ids = pool[pool >= 0]
+                s = O.index_scores(qi, wt, k_raw, ek, rows=ids)
+                cur = O.topk(s, w.K, ids)
+            sel = [int(i) for i in cur if i >= 0]
+            c, sc = O.quantize_entries(src[sel])
+            rows = np.concatenate([O.dequant_entries(c, sc),
+                                   O.e4m3_array_to_f64(swa).reshape(-1, 512)])
+            O.attention(O.bf16_array_to_f64(qb).reshape(-1, 512), rows, state.tau)
+        t_total += time.perf_counter() - t0
+        done += 1
+        b += 1
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return done, t_total, cores
+
+
+# ---- main -------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=1234)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, rank, world, local)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    w = synth.WORKLOADS[args.workload]
+    if w.kind != "decode":
+        raise SystemExit("bench.py times the decode path; prefill is covered by the tests")
+    state = Decode(w, args.seed + 7919 * rank, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(3, args.warmup)):
+        state.step()
+    torch.cuda.synchronize()
+    assert csa2.read_device_status(state.ws_idx) == 0, "device status set during warm-up"
+    assert csa2.read_device_status(state.ws_attn) == 0
+
+    clocks = Clocks(local)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)                   # evict L2 between steps (outside the events)
+        ev[k][0].record(stream)
+        state.step(scan_events=sev[k])
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if pg:
+        pg.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    scan_ms = [a.elapsed_time(b) for a, b in sev]
+    total_ms = sum(step_ms)
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end-to-end: host inputs -> device -> step -> host output, through the public API
+    ins = state.step_inputs()
+    outs = state.step_outputs()
+    h_in = [x.detach().cpu().pin_memory() for x in ins]
+    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    bi = sum(x.numel() * x.element_size() for x in h_in)
+    bo = sum(x.numel() * x.element_size() for x in h_out)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        e2e_ev[k][0].record(stream)
+        for d, h in zip(ins, h_in):
+            d.copy_(h, non_blocking=True)
+        state.step()
+        for h, o in zip(h_out, outs):
+            h.copy_(o, non_blocking=True)
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st_i = csa2.read_device_status(state.ws_idx)
+    st_a = csa2.read_device_status(state.ws_attn)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, secs, cores = oracle_queries(state, args.cpu_budget)
+        cpu = {"value": n / secs, "unit": "queries/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n} whole decode queries (sequences 0..{n - 1}) of the same workload, "
+                         f"{secs:.1f} s of oracle time"}
+
+    if rank == 0:
+        alg_bytes, scan_bytes = state.algorithmic_bytes()
+        per_step_ms = total_ms / args.steps
+        queries = w.B * world * args.steps
+        value = queries / (total_ms / 1e3)
+        peak, src = peaks()
+        scan_avg = sum(scan_ms) / len(scan_ms)
+        achieved = scan_bytes / (scan_avg / 1e3) / 1e9
+        sha = hashlib.sha1(open(SCAN_KERNEL_SRC, "rb").read()).hexdigest()
+        tr = SCAN_TRAFFIC.get(args.workload)
+        traffic = tr[1] if tr and tr[0] == sha else None
+        line = {
+            "metric": "CSA2 decode queries/s & HBM GB/s at 64K-1M ctx (frac of roofline), 1 B200",
+            "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": per_step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3/fp4/fp16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": args.workload, "batch_per_gpu": w.B, "context_tokens": w.ctx,
+                       "ratio": w.ratio, "compressed_entries": w.N, "topk": w.K,
+                       "indexer_heads": w.H_I, "indexer_dtype": w.idx_dtype, "query_heads": w.H,
+                       "window": synth.WINDOW, "layers": list(w.layers),
+                       "parallelism": f"dp{world} (independent batches)",
+                       "l2": "flushed between steps (256 MiB write)"},
+            "hbm_gbs_step": alg_bytes / (per_step_ms / 1e3) / 1e9,
+            "roofline": {"kernel": "csa2 indexer scan (tcgen05, FP8 keys)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": src,
+                         "frac_of_8TBs": achieved / 8000.0,
+                         "bytes_per_launch": scan_bytes, "avg_launch_ms": scan_avg,
+                         "traffic": traffic},
+            "step_roofline_frac": (alg_bytes / (per_step_ms / 1e3) / 1e9) / peak,
+            "e2e": {"value": queries / (e2e_ms / 1e3), "unit": "queries/s",
+                    "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+            "gpu_launches": state.launches_per_step() * args.steps,
+            "clocks": clk,
+            "device_status": [st_i, st_a],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def reference_arm(args, rank, world, local):
+    """The oracle, as it stands, timed on the host cores: rank 0 only."""
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        torch.cuda.set_device(local)
+    state = Decode(w, args.seed, dev)
+    # each step is a bounded sample: whole queries until ~budget/steps seconds
+    per = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_queries(state, per)
+    n_tot, s_tot, cores = 0, 0.0, 1
+    for _ in range(args.steps):
+        n, s, cores = oracle_queries(state, per)
+        n_tot += n
+        s_tot += s
+    value = n_tot / s_tot
+    line = {"impl": "reference",
+            "metric": "CSA2 decode queries/s & HBM GB/s at 64K-1M ctx (frac of roofline), 1 B200",
+            "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * s_tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "batch_per_gpu": w.B},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{n_tot} whole decode queries over {args.steps} steps"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

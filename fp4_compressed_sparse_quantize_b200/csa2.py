@@ -1,0 +1,221 @@
+"""Thin Python binding of libcsa2 (ctypes). Argument marshalling only: every step of the
+CSA2 path runs in the library's CUDA kernels. torch supplies device memory and streams.
+
+The names mirror the C ABI in include/csa2.h (csa2_quantize_kv -> quantize_kv, ...).
+Importing this module does not need a GPU; calling an operation does, and raises
+Csa2Error when the library is missing or reports an error. There is no fallback.
+"""
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE = range(6)
+MODE = {"full": 0, "reindex": 1, "reuse": 2}
+DTYPE = {torch.bfloat16: 0, torch.float8_e4m3fn: 1}
+OP_INDEX_SCORE_TOPK, OP_SPARSE_ATTN_DECODE, OP_SPARSE_ATTN_PREFILL = 0, 1, 2
+DEV_BAD_INDEX, DEV_BAD_COUNT, DEV_TIMEOUT = 1, 2, 4
+D_MAIN, D_INDEX, POOL_BLOCK = 512, 128, 8
+EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode",
+           "csa2_sparse_attn_prefill", "csa2_workspace_bytes", "csa2_status_string",
+           "csa2_read_device_status", "csa2_reset_device_status", "csa2_version",
+           "csa2_debug_bounded_wait", "csa2_set_stage_events")
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libcsa2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise Csa2Error(ERR_CUDA, f"{LIB_PATH} is missing; build it with "
+                                      "python fp4_compressed_sparse_quantize_b200/build.py")
+        L = C.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
+        L.csa2_quantize_kv.argtypes = [P, i32, i32, i64, i64, P, P, P, i64, P, P]
+        L.csa2_index_score_topk.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P, i32, P,
+                                            i32, P, i32, P, i32, P, P, P, sz, P]
+        L.csa2_sparse_attn_decode.argtypes = [i32, i32, i32, P, P, P, i64, P, i32, P, i32, P,
+                                              f32, P, P, sz, P]
+        L.csa2_sparse_attn_prefill.argtypes = [i32, i32, i32, P, P, P, i64, P, i32, P, i32, P,
+                                               f32, P, P, sz, P]
+        L.csa2_workspace_bytes.argtypes = [i32, i32, i32, i32, i64, i32, i32]
+        L.csa2_workspace_bytes.restype = sz
+        L.csa2_status_string.argtypes = [i32]
+        L.csa2_status_string.restype = C.c_char_p
+        L.csa2_read_device_status.argtypes = [P, P, P]
+        L.csa2_reset_device_status.argtypes = [P, P]
+        L.csa2_debug_bounded_wait.argtypes = [P, C.c_uint64, P]
+        L.csa2_set_stage_events.argtypes = [P, P]
+        for name in EXPORTS:
+            if name not in ("csa2_workspace_bytes", "csa2_status_string"):
+                getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().csa2_status_string(int(status)).decode()
+
+
+def _p(t):
+    if t is None:
+        return None
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _check(status, what):
+    if status != OK:
+        raise Csa2Error(status, what)
+
+
+def _need(t, dtype, name, dev=True):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise Csa2Error(ERR_ARG, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise Csa2Error(ERR_ARG, f"{name} must be contiguous")
+    if dev and not t.is_cuda:
+        raise Csa2Error(ERR_ARG, f"{name} must be a CUDA tensor")
+
+
+# ---- workspace ---------------------------------------------------------------------------
+
+def workspace_bytes(op, B, T, H, cap, K, pool_blocks=0):
+    return int(lib().csa2_workspace_bytes(int(op), int(B), int(T), int(H), int(cap), int(K),
+                                          int(pool_blocks)))
+
+
+def new_workspace(nbytes, device="cuda"):
+    """Zero-filled workspace (the device status word starts cleared)."""
+    n = max(int(nbytes), 256)
+    return torch.zeros((n + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+
+def read_device_status(ws, stream=None):
+    out = C.c_int32(0)
+    st = lib().csa2_read_device_status(_p(ws), C.byref(out), _stream(stream))
+    if st not in (OK, ERR_DEVICE):
+        _check(st, "csa2_read_device_status")
+    return out.value
+
+
+def reset_device_status(ws, stream=None):
+    _check(lib().csa2_reset_device_status(_p(ws), _stream(stream)), "csa2_reset_device_status")
+
+
+def set_stage_events(ev_start, ev_stop):
+    """Record torch.cuda.Event pair around the next indexer-scan launch of this thread."""
+    a = C.c_void_p(ev_start.cuda_event) if ev_start is not None else None
+    b = C.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
+    _check(lib().csa2_set_stage_events(a, b), "csa2_set_stage_events")
+
+
+def debug_bounded_wait(status_word, timeout_ns, stream=None):
+    _need(status_word, torch.int32, "status_word")
+    _check(lib().csa2_debug_bounded_wait(_p(status_word), int(timeout_ns), _stream(stream)),
+           "csa2_debug_bounded_wait")
+
+
+# ---- operations ---------------------------------------------------------------------------
+
+def quantize_kv(kv, dst_off, codes, scales, status=None, stream=None):
+    """kv bf16 [B, n_new, 512] (row stride may exceed 512); dst_off int32 [B];
+    codes uint8 [B, cap, 256]; scales uint8 [B, cap, 32]."""
+    _need(dst_off, torch.int32, "dst_off")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    if kv.dtype != torch.bfloat16 or kv.stride(-1) != 1 or not kv.is_cuda:
+        raise Csa2Error(ERR_ARG, "kv must be a CUDA bf16 tensor with unit channel stride")
+    B, n_new, D = kv.shape
+    cap = codes.shape[1]
+    st = lib().csa2_quantize_kv(_p(kv), B, n_new, kv.stride(1), kv.stride(0), _p(dst_off),
+                                _p(codes), _p(scales), cap, _p(status), _stream(stream))
+    _check(st, "csa2_quantize_kv")
+
+
+def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None, ratio=1,
+                     pool_in=None, pool_out=None, pool_blocks=0, scores_out=None, stream=None):
+    """q_I [B, T, H_I, 128] (bf16 or E4M3), w fp32 [B, T, H_I], k_I [B, cap, 128] of the same
+    dtype, idx_out int32 [B, T, K]. Decode: n_vis0 int32 [B]. Prefill: q_pos0 int32 [B] and
+    ratio. Reindex: pool_in int32 [B, T, P]. Full with a pool: pool_out int32
+    [B, T, pool_blocks * 8]."""
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    B, T, H_I, Di = q_I.shape
+    if q_I.dtype not in DTYPE or k_I.dtype != q_I.dtype:
+        raise Csa2Error(ERR_ARG, "q_I and k_I must share a dtype (bf16 or float8_e4m3fn)")
+    for t, nm in ((q_I, "q_I"), (k_I, "k_I")):
+        _need(t, q_I.dtype, nm)
+    _need(w, torch.float32, "w")
+    _need(idx_out, torch.int32, "idx_out")
+    _need(n_vis0, torch.int32, "n_vis0")
+    _need(q_pos0, torch.int32, "q_pos0")
+    _need(pool_in, torch.int32, "pool_in")
+    _need(pool_out, torch.int32, "pool_out")
+    _need(scores_out, torch.float32, "scores_out")
+    cap = k_I.shape[1]
+    P_in = pool_in.shape[-1] if pool_in is not None else 0
+    st = lib().csa2_index_score_topk(
+        m, B, T, H_I, DTYPE[q_I.dtype], _p(q_I), _p(w), _p(k_I), cap, _p(n_vis0), int(ratio),
+        _p(q_pos0), int(K), _p(pool_in), P_in, _p(pool_out), int(pool_blocks), _p(idx_out),
+        _p(scores_out), _p(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    _check(st, "csa2_index_score_topk")
+
+
+def sparse_attn_decode(mode, q, codes, scales, idx, swa, out, ws, scale=None, swa_valid=None,
+                       stream=None):
+    """q bf16 [B, H, 512]; idx int32 [B, K]; swa E4M3 [B, W, 512]; out fp32 [B, H, 512]."""
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    _need(q, torch.bfloat16, "q")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    _need(idx, torch.int32, "idx")
+    _need(swa, torch.float8_e4m3fn, "swa")
+    _need(out, torch.float32, "out")
+    _need(swa_valid, torch.int32, "swa_valid")
+    B, H, D = q.shape
+    K = idx.shape[-1] if idx is not None else 0
+    W = swa.shape[1] if swa is not None else 0
+    sc = float(scale) if scale is not None else D_MAIN ** -0.5
+    st = lib().csa2_sparse_attn_decode(m, B, H, _p(q), _p(codes), _p(scales), codes.shape[1],
+                                       _p(idx), K, _p(swa), W, _p(swa_valid), sc, _p(out),
+                                       _p(ws), ws.numel(), _stream(stream))
+    _check(st, "csa2_sparse_attn_decode")
+
+
+def sparse_attn_prefill(q, codes, scales, idx, swa, out, ws, W, q_pos0=None, scale=None,
+                        stream=None):
+    """q bf16 [B, T, H, 512]; idx int32 [B, T, K]; swa E4M3 [B, W-1+T, 512];
+    out fp32 [B, T, H, 512]."""
+    _need(q, torch.bfloat16, "q")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    _need(idx, torch.int32, "idx")
+    _need(swa, torch.float8_e4m3fn, "swa")
+    _need(out, torch.float32, "out")
+    _need(q_pos0, torch.int32, "q_pos0")
+    B, T, H, D = q.shape
+    K = idx.shape[-1]
+    sc = float(scale) if scale is not None else D_MAIN ** -0.5
+    st = lib().csa2_sparse_attn_prefill(B, T, H, _p(q), _p(codes), _p(scales), codes.shape[1],
+                                        _p(idx), K, _p(swa), int(W), _p(q_pos0), sc, _p(out),
+                                        _p(ws), ws.numel(), _stream(stream))
+    _check(st, "csa2_sparse_attn_prefill")

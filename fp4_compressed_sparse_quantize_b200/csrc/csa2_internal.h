@@ -1,0 +1,95 @@
+// Internal launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+namespace csa2 {
+
+struct ScanLaunch {
+    int B, T, rows, G, H_I, esz;
+    int64_t cap;
+    const void* q;          // [rows][H_I][128]
+    const void* k;          // [B][cap][128]
+    const float* w;         // [rows][H_I]
+    const int32_t* n_row;   // [rows]
+    const int64_t* prefix;  // [rows/G + 1]
+    float* scores;
+    int64_t ld_scores;
+    uint32_t* hist;
+    bool pool_build;
+    uint32_t* bkey;
+    int64_t ld_bkey;
+    uint32_t* bhist;
+    bool gather;
+    const int32_t* pool;
+    int P;
+    int32_t* status;
+};
+
+cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
+                               int64_t bstride_kv, const int32_t* dst_off, uint8_t* codes,
+                               uint8_t* scales, int64_t cap, int32_t* status,
+                               cudaStream_t stream);
+
+cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
+                             const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
+                             int32_t* n_row, int64_t* prefix, int32_t* status,
+                             cudaStream_t st);
+
+cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st);
+
+// Exact Top-K over rows of fp32 scores or u32 keys.
+struct TopkLaunch {
+    int R;                   // rows
+    int K;                   // picks per row
+    const float* scores;     // [R][ld] or null (then keys)
+    const uint32_t* keys;    // [R][ld] order-preserving keys
+    int64_t ld;
+    int64_t max_n;           // largest row length (grid sizing)
+    const int32_t* n_row;    // [R] candidate count per row (prefix [0, n))
+    int n_row_div;           // n_row[r] is divided by this (rounded up): 8 for pool blocks
+    const int32_t* ids;      // [R][ld] ids (gather mode), or null: id = position
+    const int32_t* id_limit; // [R] ids must be < id_limit[r] (gather mode)
+    const uint32_t* hist;    // [R][4096] histogram of key >> 20
+    int32_t* out;            // [R][K] (or [R][K*8] with expand8)
+    bool expand8;            // output = 8 positions per picked block, < n_row[r]
+    const int32_t* expand_limit; // [R] visible positions for expand8
+    uint32_t* counters;      // [R][4]
+    uint64_t* winners;       // [R][K]
+    uint64_t* cands;         // [R][ccap]
+    int ccap;
+    int32_t* status;
+};
+
+cudaError_t launch_topk(const TopkLaunch& a, cudaStream_t st);
+
+struct AttnLaunch {
+    int Q;                   // query rows (B for decode, B*T for prefill)
+    int T;                   // tokens per sequence (1 for decode)
+    int H;
+    const void* q;           // bf16 [Q][H][512]
+    const uint8_t* codes;    // [B][cap][256]
+    const uint8_t* scales;   // [B][cap][32]
+    int64_t cap;
+    const int32_t* idx;      // [Q][K]
+    int K;
+    const uint8_t* swa;      // decode [B][W][512]; prefill [B][W-1+T][512]
+    int W;
+    const int32_t* swa_valid;  // decode, nullable
+    const int32_t* q_pos0;     // prefill, nullable
+    bool prefill;
+    float scale;
+    float* out;              // [Q][H][512]
+    float* partial;          // workspace for split rows
+    int nsplit;
+    int32_t* status;
+};
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+int attention_splits(int Q, int K, int W, bool prefill);
+
+int device_sm_count();
+
+}  // namespace csa2

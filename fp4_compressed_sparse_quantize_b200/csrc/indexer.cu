@@ -1,0 +1,626 @@
+// Indexer scoring on the 5th-generation tensor cores (tcgen05), fused with the first
+// radix-select histogram of the exact Top-K and with the candidate-pool block maxima.
+//
+// "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression" (AI summary),
+// Methodology in Plain English: Full layers score every causally visible compressed entry
+// with their own indexer query; Reindex layers rescore the latest Full layer's indexer keys
+// with their own query but only inside the candidate pool; the first decoder Full layer
+// also keeps the blocks with the highest maximum score ("2,048 blocks of 8 positions").
+// "DeepSeek-V4.1-Flash: A New Era in Efficient Large-Scale LLM Serving", Compressed
+// Sparse Attention 2 (CSA2): Full / Reindex / Reuse modes, Top-512.
+//
+// Score (reading adopted; the pages print no formula):
+//     s[r, j] = sum_{h < H_I} w[r, h] * max(0, <q_I[r, h, :], k_I[j, :]>)
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      producer: TMA tiles of 128 indexer keys (contiguous, 128-byte swizzle) into
+//               an S-stage ring; in gather mode (Reindex) cp.async of the pool's rows into
+//               the same swizzled layout; plus the query-group operand per row group.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128 keys,
+//               N = G queries x H_I heads, K = 128 channels) into a TMEM accumulator ring.
+//   warps 2..5  epilogue: tcgen05.ld of one key row per thread, ReLU-weighted head sum in
+//               fp32, coalesced score stores, shared-memory histogram of the top 12 key
+//               bits per query row (first radix-select digit), 8-entry block maxima.
+// Every wait is bounded (2 s) and sets CSA2_DEV_TIMEOUT instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "csa2_common.cuh"
+#include "csa2_internal.h"
+
+namespace csa2 {
+
+constexpr int kTileRows = 128;  // keys per tile (MMA M, TMEM lanes)
+constexpr int kBins = 4096;     // first radix digit: key >> 20
+
+struct ScanParams {
+    int rows;               // query rows R (B*T)
+    int G;                  // query rows per row group (they share a key tile)
+    int T;                  // query rows per sequence
+    int H_I;
+    int64_t cap;            // key capacity per sequence
+    const int32_t* n_row;   // [R] visible entries per query row (clamped)
+    const int64_t* prefix;  // [R/G + 1] exclusive prefix of tiles per row group
+    const float* w;         // [R][H_I]
+    float* scores;          // [R][ld_scores]
+    int64_t ld_scores;
+    uint32_t* hist;         // [R][kBins]
+    uint32_t* bkey;         // [R][ld_bkey] block-max keys, or null
+    int64_t ld_bkey;
+    uint32_t* bhist;        // [R][kBins] or null
+    const int32_t* pool;    // gather mode: [R][P] positions, -1 = empty
+    int P;
+    const uint8_t* keys;    // gather mode: raw key base (row-major [B*cap][128*esize])
+    int32_t* status;
+};
+
+// ---- shared memory plan ----------------------------------------------------------------
+template <int NQ, int ESZ, int STAGES, int ACC, int G>
+struct ScanSmem {
+    static constexpr int kTileBytes = kTileRows * 128 * ESZ;
+    static constexpr int kQBytes = NQ * 128 * ESZ;
+    static constexpr int kStageOff = 0;
+    static constexpr int kQOff = kStageOff + STAGES * kTileBytes;
+    static constexpr int kHistOff = kQOff + 2 * kQBytes;
+    static constexpr int kBHistOff = kHistOff + G * kBins * 4;
+    static constexpr int kWOff = kBHistOff + kBins * 4;
+    static constexpr int kBarOff = kWOff + 2 * NQ * 4;
+    static constexpr int kNumBars = 2 * STAGES + 4 + 2 * ACC + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kBytes = kMiscOff + 64;
+    static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KiB alignment
+};
+
+__device__ __forceinline__ void epi_bar_sync() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Advance (b-group, tile) iteration state so that tile index t lies in row group g.
+__device__ __forceinline__ int find_group(const int64_t* prefix, int ngroups, int64_t t) {
+    int lo = 0, hi = ngroups - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= t)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// NQ   = MMA N: G * H_I rounded up to a multiple of 16 (padding rows are ignored)
+// ESZ  = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
+// GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
+template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL>
+__global__ void __launch_bounds__(192, 1)
+    scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G>;
+    constexpr int kKSteps = (128 * ESZ) / 32;        // 32 bytes of K per MMA instruction
+    constexpr uint32_t kHalf = kTileRows * 128;      // bytes of one 128-byte-wide K slab
+    constexpr uint32_t kQHalf = NQ * 128;
+    constexpr uint32_t kAccCols = NQ;
+    constexpr uint32_t kTmemCols = (ACC * NQ <= 32) ? 32 : (ACC * NQ <= 64) ? 64
+                                 : (ACC * NQ <= 128) ? 128 : (ACC * NQ <= 256) ? 256 : 512;
+    constexpr uint32_t kIdesc = make_idesc(128, NQ, ESZ == 2 ? 1u : 0u, ESZ == 2 ? 1u : 0u);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* stage_base = smem + L::kStageOff;
+    uint8_t* q_base = smem + L::kQOff;
+    uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
+    uint32_t* bhist_s = reinterpret_cast<uint32_t*>(smem + L::kBHistOff);
+    float* w_s = reinterpret_cast<float*>(smem + L::kWOff);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* qfull = bars + 2 * STAGES;
+    uint64_t* qempty = qfull + 2;
+    uint64_t* accfull = qempty + 2;
+    uint64_t* accempty = accfull + ACC;
+    uint64_t* done_bar = accempty + ACC;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int ngroups = p.rows / G;
+    const int64_t total = __ldg(p.prefix + ngroups);
+    const int64_t t0 = total * blockIdx.x / gridDim.x;
+    const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+    if (t0 >= t1) return;  // uniform across the CTA
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], GATHER ? 1 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&qempty[s], 1);
+        }
+        for (int s = 0; s < ACC; ++s) {
+            mbar_init(&accfull[s], 1);
+            mbar_init(&accempty[s], 4);
+        }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp >= 2) {
+        for (int i = threadIdx.x - 64; i < G * kBins; i += 128) hist_s[i] = 0;
+        if (POOL)
+            for (int i = threadIdx.x - 64; i < kBins; i += 128) bhist_s[i] = 0;
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+    if (warp == 0 && lane == 0 && !GATHER) {
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_q);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int g = find_group(p.prefix, ngroups, t0);
+        int qg = -1, qcount = 0;
+        int64_t it = 0;
+        const uint64_t policy = l2_policy_evict_first();
+        for (int64_t t = t0; t < t1; ++t, ++it) {
+            if (*abort_flag) break;
+            while (t >= __ldg(p.prefix + g + 1)) ++g;
+            const int64_t jt = t - __ldg(p.prefix + g);
+            const int r0 = g * G;
+            const int b = r0 / p.T;
+            if (g != qg) {
+                const int qs = qcount & 1;
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&qempty[qs], ((qcount >> 1) & 1) ^ 1, p.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) { if (lane == 0) *abort_flag = 1; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&qfull[qs], 2 * 0 + (uint32_t)L::kQBytes);
+                    uint8_t* dst = q_base + qs * L::kQBytes;
+                    for (int h = 0; h < ESZ; ++h)
+                        tma_load_2d(dst + h * kQHalf, &tmap_q, &qfull[qs], h * 64 * (ESZ == 2),
+                                    r0 * p.H_I);
+                }
+                qg = g;
+                ++qcount;
+            }
+            const int s = (int)(it % STAGES);
+            const uint32_t round = (uint32_t)(it / STAGES);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&empty[s], (round & 1) ^ 1, p.status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { if (lane == 0) *abort_flag = 1; break; }
+            uint8_t* dst = stage_base + s * L::kTileBytes;
+            if (!GATHER) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)L::kTileBytes);
+                    const int64_t row = (int64_t)b * p.cap + jt * kTileRows;
+                    for (int h = 0; h < ESZ; ++h)
+                        tma_load_2d_hint(dst + h * kHalf, &tmap_k, &full[s], h * 64 * (ESZ == 2),
+                                         (int32_t)row, policy);
+                }
+            } else {
+                // pool rows of query row r0 (G == 1 in gather mode)
+                const int32_t* pl = p.pool + (int64_t)r0 * p.P + jt * kTileRows;
+                const int n_vis = __ldg(p.n_row + r0);
+                const uint32_t dst_u = smem_u32(dst);
+                for (int rr = 0; rr < kTileRows; rr += 4) {
+                    const int rl = rr + (lane >> 3);       // 4 rows per pass, 8 lanes per row
+                    const int64_t slot = jt * kTileRows + rl;
+                    int pos = (slot < p.P) ? __ldg(pl + rl) : -1;
+                    if (pos >= n_vis) pos = -1;
+                    if (pos >= 0) {
+                        const uint8_t* src = p.keys + ((int64_t)b * p.cap + pos) * (128 * ESZ);
+                        for (int h = 0; h < ESZ; ++h) {
+                            const int c = lane & 7;         // 16-byte chunk within 128 bytes
+                            const uint32_t off = h * kHalf + rl * 128 + ((c ^ (rl & 7)) << 4);
+                            cp_async16(dst_u + off, src + h * 128 + c * 16);
+                        }
+                    }
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
+            }
+        }
+        // Drain: every TMA issued into this CTA's shared memory must land before exit.
+        if (!GATHER && lane == 0) {
+            const int64_t n_issued = it;
+            for (int64_t k = (n_issued > STAGES ? n_issued - STAGES : 0); k < n_issued; ++k)
+                mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), p.status);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int g = find_group(p.prefix, ngroups, t0);
+            int qg = -1, qcount = 0, qs = 0;
+            int64_t it = 0;
+            for (int64_t t = t0; t < t1; ++t, ++it) {
+                if (*abort_flag) break;
+                while (t >= __ldg(p.prefix + g + 1)) ++g;
+                if (g != qg) {
+                    if (qg >= 0) mma_commit(&qempty[qs]);
+                    qs = qcount & 1;
+                    if (!mbar_wait(&qfull[qs], (qcount >> 1) & 1, p.status)) { *abort_flag = 1; break; }
+                    qg = g;
+                    ++qcount;
+                }
+                const int s = (int)(it % STAGES);
+                if (!mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), p.status)) { *abort_flag = 1; break; }
+                const int a = (int)(it % ACC);
+                if (!mbar_wait(&accempty[a], (uint32_t)(((it / ACC) & 1) ^ 1), p.status)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + a * kAccCols;
+                const uint32_t a_addr = smem_u32(stage_base + s * L::kTileBytes);
+                const uint32_t b_addr = smem_u32(q_base + qs * L::kQBytes);
+#pragma unroll
+                for (int kk = 0; kk < kKSteps; ++kk) {
+                    const uint32_t koff = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    const uint32_t qoff = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                    const uint64_t ad = sw128_desc(a_addr + koff, 16, 1024);
+                    const uint64_t bd = sw128_desc(b_addr + qoff, 16, 1024);
+                    if (ESZ == 1)
+                        mma_f8(d, ad, bd, kIdesc, kk > 0);
+                    else
+                        mma_f16(d, ad, bd, kIdesc, kk > 0);
+                }
+                mma_commit(&empty[s]);
+                mma_commit(&accfull[a]);
+            }
+            // all MMAs must complete before TMEM is released
+            mma_commit(done_bar);
+            mbar_wait(done_bar, 0, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (128 thr)
+        const int et = threadIdx.x - 64;           // 0..127
+        const int row = 32 * (warp & 3) + lane;    // TMEM lane == key row within the tile
+        const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+        int g = find_group(p.prefix, ngroups, t0);
+        int cur = -1, wslot = 0;
+        int64_t it = 0;
+        bool aborted = false;
+        for (int64_t t = t0; t < t1; ++t, ++it) {
+            while (t >= __ldg(p.prefix + g + 1)) ++g;
+            const int64_t jt = t - __ldg(p.prefix + g);
+            const int r0 = g * G;
+            if (g != cur) {
+                // flush the previous row group's histograms, then load the new weights
+                epi_bar_sync();
+                if (cur >= 0) {
+                    for (int gg = 0; gg < G; ++gg)
+                        for (int i = et; i < kBins; i += 128) {
+                            const uint32_t v = hist_s[gg * kBins + i];
+                            if (v) {
+                                atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
+                                hist_s[gg * kBins + i] = 0;
+                            }
+                        }
+                    if (POOL)
+                        for (int i = et; i < kBins; i += 128) {
+                            const uint32_t v = bhist_s[i];
+                            if (v) {
+                                atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
+                                bhist_s[i] = 0;
+                            }
+                        }
+                }
+                wslot ^= 1;
+                for (int i = et; i < NQ; i += 128)
+                    w_s[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
+                epi_bar_sync();
+                cur = g;
+            }
+            const int a = (int)(it % ACC);
+            aborted = aborted || *abort_flag;
+            if (!aborted) {
+                if (!mbar_wait(&accfull[a], (uint32_t)((it / ACC) & 1), p.status)) {
+                    aborted = true;
+                    *abort_flag = 1;
+                }
+            }
+            if (aborted) continue;
+            tc_fence_after();
+            float sc[G];
+            const float* wv = w_s + wslot * NQ;
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg) {
+                float s = 0.f;
+                int h0 = gg * p.H_I;
+                // columns [h0, h0 + H_I) of this accumulator, loaded 16 at a time
+                for (int c0 = (h0 & ~15); c0 < h0 + p.H_I; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_base + lane_addr + a * kAccCols + c0, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int h = c0 + k;
+                        if (h >= h0 && h < h0 + p.H_I)
+                            s = fmaf(wv[h], fmaxf(__uint_as_float(v[k]), 0.f), s);
+                    }
+                }
+                sc[gg] = s + 0.0f;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[a]);
+
+            const int64_t j = jt * kTileRows + row;   // entry (or pool slot) index
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg) {
+                const int r = r0 + gg;
+                bool vis;
+                if (!GATHER) {
+                    vis = j < __ldg(p.n_row + r);
+                } else {
+                    int pos = (j < p.P) ? __ldg(p.pool + (int64_t)r * p.P + j) : -1;
+                    vis = pos >= 0 && pos < __ldg(p.n_row + r);
+                }
+                const uint32_t key = score_key(sc[gg]);
+                if (vis) {
+                    p.scores[(int64_t)r * p.ld_scores + j] = sc[gg];
+                    atomicAdd(&hist_s[gg * kBins + (key >> 20)], 1u);
+                }
+                if (POOL) {
+                    uint32_t bk = vis ? key : 0u;
+                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
+                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
+                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
+                    if ((row & 7) == 0 && j < __ldg(p.n_row + r)) {
+                        p.bkey[(int64_t)r * p.ld_bkey + (j >> 3)] = bk;
+                        atomicAdd(&bhist_s[bk >> 20], 1u);
+                    }
+                }
+            }
+        }
+        // final flush
+        epi_bar_sync();
+        if (cur >= 0) {
+            for (int gg = 0; gg < G; ++gg)
+                for (int i = et; i < kBins; i += 128) {
+                    const uint32_t v = hist_s[gg * kBins + i];
+                    if (v) atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
+                }
+            if (POOL)
+                for (int i = et; i < kBins; i += 128) {
+                    const uint32_t v = bhist_s[i];
+                    if (v) atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
+                }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---- per-row visible counts and tile prefix ---------------------------------------------
+// decode: n_row[r] = n_vis0[r]; prefill: n_row[b*T+t] = floor((q_pos0[b]+t+1)/ratio).
+// Counts are clamped to [0, cap] (CSA2_DEV_BAD_COUNT when clamping was needed); gather
+// mode counts pool slots instead of entries for the tile prefix.
+__global__ void __launch_bounds__(1024) prep_rows_kernel(
+    int rows, int T, int G, const int32_t* n_vis0, const int32_t* q_pos0, int ratio,
+    int64_t cap, int P_gather, int32_t* n_row, int64_t* prefix, int32_t* status) {
+    __shared__ int64_t warp_sums[32];
+    __shared__ int64_t carry;
+    if (threadIdx.x == 0) carry = 0;
+    const int ngroups = rows / G;
+    for (int base = 0; base < rows; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        if (r < rows) {
+            int64_t n;
+            if (q_pos0) {
+                const int b = r / T, t = r - b * T;
+                n = ((int64_t)__ldg(q_pos0 + b) + t + 1) / ratio;
+            } else {
+                n = __ldg(n_vis0 + r);
+            }
+            if (n < 0 || n > cap) {
+                set_status(status, CSA2_DEV_BAD_COUNT);
+                n = n < 0 ? 0 : cap;
+            }
+            n_row[r] = (int32_t)n;
+        }
+    }
+    __syncthreads();
+    for (int base = 0; base < ngroups; base += blockDim.x) {
+        const int gi = base + threadIdx.x;
+        int64_t tiles = 0;
+        if (gi < ngroups) {
+            const int64_t n = P_gather > 0 ? P_gather : n_row[gi * G + G - 1];
+            tiles = (n + kTileRows - 1) / kTileRows;
+        }
+        // block-wide exclusive scan of `tiles`
+        int64_t v = tiles;
+        for (int o = 1; o < 32; o <<= 1) {
+            int64_t u = __shfl_up_sync(0xffffffffu, v, o);
+            if ((threadIdx.x & 31) >= o) v += u;
+        }
+        if ((threadIdx.x & 31) == 31) warp_sums[threadIdx.x >> 5] = v;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            int64_t ws = warp_sums[threadIdx.x];
+            for (int o = 1; o < 32; o <<= 1) {
+                int64_t u = __shfl_up_sync(0xffffffffu, ws, o);
+                if (threadIdx.x >= o) ws += u;
+            }
+            warp_sums[threadIdx.x] = ws;
+        }
+        __syncthreads();
+        const int64_t before = carry + (threadIdx.x >= 32 ? warp_sums[(threadIdx.x >> 5) - 1] : 0) +
+                               v - tiles;
+        if (gi < ngroups) prefix[gi] = before;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = before + tiles;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) prefix[ngroups] = carry;
+}
+
+// ---- host side -------------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over a [rows][row_bytes] byte matrix, box = 128 bytes x box_rows, 128B swizzle.
+static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int esz, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const CUtensorMapDataType dt =
+        esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    cuuint64_t dims[2] = {(cuuint64_t)128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(128 * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL>
+static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
+                                 const ScanParams& p, cudaStream_t st) {
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G>;
+    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::kAlloc);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms(), 192, L::kAlloc, st>>>(mk, mq, p);
+    return cudaGetLastError();
+}
+
+// Dispatch on (padded query columns, element size, group size, mode).
+cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
+    const int esz = a.esz;
+    const int NQreq = a.G * a.H_I;
+    int NQ = (NQreq + 15) & ~15;
+    CUtensorMap mk, mq;
+    memset(&mk, 0, sizeof mk);
+    memset(&mq, 0, sizeof mq);
+    if (!make_map(&mq, a.q, (int64_t)a.rows * a.H_I, esz, NQ)) return cudaErrorInvalidValue;
+    if (!a.gather && !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, kTileRows))
+        return cudaErrorInvalidValue;
+    ScanParams p;
+    p.rows = a.rows;
+    p.G = a.G;
+    p.T = a.T;
+    p.H_I = a.H_I;
+    p.cap = a.cap;
+    p.n_row = a.n_row;
+    p.prefix = a.prefix;
+    p.w = a.w;
+    p.scores = a.scores;
+    p.ld_scores = a.ld_scores;
+    p.hist = a.hist;
+    p.bkey = a.bkey;
+    p.ld_bkey = a.ld_bkey;
+    p.bhist = a.bhist;
+    p.pool = a.pool;
+    p.P = a.P;
+    p.keys = reinterpret_cast<const uint8_t*>(a.k);
+    p.status = a.status;
+
+#define CSA2_SCAN(NQv, ESZv, STv, ACCv, Gv, GA, PO) \
+    return launch_scan_t<NQv, ESZv, STv, ACCv, Gv, GA, PO>(mk, mq, p, st)
+
+    if (a.G == 1) {
+        if (a.gather) {
+            if (esz == 1) {
+                if (NQ <= 32) CSA2_SCAN(32, 1, 4, 4, 1, true, false);
+                if (NQ <= 64) CSA2_SCAN(64, 1, 4, 4, 1, true, false);
+                CSA2_SCAN(128, 1, 4, 2, 1, true, false);
+            } else {
+                if (NQ <= 32) CSA2_SCAN(32, 2, 2, 4, 1, true, false);
+                if (NQ <= 64) CSA2_SCAN(64, 2, 2, 4, 1, true, false);
+                CSA2_SCAN(128, 2, 2, 2, 1, true, false);
+            }
+        }
+        if (esz == 1) {
+            if (a.pool_build) {
+                if (NQ <= 16) CSA2_SCAN(16, 1, 8, 4, 1, false, true);
+                if (NQ <= 32) CSA2_SCAN(32, 1, 8, 4, 1, false, true);
+                if (NQ <= 64) CSA2_SCAN(64, 1, 8, 4, 1, false, true);
+                CSA2_SCAN(128, 1, 6, 2, 1, false, true);
+            }
+            if (NQ <= 16) CSA2_SCAN(16, 1, 8, 4, 1, false, false);
+            if (NQ <= 32) CSA2_SCAN(32, 1, 8, 4, 1, false, false);
+            if (NQ <= 64) CSA2_SCAN(64, 1, 8, 4, 1, false, false);
+            CSA2_SCAN(128, 1, 6, 2, 1, false, false);
+        } else {
+            if (a.pool_build) {
+                if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, true);
+                if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, true);
+                if (NQ <= 64) CSA2_SCAN(64, 2, 4, 4, 1, false, true);
+                CSA2_SCAN(128, 2, 3, 2, 1, false, true);
+            }
+            if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, false);
+            if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, false);
+            if (NQ <= 64) CSA2_SCAN(64, 2, 4, 4, 1, false, false);
+            CSA2_SCAN(128, 2, 3, 2, 1, false, false);
+        }
+    } else if (a.G == 4 && NQ == 256 && esz == 1 && !a.gather && !a.pool_build) {
+        CSA2_SCAN(256, 1, 4, 2, 4, false, false);
+    } else if (a.G == 2 && NQ <= 128 && esz == 1 && !a.gather && !a.pool_build) {
+        CSA2_SCAN(128, 1, 6, 2, 2, false, false);
+    }
+#undef CSA2_SCAN
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
+                             const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
+                             int32_t* n_row, int64_t* prefix, int32_t* status,
+                             cudaStream_t st) {
+    prep_rows_kernel<<<1, 1024, 0, st>>>(rows, T, G, n_vis0, q_pos0, ratio, cap, P_gather,
+                                         n_row, prefix, status);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,98 @@
+// FP4 quantize-on-write of main-KV entries.
+//
+// "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression" (AI summary), Main
+// Findings, FP4 format choice; "DeepSeek-V4.1-Flash: A New Era in Efficient Large-Scale
+// LLM Serving", Quantization and Memory Management: E2M1 elements, one E4M3 scale per
+// 16 channels, NVFP4 without the second-level global scale.
+//
+// One warp per 512-channel entry: lane l owns channels [16l, 16l+16), i.e. exactly one
+// scale block. Loads are two 16-byte vectors per lane (a warp reads the 1 KiB row in one
+// coalesced sweep); stores are 8 code bytes and 1 scale byte per lane (256 + 32 B per
+// warp, contiguous). The work is trivially HBM-bound (1 KiB in, 288 B out per entry).
+//
+// Rounding: the scale is E4M3(amax / 6) and each magnitude is E2M1(|x| / s), both with
+// round-to-nearest-even and saturation (cvt.rn.satfinite), where the quotients are IEEE
+// fp32 divisions. Neither quotient can land on a rounding midpoint unless the exact
+// quotient does: the numerator has 8 significant bits and the divisor (6, or an E4M3
+// value with at most 4) leaves a non-dyadic quotient far from every dyadic midpoint, and
+// a dyadic quotient is exact in fp32. A reciprocal-multiply would not have that property.
+#include "csa2_common.cuh"
+
+namespace csa2 {
+
+__global__ void __launch_bounds__(256) quantize_kv_kernel(
+    const __nv_bfloat16* __restrict__ kv, int B, int n_new, int64_t ld_kv, int64_t bstride_kv,
+    const int32_t* __restrict__ dst_off, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, int64_t cap, int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t entry = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (entry >= (int64_t)B * n_new) return;
+    const int b = (int)(entry / n_new);
+    const int i = (int)(entry - (int64_t)b * n_new);
+    const int64_t dst = (int64_t)__ldg(dst_off + b) + i;
+    if (dst < 0 || dst >= cap) {
+        if (lane == 0) set_status(status, CSA2_DEV_BAD_INDEX);
+        return;
+    }
+    const __nv_bfloat16* row = kv + (int64_t)b * bstride_kv + (int64_t)i * ld_kv + lane * 16;
+    uint4 v0 = __ldg(reinterpret_cast<const uint4*>(row));
+    uint4 v1 = __ldg(reinterpret_cast<const uint4*>(row) + 1);
+    uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float x[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        x[2 * k] = __uint_as_float(w[k] << 16);
+        x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
+
+    // scale code: E4M3(amax / 6), RNE, saturating
+    const float q = __fdiv_rn(amax, 6.0f);
+    uint16_t sc2;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sc2) : "f"(0.0f), "f"(q));
+    const uint8_t sc = (uint8_t)(sc2 & 0xFF);
+    const float s = e4m3_to_float(sc);
+
+    uint32_t packed_lo = 0, packed_hi = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        // channel 2k -> low nibble, 2k+1 -> high nibble
+        const float a = (s > 0.f) ? __fdiv_rn(fabsf(x[2 * k]), s) : 0.f;
+        const float c = (s > 0.f) ? __fdiv_rn(fabsf(x[2 * k + 1]), s) : 0.f;
+        uint16_t byte;
+        asm("{\n\t.reg .b8 t;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+            "cvt.u16.u8 %0, t;\n\t}"
+            : "=h"(byte)
+            : "f"(c), "f"(a));
+        uint32_t bb = byte & 0x77u;  // magnitudes only
+        bb |= (__float_as_uint(x[2 * k]) >> 31) << 3;
+        bb |= (__float_as_uint(x[2 * k + 1]) >> 31) << 7;
+        if (k < 4)
+            packed_lo |= bb << (8 * k);
+        else
+            packed_hi |= bb << (8 * (k - 4));
+    }
+    const int64_t e = (int64_t)b * cap + dst;
+    reinterpret_cast<uint2*>(codes + e * CSA2_ENTRY_CODE_BYTES)[lane] =
+        make_uint2(packed_lo, packed_hi);
+    scales[e * CSA2_ENTRY_SCALE_BYTES + lane] = sc;
+}
+
+cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
+                               int64_t bstride_kv, const int32_t* dst_off, uint8_t* codes,
+                               uint8_t* scales, int64_t cap, int32_t* status,
+                               cudaStream_t stream) {
+    const int64_t entries = (int64_t)B * n_new;
+    if (entries == 0) return cudaSuccess;
+    const int warps = 8;
+    const int64_t grid = (entries + warps - 1) / warps;
+    quantize_kv_kernel<<<(unsigned)grid, warps * 32, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(kv), B, n_new, ld_kv, bstride_kv, dst_off, codes,
+        scales, cap, status);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

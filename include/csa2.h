@@ -1,0 +1,241 @@
+/*
+ * csa2.h — C ABI of libcsa2: CSA2 compressed sparse attention over an FP4 main-KV cache,
+ * hand-written for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are web pages about the DeepSeek-V4.1-Flash
+ * report; each entry point cites the passage that defines its operation):
+ *   [AIS] "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression" (ai.info
+ *         AI summary): "Main Findings" (FP4 format choice), "Methodology in Plain
+ *         English" (CSA2 modes, Hierarchical Sparse Indexer, indexer K).
+ *   [TDG] "DeepSeek-V4.1-Flash: A New Era in Efficient Large-Scale LLM Serving":
+ *         "Compressed Sparse Attention 2 (CSA2)", "Quantization and Memory
+ *         Management", "Causal Encoder-Decoder" (128-token SWA in every layer).
+ *   [TLB] "DeepSeek V4.1 Flash: smaller KV cache, same post-training": "How did
+ *         DeepSeek V4.1 reduce the KV cache?" (three modes, FP4 KV cache, SWA).
+ *
+ * Conventions for every entry point
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise. The caller
+ *     owns all memory; the library never allocates device memory. Scratch space comes
+ *     from a caller-supplied workspace sized by csa2_workspace_bytes().
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and returns before the device work finishes.
+ *   - Row-major layouts, last dimension contiguous. Pointers to codes, scales, keys,
+ *     queries, window rows and outputs must be 16-byte aligned.
+ *   - Argument errors are reported as CSA2_ERR_ARG / CSA2_ERR_UNSUPPORTED /
+ *     CSA2_ERR_WORKSPACE before anything is launched. Launch failures return
+ *     CSA2_ERR_CUDA. Errors found on the device (an index outside its buffer, a
+ *     visible count above the capacity, a bounded wait that ran out) never fault: the
+ *     offending item is skipped and a bit is OR-ed into the device status word that
+ *     lives in the first 4 bytes of the workspace; read it with
+ *     csa2_read_device_status(). The status word is sticky until
+ *     csa2_reset_device_status() clears it. A workspace must be zero-filled (or reset)
+ *     once before first use.
+ *   - The library keeps no global mutable state; calls on different streams with
+ *     different workspaces may run concurrently. Calls that share a workspace must be
+ *     ordered (same stream).
+ *   - Fixed geometry: main-KV latent D = 512 channels, indexer dimension 128, candidate
+ *     pool blocks of 8 positions. Other sizes return CSA2_ERR_UNSUPPORTED.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa2_status {
+    CSA2_OK = 0,
+    CSA2_ERR_ARG = 1,          /* null pointer, bad size, misalignment, mode/pool mismatch */
+    CSA2_ERR_UNSUPPORTED = 2,  /* geometry or dtype not built */
+    CSA2_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed */
+    CSA2_ERR_WORKSPACE = 4,    /* workspace missing or smaller than csa2_workspace_bytes() */
+    CSA2_ERR_DEVICE = 5        /* csa2_read_device_status() found a non-zero status word */
+} csa2_status_t;
+
+/* Per-layer CSA2 mode [AIS Methodology], [TDG CSA2], [TLB three modes]. */
+typedef enum csa2_mode {
+    CSA2_MODE_FULL = 0,    /* score every visible entry, pick fresh Top-K (and the pool) */
+    CSA2_MODE_REINDEX = 1, /* rescore only the candidate pool of the latest Full layer   */
+    CSA2_MODE_REUSE = 2    /* no indexer work: the earlier layer's indices are reused     */
+} csa2_mode_t;
+
+/* Storage type of the indexer query and key. */
+typedef enum csa2_dtype {
+    CSA2_DTYPE_BF16 = 0,
+    CSA2_DTYPE_E4M3 = 1    /* OCP FP8 E4M3 ("fn": no infinities, max 448) */
+} csa2_dtype_t;
+
+/* Operations that need a workspace. */
+typedef enum csa2_op {
+    CSA2_OP_INDEX_SCORE_TOPK = 0,
+    CSA2_OP_SPARSE_ATTN_DECODE = 1,
+    CSA2_OP_SPARSE_ATTN_PREFILL = 2
+} csa2_op_t;
+
+/* Bits of the device status word. */
+#define CSA2_DEV_BAD_INDEX   0x1  /* an index / offset pointed outside its buffer       */
+#define CSA2_DEV_BAD_COUNT   0x2  /* a visible count was negative or above capacity     */
+#define CSA2_DEV_TIMEOUT     0x4  /* a bounded wait inside a kernel gave up             */
+
+#define CSA2_D_MAIN 512           /* main-KV latent channels                            */
+#define CSA2_D_INDEX 128          /* indexer query / key channels                       */
+#define CSA2_SCALE_GROUP 16       /* channels per E4M3 scale                            */
+#define CSA2_ENTRY_CODE_BYTES 256 /* packed E2M1 bytes per main-KV entry (512 / 2)      */
+#define CSA2_ENTRY_SCALE_BYTES 32 /* E4M3 scale bytes per main-KV entry (512 / 16)      */
+#define CSA2_POOL_BLOCK 8         /* positions per candidate-pool block                 */
+
+/*
+ * csa2_quantize_kv — FP4 quantize-on-write of new main-KV entries.
+ * [AIS Main Findings, FP4 format choice], [TDG Quantization and Memory Management],
+ * [TLB FP4 KV cache]: E2M1 elements with one E4M3 scale per 16 channels (NVFP4 without
+ * its second-level global scale). Per 16-channel block: amax = max|x|; scale =
+ * E4M3(amax / 6) rounded to nearest-even and saturated at 448; each element code =
+ * E2M1(|x| / scale) rounded to nearest-even, saturated at 6, with the sign bit of x
+ * (a zero scale gives zero magnitudes). Quotients are IEEE-rounded fp32 divisions.
+ *
+ *   kv       bf16 [B][n_new][512]: element (b,i,c) at kv[b*bstride_kv + i*ld_kv + c]
+ *            (strides in elements; ld_kv >= 512, multiples of 8). Must be finite:
+ *            non-finite input gives unspecified codes.
+ *   dst_off  int32 [B]: entry index where sequence b's first new entry is written.
+ *   codes    uint8 [B][cap][256]: channel 2k in the low nibble of byte k.
+ *   scales   uint8 [B][cap][32]: E4M3 bit patterns, one per 16 channels.
+ * Entries outside [0, cap) are skipped and set CSA2_DEV_BAD_INDEX; with no workspace
+ * argument that bit goes to `status` (nullable int32 device word).
+ */
+CSA2_API csa2_status_t csa2_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
+                               int64_t bstride_kv, const int32_t* dst_off, uint8_t* codes,
+                               uint8_t* scales, int64_t cap, int32_t* status, void* stream);
+
+/*
+ * csa2_index_score_topk — indexer scoring + exact Top-K selection, per layer mode.
+ * [AIS Methodology]: each layer has its own indexer query; Full layers score, Reindex
+ * layers rescore the latest Full layer's keys, Reuse layers skip indexing; the first
+ * decoder Full layer scores the whole causally visible range and also keeps the blocks
+ * with the highest maximum score (e.g. 2,048 blocks of 8 = 16,384 positions) as a
+ * candidate pool that later Reindex layers search. [TDG CSA2]: Top-512.
+ * Score (the pages print no formula; reading adopted):
+ *     s[t,j] = sum_{h<H_I} w[t,h] * max(0, <q_I[t,h,:], k_I[j,:]>)
+ * computed with fp32 accumulation. Top-K key: (score descending, position ascending).
+ *
+ *   mode      FULL / REINDEX / REUSE. REUSE validates arguments and launches nothing.
+ *   B, T      sequences and query tokens per sequence (T = 1 for decode).
+ *   H_I       indexer heads, 1..128.
+ *   qk_dtype  storage type of q_I and k_I.
+ *   q_I       [B][T][H_I][128];  w  fp32 [B][T][H_I];  k_I  [B][cap][128].
+ *   n_vis0    int32 [B]: visible entries per sequence (decode, q_pos0 == NULL).
+ *   ratio, q_pos0
+ *             prefill visibility (q_pos0 != NULL): token t of sequence b sits at
+ *             position p = q_pos0[b] + t and sees entries j with (j+1)*ratio <= p+1,
+ *             i.e. N(t) = floor((p + 1) / ratio). Ignored when q_pos0 == NULL.
+ *   K         entries to select (1..2048).
+ *   pool_in   REINDEX only: int32 [B][T][P_in] candidate positions (-1 = empty slot);
+ *             must be non-NULL for REINDEX and NULL otherwise.
+ *   pool_out  FULL only, nullable: int32 [B][T][pool_blocks*8]: visible positions of the
+ *             pool_blocks blocks with the highest block maximum (ties: lower block),
+ *             ascending, padded with -1.
+ *   idx_out   int32 [B][T][K]: chosen positions in ascending order, padded with -1 when
+ *             fewer than K are visible.
+ *   scores_out nullable fp32 [B][T][cap] (FULL) or [B][T][P_in] (REINDEX): the scores;
+ *             entries not visible are left untouched.
+ *   ws, ws_bytes  workspace of at least csa2_workspace_bytes(CSA2_OP_INDEX_SCORE_TOPK,..).
+ */
+CSA2_API csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
+                                    csa2_dtype_t qk_dtype, const void* q_I, const float* w,
+                                    const void* k_I, int64_t cap, const int32_t* n_vis0,
+                                    int ratio, const int32_t* q_pos0, int K,
+                                    const int32_t* pool_in, int P_in, int32_t* pool_out,
+                                    int pool_blocks, int32_t* idx_out, float* scores_out,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * csa2_sparse_attn_decode — gather + dequantise the selected FP4 main-KV rows and
+ * attend over them together with the sliding-window rows.
+ * [AIS Methodology]: a compressed global branch plus a sliding-window local branch;
+ * every layer has its own query and window KV. [TDG Causal Encoder-Decoder, CSA2]:
+ * 128-token window in every layer. [AIS Main Findings]: window KV stays FP8.
+ * Reading adopted (pages silent): one softmax over the union of the K selected entries
+ * and the window rows, logits = scale * <q_h, x_i>, output sum_i p_i x_i (keys and values
+ * are the same latent row), no de-duplication and no sink; an empty row set gives 0.
+ *
+ *   mode      recorded and validated only: Full, Reindex and Reuse layers run the same
+ *             kernel (a Reuse layer passes the earlier layer's idx).
+ *   q         bf16 [B][H][512], H in 1..128.
+ *   codes, scales  main-KV cache as written by csa2_quantize_kv, capacity cap.
+ *   idx       int32 [B][K]; -1 entries are skipped; other entries outside [0, cap) are
+ *             skipped and set CSA2_DEV_BAD_INDEX.
+ *   swa       E4M3 [B][W][512]: the last W window rows, oldest first; W in 0..1024.
+ *   swa_valid nullable int32 [B]: only the last swa_valid[b] rows are used.
+ *   scale     logit multiplier (e.g. 1/sqrt(512)).
+ *   out       fp32 [B][H][512].
+ */
+CSA2_API csa2_status_t csa2_sparse_attn_decode(csa2_mode_t mode, int B, int H, const void* q,
+                                      const uint8_t* codes, const uint8_t* scales,
+                                      int64_t cap, const int32_t* idx, int K,
+                                      const uint8_t* swa, int W, const int32_t* swa_valid,
+                                      float scale, float* out, void* ws, size_t ws_bytes,
+                                      void* stream);
+
+/*
+ * csa2_sparse_attn_prefill — csa2_sparse_attn_decode for T new tokens per sequence,
+ * each with its own indices and a causal window ([TDG Causal Encoder-Decoder]).
+ *   q         bf16 [B][T][H][512];  idx  int32 [B][T][K].
+ *   swa       E4M3 [B][W-1+T][512]: row r holds position q_pos0[b] - (W-1) + r; token t
+ *             uses rows t .. t+W-1 (the last one is itself); rows whose position is
+ *             negative are skipped.
+ *   q_pos0    nullable int32 [B] (NULL: every row is valid).
+ *   out       fp32 [B][T][H][512].
+ */
+CSA2_API csa2_status_t csa2_sparse_attn_prefill(int B, int T, int H, const void* q,
+                                       const uint8_t* codes, const uint8_t* scales,
+                                       int64_t cap, const int32_t* idx, int K,
+                                       const uint8_t* swa, int W, const int32_t* q_pos0,
+                                       float scale, float* out, void* ws, size_t ws_bytes,
+                                       void* stream);
+
+/* Workspace bytes an operation needs (0 on invalid arguments).
+ *   CSA2_OP_INDEX_SCORE_TOPK: H = H_I; cap = cache capacity (Full) or P_in (Reindex);
+ *                             pool_blocks = 0 when no pool is built.
+ *   CSA2_OP_SPARSE_ATTN_*:    H = query heads; cap and pool_blocks are ignored.
+ * The size depends on the device's SM count for the decode attention (query rows are split
+ * across SMs), so query it on the device that will run the call. */
+CSA2_API size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t cap, int K,
+                            int pool_blocks);
+
+/* Static text for a status code. Never NULL. */
+CSA2_API const char* csa2_status_string(csa2_status_t status);
+
+/* Copy the device status word (first 4 bytes of `ws`, a device pointer) to *out (host)
+ * after synchronising `stream`. Returns CSA2_ERR_DEVICE when the word is non-zero. */
+CSA2_API csa2_status_t csa2_read_device_status(const void* ws, int32_t* out, void* stream);
+
+/* Clear the device status word (asynchronous on `stream`). */
+CSA2_API csa2_status_t csa2_reset_device_status(void* ws, void* stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+CSA2_API int csa2_version(void);
+
+/* Benchmark hook: when set, the next csa2_index_score_topk() issued from the calling host
+ * thread records `ev_start` (a cudaEvent_t passed as void*) on its stream right before
+ * its indexer-scan kernel launch and `ev_stop` right after it, then forgets both. The
+ * setting is per host thread and consumed by one call; NULL, NULL clears it. */
+CSA2_API csa2_status_t csa2_set_stage_events(void* ev_start, void* ev_stop);
+
+/* Test hook for the bounded waits: launches one block that waits on an mbarrier that is
+ * never signalled, gives up after timeout_ns and sets CSA2_DEV_TIMEOUT in `status`
+ * (device int32). Never faults or hangs. */
+CSA2_API csa2_status_t csa2_debug_bounded_wait(int32_t* status, uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */
