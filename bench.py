@@ -225,6 +225,25 @@ class Decode:
         return tot, scan
 
 
+def max_over_ranks(ms, pg, dev):
+    """Device-timed milliseconds of this rank -> the slowest rank's (every rank gets it)."""
+    if pg is None:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(batch_per_rank, world, steps, total_ms):
+    """Whole-job queries/s: every rank's queries over the slowest rank's time."""
+    return batch_per_rank * world * steps / (total_ms / 1e3)
+
+
+def rank_seed(seed, rank):
+    """Each rank draws its own independent batch."""
+    return seed + 7919 * rank
+
+
 def csa2_attn_splits(w):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     nch = (w.K + synth.WINDOW + 63) // 64
@@ -326,7 +345,7 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if w.kind != "decode":
         raise SystemExit("bench.py times the decode path; prefill is covered by the tests")
-    state = Decode(w, args.seed + 7919 * rank, dev)
+    state = Decode(w, rank_seed(args.seed, rank), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -341,6 +360,9 @@ def main():
           for _ in range(args.steps)]
     sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    for a, b in sev:           # torch creates the CUDA event on first record
+        a.record(stream)
+        b.record(stream)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
@@ -356,11 +378,7 @@ def main():
         pg.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     scan_ms = [a.elapsed_time(b) for a, b in sev]
-    total_ms = sum(step_ms)
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), pg, dev)
 
     # end-to-end: host inputs -> device -> step -> host output, through the public API
     ins = state.step_inputs()
@@ -381,11 +399,7 @@ def main():
             h.copy_(o, non_blocking=True)
         e2e_ev[k][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), pg, dev)
     st_i = csa2.read_device_status(state.ws_idx)
     st_a = csa2.read_device_status(state.ws_attn)
 
@@ -400,7 +414,7 @@ def main():
         alg_bytes, scan_bytes = state.algorithmic_bytes()
         per_step_ms = total_ms / args.steps
         queries = w.B * world * args.steps
-        value = queries / (total_ms / 1e3)
+        value = job_throughput(w.B, world, args.steps, total_ms)
         peak, src = peaks()
         scan_avg = sum(scan_ms) / len(scan_ms)
         achieved = scan_bytes / (scan_avg / 1e3) / 1e9

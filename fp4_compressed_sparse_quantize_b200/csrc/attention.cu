@@ -125,46 +125,57 @@ __global__ void __launch_bounds__(256, 1) attn_kernel(const AttnDev a) {
     const int c_end = min(a.nchunks, c_begin + a.chunks_per_split);
 
     // ---- query: per-head power-of-two rescale into fp16 ---------------------------------
-    for (int h = warp; h < kHP; h += 8) {
-        float v[16];
-        float amax = 0.f;
-        if (h < a.H) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                a.q + ((int64_t)qrow * a.H + h) * kDm + lane * 16);
-            uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-            uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                v[2 * k] = __uint_as_float(w8[k] << 16);
-                v[2 * k + 1] = __uint_as_float(w8[k] & 0xFFFF0000u);
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(v[k]));
-        } else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = 0.f;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        int shift = 0;
-        if (amax > 0.f) {
-            const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-            shift = min(126, max(-126, 14 - e));
-        }
-        const float mul = ldexpf(1.0f, shift);
-        uint32_t hw[8];
+    {
+        uint4 raw[8][2];   // the warp's 8 heads, all loads in flight before use
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            __half2 h2 = __floats2half2_rn(v[2 * k] * mul, v[2 * k + 1] * mul);
-            hw[k] = *reinterpret_cast<uint32_t*>(&h2);
+            const int h = warp + 8 * k;
+            if (h < a.H) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    a.q + ((int64_t)qrow * a.H + h) * kDm + lane * 16);
+                raw[k][0] = __ldg(src);
+                raw[k][1] = __ldg(src + 1);
+            } else {
+                raw[k][0] = raw[k][1] = make_uint4(0, 0, 0, 0);
+            }
         }
-        // lane owns channels [16 lane, 16 lane + 16) = chunks 2 lane, 2 lane + 1
-        uint32_t d0 = sQ + swz(h, 2 * lane, 1024), d1 = sQ + swz(h, 2 * lane + 1, 1024);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(d0), "r"(hw[0]), "r"(hw[1]),
-                     "r"(hw[2]), "r"(hw[3]));
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(d1), "r"(hw[4]), "r"(hw[5]),
-                     "r"(hw[6]), "r"(hw[7]));
-        if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * ldexpf(1.0f, -shift);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int h = warp + 8 * k;
+            float v[16];
+            const uint32_t w8[8] = {raw[k][0].x, raw[k][0].y, raw[k][0].z, raw[k][0].w,
+                                    raw[k][1].x, raw[k][1].y, raw[k][1].z, raw[k][1].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[2 * e] = __uint_as_float(w8[e] << 16);
+                v[2 * e + 1] = __uint_as_float(w8[e] & 0xFFFF0000u);
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            int shift = 0;
+            if (amax > 0.f) {
+                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                shift = min(126, max(-126, 14 - ex));
+            }
+            const float mul = ldexpf(1.0f, shift);
+            uint32_t hw[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                __half2 h2 = __floats2half2_rn(v[2 * e] * mul, v[2 * e + 1] * mul);
+                hw[e] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            // lane owns channels [16 lane, 16 lane + 16) = chunks 2 lane, 2 lane + 1
+            const uint32_t d0 = sQ + swz(h, 2 * lane, 1024), d1 = sQ + swz(h, 2 * lane + 1, 1024);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(d0), "r"(hw[0]),
+                         "r"(hw[1]), "r"(hw[2]), "r"(hw[3]));
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(d1), "r"(hw[4]),
+                         "r"(hw[5]), "r"(hw[6]), "r"(hw[7]));
+            if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * ldexpf(1.0f, -shift);
+        }
     }
 
     const int hg = warp & 3;       // head group: heads [16 hg, 16 hg + 16)
@@ -409,32 +420,48 @@ __global__ void __launch_bounds__(256, 1) attn_kernel(const AttnDev a) {
     }
 }
 
-// Merge the per-split partial results of each query row: out = sum_s 2^(m_s - M) O_s /
-// sum_s 2^(m_s - M) l_s (base-2 logits).
-__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ partial,
+// Merge the per-split partial results of one (query row, head): out = sum_s 2^(m_s - M)
+// O_s / sum_s 2^(m_s - M) l_s (base-2 logits). One CTA per (row, head), 4 channels/thread.
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ partial,
                                                            int nsplit, int H,
                                                            float* __restrict__ out) {
-    const int qrow = blockIdx.x;
+    __shared__ float wgt[64];
+    __shared__ float inv_s;
+    const int qrow = blockIdx.x, h = blockIdx.y;
     const int64_t stride = (int64_t)H * (kDm + 2);
     const float* base = partial + (int64_t)qrow * nsplit * stride;
-    for (int h = 0; h < H; ++h) {
-        float M = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * stride + (int64_t)H * kDm + h]);
-        const float Mb = (M == -INFINITY) ? 0.f : M;
-        float Ls = 0.f;
-        for (int s = 0; s < nsplit; ++s)
-            Ls += exp2f(base[s * stride + (int64_t)H * kDm + h] - Mb) *
-                  base[s * stride + (int64_t)H * kDm + H + h];
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        for (int c = threadIdx.x; c < kDm; c += blockDim.x) {
-            float acc = 0.f;
-            for (int s = 0; s < nsplit; ++s) {
-                const float wgt = exp2f(base[s * stride + (int64_t)H * kDm + h] - Mb);
-                acc += wgt * base[s * stride + (int64_t)h * kDm + c];
-            }
-            out[((int64_t)qrow * H + h) * kDm + c] = acc * inv;
+    if (threadIdx.x < 32) {
+        const int s = threadIdx.x;
+        float m = -INFINITY, l = 0.f;
+        if (s < nsplit) {
+            m = base[s * stride + (int64_t)H * kDm + h];
+            l = base[s * stride + (int64_t)H * kDm + H + h];
         }
+        float M = m;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float Mb = (M == -INFINITY) ? 0.f : M;
+        const float wv = (s < nsplit) ? exp2f(m - Mb) : 0.f;
+        float L = wv * l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (s < nsplit) wgt[s] = wv;
+        if (s == 0) inv_s = L > 0.f ? 1.f / L : 0.f;
     }
+    __syncthreads();
+    const int c = threadIdx.x * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < nsplit; ++s) {
+        const float4 v = *reinterpret_cast<const float4*>(base + s * stride + (int64_t)h * kDm + c);
+        const float wv = wgt[s];
+        acc.x += wv * v.x;
+        acc.y += wv * v.y;
+        acc.z += wv * v.z;
+        acc.w += wv * v.w;
+    }
+    const float inv = inv_s;
+    *reinterpret_cast<float4*>(out + ((int64_t)qrow * H + h) * kDm + c) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }
 
 int attention_splits(int Q, int K, int W, bool prefill) {
@@ -443,6 +470,7 @@ int attention_splits(int Q, int K, int W, bool prefill) {
     const int sms = device_sm_count();
     int ns = (2 * sms + Q - 1) / Q;
     if (ns > nchunks) ns = nchunks;
+    if (ns > 32) ns = 32;
     if (ns < 1) ns = 1;
     // equalise chunks per split
     const int cps = (nchunks + ns - 1) / ns;
@@ -481,7 +509,8 @@ cudaError_t launch_attention(const AttnLaunch& l, cudaStream_t st) {
     attn_kernel<<<grid, 256, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess || l.nsplit == 1) return e;
-    attn_combine_kernel<<<l.Q, 256, 0, st>>>(l.partial, l.nsplit, l.H, l.out);
+    attn_combine_kernel<<<dim3((unsigned)l.Q, (unsigned)l.H), 128, 0, st>>>(l.partial, l.nsplit,
+                                                                          l.H, l.out);
     return cudaGetLastError();
 }
 

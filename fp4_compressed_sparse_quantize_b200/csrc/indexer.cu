@@ -55,24 +55,25 @@ struct ScanParams {
 };
 
 // ---- shared memory plan ----------------------------------------------------------------
-template <int NQ, int ESZ, int STAGES, int ACC, int G>
+template <int NQ, int ESZ, int STAGES, int ACC, int G, int EPI, bool POOL>
 struct ScanSmem {
     static constexpr int kTileBytes = kTileRows * 128 * ESZ;
     static constexpr int kQBytes = NQ * 128 * ESZ;
     static constexpr int kStageOff = 0;
     static constexpr int kQOff = kStageOff + STAGES * kTileBytes;
     static constexpr int kHistOff = kQOff + 2 * kQBytes;
-    static constexpr int kBHistOff = kHistOff + G * kBins * 4;
-    static constexpr int kWOff = kBHistOff + kBins * 4;
-    static constexpr int kBarOff = kWOff + 2 * NQ * 4;
+    static constexpr int kBHistOff = kHistOff + EPI * G * kBins * 4;
+    static constexpr int kWOff = kBHistOff + (POOL ? EPI * kBins * 4 : 0);
+    static constexpr int kBarOff = kWOff + EPI * 2 * NQ * 4;
     static constexpr int kNumBars = 2 * STAGES + 4 + 2 * ACC + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1 KiB alignment
 };
 
-__device__ __forceinline__ void epi_bar_sync() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+// named barrier of one 128-thread epilogue group (ids 1.. ; 0 is __syncthreads)
+__device__ __forceinline__ void epi_bar_sync(int group) {
+    asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory");
 }
 
 // Advance (b-group, tile) iteration state so that tile index t lies in row group g.
@@ -105,11 +106,12 @@ __device__ __forceinline__ void fence_proxy_async() {
 // NQ   = MMA N: G * H_I rounded up to a multiple of 16 (padding rows are ignored)
 // ESZ  = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
 // GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
-template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL>
-__global__ void __launch_bounds__(192, 1)
+template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI>
+__global__ void __launch_bounds__(64 + 128 * EPI, 1)
     scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
-    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G>;
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL>;
+    static_assert(ACC % EPI == 0, "each epilogue group owns fixed accumulators");
     constexpr int kKSteps = (128 * ESZ) / 32;        // 32 bytes of K per MMA instruction
     constexpr uint32_t kHalf = kTileRows * 128;      // bytes of one 128-byte-wide K slab
     constexpr uint32_t kQHalf = NQ * 128;
@@ -163,9 +165,9 @@ __global__ void __launch_bounds__(192, 1)
         fence_mbar_init();
     }
     if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < G * kBins; i += 128) hist_s[i] = 0;
+        for (int i = threadIdx.x - 64; i < EPI * G * kBins; i += 128 * EPI) hist_s[i] = 0;
         if (POOL)
-            for (int i = threadIdx.x - 64; i < kBins; i += 128) bhist_s[i] = 0;
+            for (int i = threadIdx.x - 64; i < EPI * kBins; i += 128 * EPI) bhist_s[i] = 0;
     }
     if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
     if (warp == 0 && lane == 0 && !GATHER) {
@@ -296,43 +298,50 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue (128 thr)
-        const int et = threadIdx.x - 64;           // 0..127
-        const int row = 32 * (warp & 3) + lane;    // TMEM lane == key row within the tile
+        // ------------------------------------------------------------ epilogue groups
+        // EPI groups of 4 warps take alternate tiles (group e owns iterations it = e mod
+        // EPI and therefore TMEM accumulators a = it mod ACC of that residue), each with its
+        // own histograms, weights and named barrier.
+        const int e = (warp - 2) >> 2;
+        const int et = threadIdx.x - 64 - 128 * e;  // 0..127 within the group
+        const int row = 32 * (warp & 3) + lane;     // TMEM lane == key row within the tile
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+        uint32_t* hist_e = hist_s + e * G * kBins;
+        uint32_t* bhist_e = bhist_s + e * kBins;
+        float* w_e = w_s + e * 2 * NQ;
         int g = find_group(p.prefix, ngroups, t0);
         int cur = -1, wslot = 0;
-        int64_t it = 0;
         bool aborted = false;
-        for (int64_t t = t0; t < t1; ++t, ++it) {
+        for (int64_t it = e; t0 + it < t1; it += EPI) {
+            const int64_t t = t0 + it;
             while (t >= __ldg(p.prefix + g + 1)) ++g;
             const int64_t jt = t - __ldg(p.prefix + g);
             const int r0 = g * G;
             if (g != cur) {
                 // flush the previous row group's histograms, then load the new weights
-                epi_bar_sync();
+                epi_bar_sync(e);
                 if (cur >= 0) {
                     for (int gg = 0; gg < G; ++gg)
                         for (int i = et; i < kBins; i += 128) {
-                            const uint32_t v = hist_s[gg * kBins + i];
+                            const uint32_t v = hist_e[gg * kBins + i];
                             if (v) {
                                 atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
-                                hist_s[gg * kBins + i] = 0;
+                                hist_e[gg * kBins + i] = 0;
                             }
                         }
                     if (POOL)
                         for (int i = et; i < kBins; i += 128) {
-                            const uint32_t v = bhist_s[i];
+                            const uint32_t v = bhist_e[i];
                             if (v) {
                                 atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
-                                bhist_s[i] = 0;
+                                bhist_e[i] = 0;
                             }
                         }
                 }
                 wslot ^= 1;
                 for (int i = et; i < NQ; i += 128)
-                    w_s[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
-                epi_bar_sync();
+                    w_e[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
+                epi_bar_sync(e);
                 cur = g;
             }
             const int a = (int)(it % ACC);
@@ -346,24 +355,37 @@ __global__ void __launch_bounds__(192, 1)
             if (aborted) continue;
             tc_fence_after();
             float sc[G];
-            const float* wv = w_s + wslot * NQ;
+            const float* wv = w_e + wslot * NQ;
+            constexpr int kChunks = NQ / 16 / G;      // 16-column TMEM loads per query row
+            const int nch = (p.H_I + 15) >> 4;        // chunks actually holding heads
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) {
-                float s = 0.f;
-                int h0 = gg * p.H_I;
-                // columns [h0, h0 + H_I) of this accumulator, loaded 16 at a time
-                for (int c0 = (h0 & ~15); c0 < h0 + p.H_I; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem_base + lane_addr + a * kAccCols + c0, v);
-                    tmem_ld_wait();
+                // columns [gg*H_I, gg*H_I + H_I) of this accumulator; all loads in flight
+                // before one wait
+                uint32_t v[kChunks][16];
+                const uint32_t col = tmem_base + lane_addr + a * kAccCols + gg * p.H_I;
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int h = c0 + k;
-                        if (h >= h0 && h < h0 + p.H_I)
-                            s = fmaf(wv[h], fmaxf(__uint_as_float(v[k]), 0.f), s);
+                for (int c = 0; c < kChunks; ++c)
+                    if (c < nch) tmem_ld16(col + c * 16, v[c]);
+                tmem_ld_wait();
+                // four independent accumulation chains (heads h = 4m + j go to chain j)
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float* wg = wv + gg * p.H_I;
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    if (c < nch) {
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(wg + c * 16 + k4 * 4);
+                            // heads past H_I carry weight 0 (the weights are zero-padded)
+                            s4[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[c][4 * k4 + 0]), 0.f), s4[0]);
+                            s4[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[c][4 * k4 + 1]), 0.f), s4[1]);
+                            s4[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[c][4 * k4 + 2]), 0.f), s4[2]);
+                            s4[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[c][4 * k4 + 3]), 0.f), s4[3]);
+                        }
                     }
                 }
-                sc[gg] = s + 0.0f;
+                sc[gg] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + 0.0f;
             }
             tc_fence_before();
             __syncwarp();
@@ -381,33 +403,39 @@ __global__ void __launch_bounds__(192, 1)
                     vis = pos >= 0 && pos < __ldg(p.n_row + r);
                 }
                 const uint32_t key = score_key(sc[gg]);
-                if (vis) {
-                    p.scores[(int64_t)r * p.ld_scores + j] = sc[gg];
-                    atomicAdd(&hist_s[gg * kBins + (key >> 20)], 1u);
+                if (vis) p.scores[(int64_t)r * p.ld_scores + j] = sc[gg];
+                {
+                    // scores cluster in a few bins: one shared atomic per distinct bin
+                    const uint32_t bin = vis ? (key >> 20) : 0xFFFFFFFFu;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                    if (vis && (lane == __ffs(peers) - 1))
+                        atomicAdd(&hist_e[gg * kBins + bin], (uint32_t)__popc(peers));
                 }
                 if (POOL) {
                     uint32_t bk = vis ? key : 0u;
                     bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
                     bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
                     bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
-                    if ((row & 7) == 0 && j < __ldg(p.n_row + r)) {
-                        p.bkey[(int64_t)r * p.ld_bkey + (j >> 3)] = bk;
-                        atomicAdd(&bhist_s[bk >> 20], 1u);
-                    }
+                    const bool lead = (row & 7) == 0 && j < __ldg(p.n_row + r);
+                    if (lead) p.bkey[(int64_t)r * p.ld_bkey + (j >> 3)] = bk;
+                    const uint32_t bbin = lead ? (bk >> 20) : 0xFFFFFFFFu;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, bbin);
+                    if (lead && (lane == __ffs(peers) - 1))
+                        atomicAdd(&bhist_e[bbin], (uint32_t)__popc(peers));
                 }
             }
         }
         // final flush
-        epi_bar_sync();
+        epi_bar_sync(e);
         if (cur >= 0) {
             for (int gg = 0; gg < G; ++gg)
                 for (int i = et; i < kBins; i += 128) {
-                    const uint32_t v = hist_s[gg * kBins + i];
+                    const uint32_t v = hist_e[gg * kBins + i];
                     if (v) atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
                 }
             if (POOL)
                 for (int i = et; i < kBins; i += 128) {
-                    const uint32_t v = bhist_s[i];
+                    const uint32_t v = bhist_e[i];
                     if (v) atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
                 }
         }
@@ -527,12 +555,15 @@ static int num_sms() {
 template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
-    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G>;
-    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL>;
+    // two epilogue groups when the per-tile epilogue is short (one query row per tile)
+    constexpr int EPI = (G == 1) ? 2 : 1;
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL, EPI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms(), 192, L::kAlloc, st>>>(mk, mq, p);
+    kern<<<num_sms(), 64 + 128 * EPI, L::kAlloc, st>>>(mk, mq, p);
     return cudaGetLastError();
 }
 
@@ -597,8 +628,8 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
             if (a.pool_build) {
                 if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, true);
                 if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, true);
-                if (NQ <= 64) CSA2_SCAN(64, 2, 4, 4, 1, false, true);
-                CSA2_SCAN(128, 2, 3, 2, 1, false, true);
+                if (NQ <= 64) CSA2_SCAN(64, 2, 3, 4, 1, false, true);
+                CSA2_SCAN(128, 2, 2, 2, 1, false, true);
             }
             if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, false);
             if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, false);

@@ -25,8 +25,9 @@
 namespace csa2 {
 
 constexpr int kBinsT = 4096;
-constexpr int kSortCap = 4096;
-constexpr int kCollectChunk = 8192;
+constexpr int kSortCap = 4096;   // candidates sorted in shared memory
+constexpr int kRankCap = 1024;   // candidates selected by rank counting
+constexpr int kCollectChunk = 8192;   // elements per collect CTA (32 per thread)
 constexpr int kMaxK = 2048;
 
 struct TopkDev {
@@ -81,7 +82,21 @@ __device__ bool find_digit(const uint32_t* hist, int nb, uint32_t rem, int& d_ou
     const int per = (nb + nt - 1) / nt;
     const int lo = tid * per, hi = min(nb, lo + per);
     uint32_t local = 0;
-    for (int i = lo; i < hi; ++i) local += hist[i];
+    if (per % 4 == 0 && hi - lo == per) {
+        // whole 16-byte groups: issue every load before summing
+        const uint4* h4 = reinterpret_cast<const uint4*>(hist + lo);
+        uint4 t[8];
+        const int n4 = per / 4;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k < n4) t[k] = h4[k];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k < n4) local += t[k].x + t[k].y + t[k].z + t[k].w;
+        for (int k = 8; k < n4; ++k) local += h4[k].x + h4[k].y + h4[k].z + h4[k].w;
+    } else {
+        for (int i = lo; i < hi; ++i) local += hist[i];
+    }
     // inclusive suffix sum over threads: reverse thread order
     const int lane = tid & 31, wid = tid >> 5, nw = (nt + 31) >> 5;
     uint32_t v = local;
@@ -144,13 +159,39 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(const TopkDev a) {
     const unsigned lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     uint32_t* cnt = a.counters + (int64_t)r * 4;
-    for (int64_t i0 = start; i0 < end; i0 += blockDim.x) {
-        const int64_t i = i0 + threadIdx.x;
-        uint64_t comp = 0;
-        bool valid = (i < end) && load_elem(a, r, i, comp);
-        const int dig = (int)(comp >> 52);
-        const bool win = valid && (!many || dig > d0);
-        const bool cand = valid && many && dig == d0;
+    constexpr int kPer = kCollectChunk / 256;
+    // every load of this thread in flight before any is used
+    uint64_t comp[kPer];
+    uint32_t valid = 0;
+    if (a.scores && !a.ids) {
+        // Full rows: plain score loads, all issued before any key is formed
+        float sv[kPer];
+        const float* row = a.scores + (int64_t)r * a.ld;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int64_t i = start + (int64_t)k * blockDim.x + threadIdx.x;
+            sv[k] = (i < end) ? __ldg(row + i) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int64_t i = start + (int64_t)k * blockDim.x + threadIdx.x;
+            comp[k] = ((uint64_t)score_key(sv[k]) << 32) | (uint64_t)(~(uint32_t)i);
+            if (i < end) valid |= 1u << k;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int64_t i = start + (int64_t)k * blockDim.x + threadIdx.x;
+            comp[k] = 0;
+            if (i < end && load_elem(a, r, i, comp[k])) valid |= 1u << k;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const bool ok = (valid >> k) & 1u;
+        const int dig = (int)(comp[k] >> 52);
+        const bool win = ok && (!many || dig > d0);
+        const bool cand = ok && many && dig == d0;
         unsigned m = __ballot_sync(0xffffffffu, win);
         if (m) {
             uint32_t base = 0;
@@ -159,7 +200,7 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(const TopkDev a) {
             base = __shfl_sync(0xffffffffu, base, leader);
             if (win) {
                 const uint32_t pos = base + __popc(m & lt);
-                if (pos < (uint32_t)a.K) a.winners[(int64_t)r * a.K + pos] = comp;
+                if (pos < (uint32_t)a.K) a.winners[(int64_t)r * a.K + pos] = comp[k];
             }
         }
         m = __ballot_sync(0xffffffffu, cand);
@@ -170,7 +211,7 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(const TopkDev a) {
             base = __shfl_sync(0xffffffffu, base, leader);
             if (cand) {
                 const uint32_t pos = base + __popc(m & lt);
-                if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp;
+                if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp[k];
             }
         }
     }
@@ -187,24 +228,6 @@ __device__ void bitonic_desc_u64(uint64_t* v, int n) {
                     const uint64_t p = v[i], q = v[x];
                     const bool desc = (i & k) == 0;
                     if (desc ? (p < q) : (p > q)) {
-                        v[i] = q;
-                        v[x] = p;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-}
-
-__device__ void bitonic_asc_i32(int32_t* v, int n) {
-    for (int k = 2; k <= n; k <<= 1)
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < n; i += blockDim.x) {
-                const int x = i ^ j;
-                if (x > i) {
-                    const int32_t p = v[i], q = v[x];
-                    const bool asc = (i & k) == 0;
-                    if (asc ? (p > q) : (p < q)) {
                         v[i] = q;
                         v[x] = p;
                     }
@@ -269,7 +292,21 @@ __global__ void __launch_bounds__(512) topk_finalize_kernel(const TopkDev a) {
         src.d0 = d0;
         if (src.from_row) src.n = row_len(a, r);
         uint64_t thresh = 0;
-        if (!src.from_row && ncand <= (uint32_t)kSortCap) {
+        const bool small = !src.from_row && ncand <= (uint32_t)kRankCap;
+        if (small) {
+            // rank of each candidate among the candidates (composites are unique): the
+            // `need` largest take slots nwin + rank directly
+            for (int i = threadIdx.x; i < (int)ncand; i += blockDim.x) sortbuf[i] = src.list[i];
+            __syncthreads();
+            for (int i = threadIdx.x; i < (int)ncand; i += blockDim.x) {
+                const uint64_t c = sortbuf[i];
+                uint32_t rank = 0;
+#pragma unroll 8
+                for (int j = 0; j < (int)ncand; ++j) rank += sortbuf[j] > c;
+                if (rank < need) ids[nwin + rank] = (int32_t)(~(uint32_t)(c & 0xFFFFFFFFu));
+            }
+            __syncthreads();
+        } else if (!src.from_row && ncand <= (uint32_t)kSortCap) {
             const int n2 = pow2_at_least((int)ncand);
             for (int i = threadIdx.x; i < n2; i += blockDim.x)
                 sortbuf[i] = (i < (int)ncand) ? src.list[i] : 0ull;
@@ -327,10 +364,11 @@ __global__ void __launch_bounds__(512) topk_finalize_kernel(const TopkDev a) {
         // every candidate composite >= thresh is chosen (exactly `need` of them)
         if (threadIdx.x == 0) nsel_s = 0;
         __syncthreads();
-        if (!src.from_row && ncand <= (uint32_t)kSortCap) {
+        if (small) {
+            // already placed
+        } else if (!src.from_row && ncand <= (uint32_t)kSortCap) {
             for (uint32_t i = threadIdx.x; i < need; i += blockDim.x)
                 ids[nwin + i] = (int32_t)(~(uint32_t)(sortbuf[i] & 0xFFFFFFFFu));
-            // sortbuf was overwritten? no: it still holds the sorted candidates
         } else {
             for (int64_t i = threadIdx.x; i < src.n; i += blockDim.x) {
                 uint64_t c;
@@ -344,11 +382,17 @@ __global__ void __launch_bounds__(512) topk_finalize_kernel(const TopkDev a) {
         total = nwin + need;
     }
     __syncthreads();
-    // sort chosen ids ascending and write
-    const int n2 = pow2_at_least(max((int)total, 1));
-    for (int i = (int)total + threadIdx.x; i < n2; i += blockDim.x) ids[i] = 0x7FFFFFFF;
+    // order the chosen ids ascending: each id's rank among the (distinct) chosen ids
+    int32_t* sorted = reinterpret_cast<int32_t*>(sortbuf);
+    for (int i = threadIdx.x; i < (int)total; i += blockDim.x) {
+        const int32_t v = ids[i];
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < (int)total; ++j) rank += (ids[j] < v) | ((ids[j] == v) & (j < i));
+        sorted[rank] = v;
+    }
     __syncthreads();
-    bitonic_asc_i32(ids, n2);
+    ids = sorted;
     if (!a.expand8) {
         for (int i = threadIdx.x; i < K; i += blockDim.x)
             a.out[(int64_t)r * K + i] = (i < (int)total) ? ids[i] : -1;
