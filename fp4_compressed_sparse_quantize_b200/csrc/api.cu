@@ -317,6 +317,7 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
     tl.winners = reinterpret_cast<uint64_t*>(wb + pl.off_win);
     tl.cands = reinterpret_cast<uint64_t*>(wb + pl.off_cand);
     tl.ccap = pl.ccap;
+    tl.id_bound = cap;
     tl.status = status;
     e = launch_topk(tl, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
@@ -339,6 +340,7 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
         pt.winners = reinterpret_cast<uint64_t*>(wb + pl.off_pwin);
         pt.cands = reinterpret_cast<uint64_t*>(wb + pl.off_pcand);
         pt.ccap = pl.pccap;
+        pt.id_bound = pl.nblk;
         pt.status = status;
         e = launch_topk(pt, st);
         if (e != cudaSuccess) return CSA2_ERR_CUDA;

@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
 }
 
 int attention_splits(int Q, int K, int W, bool prefill) {
-    const int nchunks = (K + W + kR - 1) / kR;
+    const int nchunks = (K + W + 127) / 128;     // 128-row chunks of the tensor-core kernel
     if (prefill || nchunks <= 1) return 1;
     const int sms = device_sm_count();
     int ns = (2 * sms + Q - 1) / Q;
@@ -477,37 +477,10 @@ int attention_splits(int Q, int K, int W, bool prefill) {
     return (nchunks + cps - 1) / cps;
 }
 
+cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st);
+
 cudaError_t launch_attention(const AttnLaunch& l, cudaStream_t st) {
-    AttnDev a;
-    a.Q = l.Q;
-    a.T = l.T;
-    a.H = l.H;
-    a.q = reinterpret_cast<const __nv_bfloat16*>(l.q);
-    a.codes = l.codes;
-    a.scales = l.scales;
-    a.cap = l.cap;
-    a.idx = l.idx;
-    a.K = l.K;
-    a.swa = l.swa;
-    a.W = l.W;
-    a.swa_valid = l.swa_valid;
-    a.q_pos0 = l.q_pos0;
-    a.prefill = l.prefill;
-    a.scale = l.scale;
-    a.out = l.out;
-    a.partial = l.partial;
-    a.nsplit = l.nsplit;
-    a.nchunks = (l.K + l.W + kR - 1) / kR;
-    if (a.nchunks < 1) a.nchunks = 1;
-    a.chunks_per_split = (a.nchunks + l.nsplit - 1) / l.nsplit;
-    a.status = l.status;
-    const int smem = AttnSmem::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
-    attn_kernel<<<grid, 256, smem, st>>>(a);
-    e = cudaGetLastError();
+    cudaError_t e = launch_attention_tc(l, st);
     if (e != cudaSuccess || l.nsplit == 1) return e;
     attn_combine_kernel<<<dim3((unsigned)l.Q, (unsigned)l.H), 128, 0, st>>>(l.partial, l.nsplit,
                                                                           l.H, l.out);

@@ -1,0 +1,519 @@
+// Fused gather + exact FP4 dequantisation + joint sparse / sliding-window attention on the
+// 5th-generation tensor cores (tcgen05, TMEM accumulators).
+//
+// "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression" (AI summary),
+// Methodology in Plain English: a compressed global branch plus a sliding-window local
+// branch; every layer, Reuse included, computes its own query and keeps its own window KV.
+// Main Findings: main KV is E2M1 with an E4M3 scale per 16 channels; the window KV stays
+// FP8. "DeepSeek-V4.1-Flash: A New Era in Efficient Large-Scale LLM Serving", Causal
+// Encoder-Decoder: a 128-token window in every layer.
+//
+// Reading adopted (the pages do not spell out the join): one softmax over the selected
+// compressed entries and the window rows together; logits = scale * <q_h, x_i>; output
+// sum_i p_i x_i (keys and values are the same 512-channel latent). No sink, no
+// de-duplication. An empty row set gives a zero output.
+//
+// Numerics. FP4 x E4M3 and E4M3 values have at most 6 significant bits inside the fp16
+// normal range, so the dequantised rows are EXACT in fp16. The query goes to fp16 after an
+// exact per-head power-of-two rescale (largest |q| in [2^14, 2^15)), which keeps every
+// element above 2^-28 of the head's largest exactly; the power of two is folded into the
+// logit scale. Probabilities enter P x V as an fp16 (high, low) pair whose products are
+// accumulated together (~22-bit probabilities: one fp16 rounding of P alone costs ~2e-3 of
+// the output RMS on heavy-tailed channels). All accumulation is fp32 in TMEM.
+//
+// One CTA owns one query row (all heads, padded to 64) and a range of 128-row chunks of
+// the concatenated [selected entries | window rows] list:
+//   1. every thread gathers its share of the chunk's rows (FP4 codes + scales, or E4M3
+//      window rows), dequantises to fp16 and stores them into X [128 rows x 512] laid out
+//      in 128-byte-swizzled slabs of 64 channels; the query Q [64 x 512] likewise;
+//   2. one thread issues S^T = X Q^T (M = 128 rows, N = 64 heads, K = 512): 32 tcgen05.mma;
+//   3. four warps read S^T from TMEM (one row per thread) into a transposed shared tile;
+//      256 threads take (head, 32-row quarter) slices for the softmax and write P (high and
+//      low fp16 parts) as the K-major B operand [64 heads x 128 rows];
+//   4. one thread issues O^T += X^T P^T (M = 128 channels per tile, 4 tiles, N = 64 heads,
+//      K = 128 rows) reading the SAME X tile as an MN-major A operand;
+//   5. eight warps read O^T from TMEM (one channel per thread) and write the output, or
+//      the (max, sum, output) partial that a merge kernel combines when the rows of a query
+//      were split over several CTAs.
+// A CTA with several chunks (prefill) first sweeps them for the exact per-head maximum,
+// then sweeps again to accumulate P x V, so no accumulator is ever rescaled.
+#include "csa2_common.cuh"
+#include "csa2_internal.h"
+
+namespace csa2 {
+
+constexpr int kRows = 128;     // rows per chunk (MMA M of S^T, K of O^T)
+constexpr int kD = 512;        // latent channels
+constexpr int kHeads = 64;     // heads per CTA (MMA N), padded
+
+struct TcAttnDev {
+    int Q, T, H;
+    const __nv_bfloat16* q;
+    const uint8_t* codes;
+    const uint8_t* scales;
+    int64_t cap;
+    const int32_t* idx;
+    int K;
+    const uint8_t* swa;
+    int W;
+    const int32_t* swa_valid;
+    const int32_t* q_pos0;
+    bool prefill;
+    float scale;
+    float* out;
+    float* partial;
+    int nsplit, nchunks, chunks_per_split;
+    int32_t* status;
+};
+
+struct TcSmem {
+    static constexpr int kX = 0;                          // 8 slabs x [128 rows x 128 B]
+    static constexpr int kXSlab = kRows * 128;            // 16 KiB
+    static constexpr int kQ = kX + 8 * kXSlab;            // 8 slabs x [64 rows x 128 B]
+    static constexpr int kQSlab = kHeads * 128;           // 8 KiB
+    // after S^T is computed the Q region holds the transposed logits and P
+    static constexpr int kS = kQ;                         // fp32 [64 heads][128 rows]
+    static constexpr int kPhi = kS + kHeads * kRows * 4;  // 2 slabs x [64 x 128 B]
+    static constexpr int kPlo = kPhi + 2 * kQSlab;
+    static constexpr int kMisc = kQ + 8 * kQSlab;
+    static constexpr int kQf = kMisc;                     // 64 floats
+    static constexpr int kM = kQf + 256;                  // 64 floats
+    static constexpr int kL = kM + 256;                   // 64 floats
+    static constexpr int kValid = kL + 256;               // 128 ints
+    static constexpr int kBar = kValid + 512;             // 2 mbarriers
+    static constexpr int kTmem = kBar + 16;
+    static constexpr int kBytes = kTmem + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(TcSmem::kPlo + 2 * TcSmem::kQSlab <= TcSmem::kMisc, "P fits in the Q region");
+
+// byte offset of 16-byte chunk `c` (0..7) of row `r` inside one 128-byte-wide slab
+__device__ __forceinline__ uint32_t slab_off(int r, int c) {
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t e2m1x2_to_h2_tc(uint32_t byte) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(out)
+        : "r"(byte));
+    return out;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// Transposed logit tile S[h][r] (fp32, 128 rows per head): within each 32-row quarter q the
+// row is rotated by 8q + (h mod 8), so both the row-per-thread writes and the
+// (head, quarter)-per-thread reads touch 32 distinct banks.
+__device__ __forceinline__ int s_idx(int h, int r) {
+    return h * kRows + (r & ~31) + (((r & 31) + 8 * (r >> 5) + (h & 7)) & 31);
+}
+
+// Gather + dequantise rows [ch*128, ch*128+128) of query row `qrow` into X (all 256 threads:
+// two threads per row, 16 groups of 16 channels each). Records per-row validity.
+__device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, int t, int ch,
+                                           uint32_t sX, int* rvalid) {
+    const int tid = threadIdx.x;
+    const int i = tid >> 1, part = tid & 1;      // row within the chunk, half of its channels
+    const int g = ch * kRows + i;
+    int kind = 0;
+    const uint8_t* src_codes = nullptr;
+    const uint8_t* src_scales = nullptr;
+    const uint8_t* src_swa = nullptr;
+    if (g < a.K) {
+        const int32_t e = __ldg(a.idx + (int64_t)qrow * a.K + g);
+        if (e >= 0 && e < a.cap) {
+            kind = 1;
+            const int64_t ent = (int64_t)b * a.cap + e;
+            src_codes = a.codes + ent * CSA2_ENTRY_CODE_BYTES + part * 128;
+            src_scales = a.scales + ent * CSA2_ENTRY_SCALE_BYTES + part * 16;
+        } else if (e != -1 && part == 0) {
+            set_status(a.status, CSA2_DEV_BAD_INDEX);
+        }
+    } else if (g < a.K + a.W) {
+        const int v = g - a.K;   // window row 0..W-1, oldest first
+        int64_t srow;
+        bool ok;
+        if (!a.prefill) {
+            const int nv = a.swa_valid ? __ldg(a.swa_valid + b) : a.W;
+            ok = v >= a.W - nv;
+            srow = (int64_t)b * a.W + v;
+        } else {
+            const int64_t rw = t + v;
+            const int64_t pos =
+                (a.q_pos0 ? (int64_t)__ldg(a.q_pos0 + b) : (int64_t)(a.W - 1)) - (a.W - 1) + rw;
+            ok = pos >= 0;
+            srow = (int64_t)b * (a.W - 1 + a.T) + rw;
+        }
+        if (ok) {
+            kind = 2;
+            src_swa = a.swa + srow * kD + part * 256;
+        }
+    }
+    if (part == 0) rvalid[i] = kind;
+    // issue every load of this thread before converting
+    uint4 raw[16];
+    uint4 sc4 = make_uint4(0, 0, 0, 0);
+    if (kind == 1) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) raw[k] = __ldg(reinterpret_cast<const uint4*>(src_codes) + k);
+        sc4 = __ldg(reinterpret_cast<const uint4*>(src_scales));
+    } else if (kind == 2) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) raw[k] = __ldg(reinterpret_cast<const uint4*>(src_swa) + k);
+    }
+    const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+    // 16 groups of 16 channels: group gl covers channels 256*part + 16*gl
+#pragma unroll
+    for (int gl = 0; gl < 16; ++gl) {
+        uint32_t hv[8];
+        if (kind == 1) {
+            const uint4 cb = raw[gl >> 1];
+            const uint32_t w0 = (gl & 1) ? cb.z : cb.x, w1 = (gl & 1) ? cb.w : cb.y;
+            const uint32_t sbyte = (scw[gl >> 2] >> (8 * (gl & 3))) & 0xFFu;
+            const __half2 s2 = __half2half2(__float2half_rn(e4m3_to_float((uint8_t)sbyte)));
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t byte = ((k < 4 ? w0 : w1) >> (8 * (k & 3))) & 0xFFu;
+                uint32_t h2 = e2m1x2_to_h2_tc(byte);
+                hv[k] = h2_bits(__hmul2(*reinterpret_cast<__half2*>(&h2), s2));
+            }
+        } else if (kind == 2) {
+            const uint4 eb = raw[gl];
+            const uint32_t ew[4] = {eb.x, eb.y, eb.z, eb.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                hv[k] = h2_bits(e4m3x2_to_half2((uint16_t)(ew[k >> 1] >> (16 * (k & 1)))));
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) hv[k] = 0u;
+        }
+        const int c0 = 256 * part + 16 * gl;         // first channel of the group
+        const uint32_t slab = sX + (c0 >> 6) * TcSmem::kXSlab;
+        const int cc = (c0 & 63) >> 3;               // 16-byte chunk within the slab row
+        st_shared_v4(slab + slab_off(i, cc), hv[0], hv[1], hv[2], hv[3]);
+        st_shared_v4(slab + slab_off(i, cc + 1), hv[4], hv[5], hv[6], hv[7]);
+    }
+}
+
+// S^T = X Q^T into TMEM columns [0, 64)
+__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sX, uint32_t sQ) {
+    constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u);
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint64_t ad = sw128_desc(sX + (kk >> 2) * TcSmem::kXSlab + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sw128_desc(sQ + (kk >> 2) * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
+        mma_f16(tmem, ad, bd, idesc, kk > 0);
+    }
+}
+
+// O^T (+)= X^T P^T for both P parts into TMEM columns [64, 320)
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sX, uint32_t sPhi,
+                                         uint32_t sPlo, bool accumulate) {
+    constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u, /*a MN-major*/ 1u, 0u);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const uint32_t sP = part ? sPlo : sPhi;
+#pragma unroll
+            for (int kk = 0; kk < kRows / 16; ++kk) {
+                // A: channels [128m, 128m+128) x rows [16kk, 16kk+16), MN-major: the two
+                // 64-channel halves are adjacent slabs (LBO), 8-row groups 1 KiB apart (SBO)
+                const uint64_t ad =
+                    sw128_desc(sX + (2 * m) * TcSmem::kXSlab + kk * 16 * 128, TcSmem::kXSlab, 1024);
+                const uint64_t bd =
+                    sw128_desc(sP + (kk >> 2) * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
+                mma_f16(tmem + kHeads + 64 * m, ad, bd, idesc,
+                        (accumulate || part > 0 || kk > 0) ? 1u : 0u);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    using L = TcSmem;
+    const uint32_t sX = smem_u32(sm + L::kX), sQ = smem_u32(sm + L::kQ),
+                   sPhi = smem_u32(sm + L::kPhi), sPlo = smem_u32(sm + L::kPlo);
+    float* Ssm = reinterpret_cast<float*>(sm + L::kS);
+    float* qf = reinterpret_cast<float*>(sm + L::kQf);
+    float* m_s = reinterpret_cast<float*>(sm + L::kM);
+    float* l_s = reinterpret_cast<float*>(sm + L::kL);
+    int* rvalid = reinterpret_cast<int*>(sm + L::kValid);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::kTmem);
+
+    const int qrow = blockIdx.x, split = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = qrow / a.T, t = qrow - b * a.T;
+    const int c_begin = split * a.chunks_per_split;
+    const int c_end = min(a.nchunks, c_begin + a.chunks_per_split);
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_holder, 512);
+    if (tid < kHeads) m_s[tid] = -INFINITY;
+
+    // ---- query: per-head power-of-two rescale into fp16, K-major swizzled slabs --------
+    auto load_q = [&]() {
+        uint4 raw[8][2];   // this warp's 8 heads, all loads in flight before use
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int h = warp + 8 * k;
+            if (h < a.H) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    a.q + ((int64_t)qrow * a.H + h) * kD + lane * 16);
+                raw[k][0] = __ldg(src);
+                raw[k][1] = __ldg(src + 1);
+            } else {
+                raw[k][0] = raw[k][1] = make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int h = warp + 8 * k;
+            float v[16];
+            const uint32_t w8[8] = {raw[k][0].x, raw[k][0].y, raw[k][0].z, raw[k][0].w,
+                                    raw[k][1].x, raw[k][1].y, raw[k][1].z, raw[k][1].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[2 * e] = __uint_as_float(w8[e] << 16);
+                v[2 * e + 1] = __uint_as_float(w8[e] & 0xFFFF0000u);
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            int shift = 0;
+            if (amax > 0.f) {
+                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                shift = min(126, max(-126, 14 - ex));
+            }
+            const float mul = ldexpf(1.0f, shift);
+            uint32_t hw[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                hw[e] = h2_bits(__floats2half2_rn(v[2 * e] * mul, v[2 * e + 1] * mul));
+            // lane owns channels [16 lane, 16 lane + 16): slab lane/4, chunks 2(lane%4), +1
+            const uint32_t slab = sQ + (lane >> 2) * L::kQSlab;
+            const int cc = (lane & 3) * 2;
+            st_shared_v4(slab + slab_off(h, cc), hw[0], hw[1], hw[2], hw[3]);
+            st_shared_v4(slab + slab_off(h, cc + 1), hw[4], hw[5], hw[6], hw[7]);
+            if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * ldexpf(1.0f, -shift);
+        }
+    };
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t quad = (uint32_t)(32 * (warp & 3)) << 16;
+    uint32_t phase[2] = {0u, 0u};
+    bool ok = true;
+
+    // wait on barrier i (all threads), bounded
+    auto wait_bar = [&](int i) {
+        if (ok && !mbar_wait(&bar[i], phase[i], a.status)) ok = false;
+        phase[i] ^= 1u;
+    };
+
+    // S^T for chunk ch -> transposed logits Ssm[h][r] (log2 domain, -inf for empty rows)
+    auto scores = [&](int ch) {
+        load_chunk(a, qrow, b, t, ch, sX, rvalid);
+        load_q();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            issue_s(tmem, sX, sQ);
+            mma_commit(&bar[0]);
+        }
+        wait_bar(0);
+        tc_fence_after();
+        if (warp < 4) {
+            const int r = 32 * warp + lane;
+            const bool valid = rvalid[r] != 0;
+            uint32_t v[4][16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld16(tmem + quad + 16 * c, v[c]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int h = 16 * c + k;
+                    Ssm[s_idx(h, r)] = valid ? __uint_as_float(v[c][k]) * qf[h] : -INFINITY;
+                }
+        }
+        tc_fence_before();
+        __syncthreads();
+    };
+
+    const int h = tid >> 2, qq = tid & 3;   // softmax slice: head h, rows [32 qq, +32)
+    float l_acc = 0.f;
+
+    // ---- pass 1 (several chunks only): exact per-head maximum ---------------------------
+    if (c_end - c_begin > 1) {
+        for (int ch = c_begin; ch < c_end; ++ch) {
+            scores(ch);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, Ssm[s_idx(h, 32 * qq + j)]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            if (qq == 0) m_s[h] = fmaxf(m_s[h], mx);
+            __syncthreads();
+        }
+    }
+
+    // ---- pass 2: softmax numerators and P x V -------------------------------------------
+    for (int ch = c_begin; ch < c_end; ++ch) {
+        scores(ch);
+        float sv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = Ssm[s_idx(h, 32 * qq + j)];
+        float m;
+        if (c_end - c_begin > 1) {
+            m = m_s[h];
+        } else {
+            m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m = fmaxf(m, sv[j]);
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        }
+        const float base = (m == -INFINITY) ? 0.f : m;
+        uint32_t hi[16], lo[16];
+        float ls = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float p0 = exp2f(sv[2 * j] - base), p1 = exp2f(sv[2 * j + 1] - base);
+            ls += p0 + p1;
+            const __half2 ph = __floats2half2_rn(p0, p1);
+            hi[j] = h2_bits(ph);
+            lo[j] = h2_bits(__floats2half2_rn(p0 - __low2float(ph), p1 - __high2float(ph)));
+        }
+        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+        l_acc += ls;
+        if (qq == 0 && c_end - c_begin == 1) m_s[h] = m;
+        __syncthreads();   // every thread has read its logits before P overwrites the tile
+        // P[h][rows 32qq .. 32qq+31]: slab qq/2, chunks 4(qq%2) .. +4, row h
+        {
+            const uint32_t ohi = sPhi + (qq >> 1) * L::kQSlab, olo = sPlo + (qq >> 1) * L::kQSlab;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int cc = 4 * (qq & 1) + c;
+                st_shared_v4(ohi + slab_off(h, cc), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                st_shared_v4(olo + slab_off(h, cc), lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            issue_pv(tmem, sX, sPhi, sPlo, ch > c_begin);
+            mma_commit(&bar[1]);
+        }
+        wait_bar(1);
+        tc_fence_after();
+        __syncthreads();   // X and the Q region may be rewritten by the next chunk
+    }
+    if (qq == 0) l_s[h] = l_acc;
+    __syncthreads();
+
+    // ---- epilogue: O^T tiles (warps 0-3: tiles 0,1; warps 4-7: tiles 2,3) ---------------
+    if (ok) {
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            const int tile = 2 * (warp >> 2) + tt;
+            const int c = 128 * tile + 32 * (warp & 3) + lane;   // channel of this thread
+            uint32_t v[4][16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tmem_ld16(tmem + quad + kHeads + 64 * tile + 16 * k, v[k]);
+            tmem_ld_wait();
+            if (a.nsplit == 1) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int hh = 16 * k + e;
+                        if (hh < a.H) {
+                            const float l = l_s[hh];
+                            a.out[((int64_t)qrow * a.H + hh) * kD + c] =
+                                l > 0.f ? __uint_as_float(v[k][e]) / l : 0.f;
+                        }
+                    }
+            } else {
+                float* base = a.partial + ((int64_t)qrow * a.nsplit + split) * ((int64_t)a.H * (kD + 2));
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int hh = 16 * k + e;
+                        if (hh < a.H) base[(int64_t)hh * kD + c] = __uint_as_float(v[k][e]);
+                    }
+                if (tile == 0 && warp == 0 && lane < 32) {
+                    for (int hh = lane; hh < a.H; hh += 32) {
+                        base[(int64_t)a.H * kD + hh] = m_s[hh];
+                        base[(int64_t)a.H * kD + a.H + hh] = l_s[hh];
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
+    TcAttnDev a;
+    a.Q = l.Q;
+    a.T = l.T;
+    a.H = l.H;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(l.q);
+    a.codes = l.codes;
+    a.scales = l.scales;
+    a.cap = l.cap;
+    a.idx = l.idx;
+    a.K = l.K;
+    a.swa = l.swa;
+    a.W = l.W;
+    a.swa_valid = l.swa_valid;
+    a.q_pos0 = l.q_pos0;
+    a.prefill = l.prefill;
+    a.scale = l.scale;
+    a.out = l.out;
+    a.partial = l.partial;
+    a.nsplit = l.nsplit;
+    a.nchunks = (l.K + l.W + kRows - 1) / kRows;
+    if (a.nchunks < 1) a.nchunks = 1;
+    a.chunks_per_split = (a.nchunks + l.nsplit - 1) / l.nsplit;
+    a.status = l.status;
+    const int smem = TcSmem::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
+    attn_tc_kernel<<<grid, 256, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -60,6 +60,7 @@ struct TopkLaunch {
     uint64_t* winners;       // [R][K]
     uint64_t* cands;         // [R][ccap]
     int ccap;
+    int64_t id_bound;        // every id is below this (0: unknown)
     int32_t* status;
 };
 

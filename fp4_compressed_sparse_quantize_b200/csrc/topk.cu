@@ -26,7 +26,7 @@ namespace csa2 {
 
 constexpr int kBinsT = 4096;
 constexpr int kSortCap = 4096;   // candidates sorted in shared memory
-constexpr int kRankCap = 1024;   // candidates selected by rank counting
+constexpr int kRankCap = 64;     // candidates selected by rank counting
 constexpr int kCollectChunk = 8192;   // elements per collect CTA (32 per thread)
 constexpr int kMaxK = 2048;
 
@@ -47,6 +47,7 @@ struct TopkDev {
     uint64_t* winners;
     uint64_t* cands;
     int ccap;
+    int bitmap_words;        // > 0: order the picks through a shared bitmap of ids
     int32_t* status;
 };
 
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(const TopkDev a) {
     const bool many = find_digit(a.hist + (int64_t)r * kBinsT, kBinsT, (uint32_t)a.K + 0u, d0,
                                  above, red);
     // many == false: at most K valid elements, all of them win
-    const unsigned lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     uint32_t* cnt = a.counters + (int64_t)r * 4;
     constexpr int kPer = kCollectChunk / 256;
@@ -186,34 +187,52 @@ __global__ void __launch_bounds__(256) topk_collect_kernel(const TopkDev a) {
             if (i < end && load_elem(a, r, i, comp[k])) valid |= 1u << k;
         }
     }
+    // pass 1: this CTA's winner / candidate counts, one global atomic per list per CTA
+    const int wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    uint32_t mw[kPer], mc[kPer];
+    uint32_t cw = 0, cc = 0;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const bool ok = (valid >> k) & 1u;
         const int dig = (int)(comp[k] >> 52);
-        const bool win = ok && (!many || dig > d0);
-        const bool cand = ok && many && dig == d0;
-        unsigned m = __ballot_sync(0xffffffffu, win);
-        if (m) {
-            uint32_t base = 0;
-            const int leader = __ffs(m) - 1;
-            if ((int)lane == leader) base = atomicAdd(cnt + 0, (uint32_t)__popc(m));
-            base = __shfl_sync(0xffffffffu, base, leader);
-            if (win) {
-                const uint32_t pos = base + __popc(m & lt);
-                if (pos < (uint32_t)a.K) a.winners[(int64_t)r * a.K + pos] = comp[k];
-            }
+        mw[k] = __ballot_sync(0xffffffffu, ok && (!many || dig > d0));
+        mc[k] = __ballot_sync(0xffffffffu, ok && many && dig == d0);
+        cw += __popc(mw[k]);
+        cc += __popc(mc[k]);
+    }
+    __shared__ uint32_t wsum[2][32], wbase[2];
+    if (lane == 0) {
+        wsum[0][wid] = cw;
+        wsum[1][wid] = cc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t tw = 0, tc = 0;
+        for (int w = 0; w < nwarps; ++w) {
+            const uint32_t a0 = wsum[0][w], a1 = wsum[1][w];
+            wsum[0][w] = tw;
+            wsum[1][w] = tc;
+            tw += a0;
+            tc += a1;
         }
-        m = __ballot_sync(0xffffffffu, cand);
-        if (m) {
-            uint32_t base = 0;
-            const int leader = __ffs(m) - 1;
-            if ((int)lane == leader) base = atomicAdd(cnt + 1, (uint32_t)__popc(m));
-            base = __shfl_sync(0xffffffffu, base, leader);
-            if (cand) {
-                const uint32_t pos = base + __popc(m & lt);
-                if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp[k];
-            }
+        wbase[0] = tw ? atomicAdd(cnt + 0, tw) : 0u;
+        wbase[1] = tc ? atomicAdd(cnt + 1, tc) : 0u;
+    }
+    __syncthreads();
+    // pass 2: write at the reserved offsets
+    uint32_t pw = wbase[0] + wsum[0][wid], pc = wbase[1] + wsum[1][wid];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        if ((mw[k] >> lane) & 1u) {
+            const uint32_t pos = pw + __popc(mw[k] & lt);
+            if (pos < (uint32_t)a.K) a.winners[(int64_t)r * a.K + pos] = comp[k];
         }
+        if ((mc[k] >> lane) & 1u) {
+            const uint32_t pos = pc + __popc(mc[k] & lt);
+            if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp[k];
+        }
+        pw += __popc(mw[k]);
+        pc += __popc(mc[k]);
     }
 }
 
@@ -382,6 +401,78 @@ __global__ void __launch_bounds__(512) topk_finalize_kernel(const TopkDev a) {
         total = nwin + need;
     }
     __syncthreads();
+    if (a.bitmap_words > 0) {
+        // ascending order without sorting: mark the picks in a bitmap of ids, then each
+        // thread emits the set bits of its word range at its exclusive-scan offset
+        uint32_t* bm = reinterpret_cast<uint32_t*>(ids + kMaxK);
+        const int nwords = a.bitmap_words;
+        for (int i = threadIdx.x; i < nwords; i += blockDim.x) bm[i] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < (int)total; i += blockDim.x) {
+            const uint32_t v = (uint32_t)ids[i];
+            if ((int)(v >> 5) < nwords) atomicOr(&bm[v >> 5], 1u << (v & 31));
+        }
+        __syncthreads();
+        const int per = (nwords + blockDim.x - 1) / blockDim.x;
+        const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
+        uint32_t cntb = 0;
+        for (int wi = w0; wi < w1; ++wi) cntb += __popc(bm[wi]);
+        // block exclusive scan of cntb
+        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+        uint32_t incl = cntb;
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        if (lane == 31) red[wid] = incl;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t acc = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+                const uint32_t t = red[w];
+                red[w] = acc;
+                acc += t;
+            }
+            ncoll_s = acc;  // distinct picks (equals `total` unless ids repeat)
+        }
+        __syncthreads();
+        uint32_t off = red[wid] + incl - cntb;
+        const int npick = (int)min(ncoll_s, (uint32_t)K);
+        if (!a.expand8) {
+            int32_t* o = a.out + (int64_t)r * K;
+            for (int wi = w0; wi < w1; ++wi) {
+                uint32_t m = bm[wi];
+                while (m) {
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (off < (uint32_t)K) o[off] = wi * 32 + b;
+                    ++off;
+                }
+            }
+            for (int i = npick + threadIdx.x; i < K; i += blockDim.x) o[i] = -1;
+        } else {
+            const int32_t lim = __ldg(a.expand_limit + r);
+            int32_t* o = a.out + (int64_t)r * K * 8;
+            for (int wi = w0; wi < w1; ++wi) {
+                uint32_t m = bm[wi];
+                while (m) {
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (off < (uint32_t)K) {
+                        const int64_t blk = (int64_t)wi * 32 + b;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int64_t pos = blk * 8 + e;
+                            o[off * 8 + e] = pos < lim ? (int32_t)pos : -1;
+                        }
+                    }
+                    ++off;
+                }
+            }
+            for (int i = npick * 8 + threadIdx.x; i < K * 8; i += blockDim.x) o[i] = -1;
+        }
+        return;
+    }
     // order the chosen ids ascending: each id's rank among the (distinct) chosen ids
     int32_t* sorted = reinterpret_cast<int32_t*>(sortbuf);
     for (int i = threadIdx.x; i < (int)total; i += blockDim.x) {
@@ -438,7 +529,11 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    const size_t smem = kSortCap * 8 + kBinsT * 4 + kMaxK * 4;
+    // ids are < id_bound: a bitmap of that many bits orders the picks if it fits
+    const int64_t words = (l.id_bound + 31) / 32;
+    const size_t base = kSortCap * 8 + kBinsT * 4 + kMaxK * 4;
+    a.bitmap_words = (l.id_bound > 0 && base + words * 4 <= 200 * 1024) ? (int)words : 0;
+    const size_t smem = base + (size_t)a.bitmap_words * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_finalize_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
