@@ -22,7 +22,8 @@ D_MAIN, D_INDEX, POOL_BLOCK = 512, 128, 8
 EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode",
            "csa2_sparse_attn_prefill", "csa2_workspace_bytes", "csa2_status_string",
            "csa2_read_device_status", "csa2_reset_device_status", "csa2_version",
-           "csa2_debug_bounded_wait", "csa2_set_stage_events")
+           "csa2_debug_bounded_wait", "csa2_set_stage_events",
+           "csa2_index_score_topk_noalloc")
 
 
 class Csa2Error(RuntimeError):
@@ -58,6 +59,8 @@ def lib():
         L.csa2_reset_device_status.argtypes = [P, P]
         L.csa2_debug_bounded_wait.argtypes = [P, C.c_uint64, P]
         L.csa2_set_stage_events.argtypes = [P, P]
+        L.csa2_index_score_topk_noalloc.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P,
+                                                    i32, P, i32, P, i32, P, i32, P, P, P, P]
         for name in EXPORTS:
             if name not in ("csa2_workspace_bytes", "csa2_status_string"):
                 getattr(L, name).restype = i32
@@ -178,6 +181,34 @@ def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None
         _p(q_pos0), int(K), _p(pool_in), P_in, _p(pool_out), int(pool_blocks), _p(idx_out),
         _p(scores_out), _p(ws), ws.numel() if ws is not None else 0, _stream(stream))
     _check(st, "csa2_index_score_topk")
+
+
+def index_score_topk_noalloc(mode, q_I, w, k_I, K, idx_out, n_vis0=None, q_pos0=None, ratio=1,
+                             pool_in=None, pool_out=None, pool_blocks=0, scores_out=None,
+                             status=None, stream=None):
+    """index_score_topk without a workspace argument, for callers that cannot allocate: the
+    library's fixed 16 MiB device scratch array is used instead (see include/csa2.h).
+    `status` is an optional int32 CUDA tensor that receives the device status bits."""
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    B, T, H_I, Di = q_I.shape
+    if q_I.dtype not in DTYPE or k_I.dtype != q_I.dtype:
+        raise Csa2Error(ERR_ARG, "q_I and k_I must share a dtype (bf16 or float8_e4m3fn)")
+    for t, nm in ((q_I, "q_I"), (k_I, "k_I")):
+        _need(t, q_I.dtype, nm)
+    _need(w, torch.float32, "w")
+    _need(idx_out, torch.int32, "idx_out")
+    _need(n_vis0, torch.int32, "n_vis0")
+    _need(q_pos0, torch.int32, "q_pos0")
+    _need(pool_in, torch.int32, "pool_in")
+    _need(pool_out, torch.int32, "pool_out")
+    _need(scores_out, torch.float32, "scores_out")
+    _need(status, torch.int32, "status")
+    P_in = pool_in.shape[-1] if pool_in is not None else 0
+    st = lib().csa2_index_score_topk_noalloc(
+        m, B, T, H_I, DTYPE[q_I.dtype], _p(q_I), _p(w), _p(k_I), k_I.shape[1], _p(n_vis0),
+        int(ratio), _p(q_pos0), int(K), _p(pool_in), P_in, _p(pool_out), int(pool_blocks),
+        _p(idx_out), _p(scores_out), _p(status), _stream(stream))
+    _check(st, "csa2_index_score_topk_noalloc")
 
 
 def sparse_attn_decode(mode, q, codes, scales, idx, swa, out, ws, scale=None, swa_valid=None,

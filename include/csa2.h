@@ -201,6 +201,27 @@ CSA2_API csa2_status_t csa2_sparse_attn_prefill(int B, int T, int H, const void*
                                        float scale, float* out, void* ws, size_t ws_bytes,
                                        void* stream);
 
+/*
+ * csa2_index_score_topk_noalloc — csa2_index_score_topk for callers that cannot allocate
+ * device memory. (This entry point has no counterpart on the source pages; it is a
+ * deployment convenience.) Callers such as plugins inside an inference engine that owns
+ * every device allocation, or latency-critical loops where an allocation may synchronise
+ * the device, cannot provide a workspace. This variant takes the same arguments minus the
+ * workspace and uses a fixed 16 MiB device array inside the library instead (held on every
+ * GPU that loads the library until the process exits).
+ *   status   nullable int32 device word: the call's device status bits are OR-ed into it.
+ * Returns CSA2_ERR_WORKSPACE when csa2_workspace_bytes() for the call exceeds 16 MiB. The
+ * first call on a device looks up the array's address with that device current; make it
+ * before any stream capture. All calls share the array, which keeps the previous call's
+ * contents (the call clears what must start at zero): calls that overlap on the GPU race,
+ * so order them on one stream. It allocates nothing.
+ */
+CSA2_API csa2_status_t csa2_index_score_topk_noalloc(
+    csa2_mode_t mode, int B, int T, int H_I, csa2_dtype_t qk_dtype, const void* q_I,
+    const float* w, const void* k_I, int64_t cap, const int32_t* n_vis0, int ratio,
+    const int32_t* q_pos0, int K, const int32_t* pool_in, int P_in, int32_t* pool_out,
+    int pool_blocks, int32_t* idx_out, float* scores_out, int32_t* status, void* stream);
+
 /* Workspace bytes an operation needs (0 on invalid arguments).
  *   CSA2_OP_INDEX_SCORE_TOPK: H = H_I; cap = cache capacity (Full) or P_in (Reindex);
  *                             pool_blocks = 0 when no pool is built.
