@@ -263,8 +263,8 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
             e = cudaMemsetAsync(wb + pl.off_pcnt, 0, sizeof(uint32_t) * 4 * (size_t)R, st);
     }
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    e = launch_prep_rows(R, T, pl.G, n_vis0, q_pos0, ratio, cap, reindex ? P_in : 0, n_row,
-                         prefix, status, st);
+    e = launch_prep_rows(R, T, pl.G, n_vis0, q_pos0, ratio, cap, reindex ? P_in : 0,
+                         scan_tile_rows(pl.G, reindex, esz), n_row, prefix, status, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
 
     ScanLaunch sl;

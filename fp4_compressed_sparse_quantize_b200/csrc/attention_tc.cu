@@ -206,7 +206,7 @@ __device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, 
 // S^T = X Q^T into TMEM columns [0, 64)
 __device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sX, uint32_t sQ) {
     constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u);
-#pragma unroll
+#pragma unroll 4
     for (int kk = 0; kk < kD / 16; ++kk) {
         const uint64_t ad = sw128_desc(sX + (kk >> 2) * TcSmem::kXSlab + (kk & 3) * 32, 16, 1024);
         const uint64_t bd = sw128_desc(sQ + (kk >> 2) * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
@@ -218,9 +218,9 @@ __device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sX, uint32_t sQ)
 __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sX, uint32_t sPhi,
                                          uint32_t sPlo, bool accumulate) {
     constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u, /*a MN-major*/ 1u, 0u);
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < 4; ++m) {
-#pragma unroll
+#pragma unroll 1
         for (int part = 0; part < 2; ++part) {
             const uint32_t sP = part ? sPlo : sPhi;
 #pragma unroll
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
                 const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
                 shift = min(126, max(-126, 14 - ex));
             }
-            const float mul = ldexpf(1.0f, shift);
+            const float mul = __int_as_float((127 + shift) << 23);   // 2^shift, exact
             uint32_t hw[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
             const int cc = (lane & 3) * 2;
             st_shared_v4(slab + slab_off(h, cc), hw[0], hw[1], hw[2], hw[3]);
             st_shared_v4(slab + slab_off(h, cc + 1), hw[4], hw[5], hw[6], hw[7]);
-            if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * ldexpf(1.0f, -shift);
+            if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
         }
     };
 

@@ -35,8 +35,11 @@ cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
 
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
                              const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
-                             int32_t* n_row, int64_t* prefix, int32_t* status,
+                             int tile_rows, int32_t* n_row, int64_t* prefix, int32_t* status,
                              cudaStream_t st);
+
+// keys per scan tile for a query-group size and mode
+int scan_tile_rows(int G, bool gather, int esz);
 
 cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st);
 

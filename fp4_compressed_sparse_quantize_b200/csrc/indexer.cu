@@ -55,9 +55,10 @@ struct ScanParams {
 };
 
 // ---- shared memory plan ----------------------------------------------------------------
-template <int NQ, int ESZ, int STAGES, int ACC, int G, int EPI, bool POOL>
+template <int NQ, int ESZ, int STAGES, int ACC, int G, int EPI, bool POOL, int TM>
 struct ScanSmem {
-    static constexpr int kTileBytes = kTileRows * 128 * ESZ;
+    static constexpr int kRowsT = kTileRows * TM;         // keys per tile
+    static constexpr int kTileBytes = kRowsT * 128 * ESZ;
     static constexpr int kQBytes = NQ * 128 * ESZ;
     static constexpr int kStageOff = 0;
     static constexpr int kQOff = kStageOff + STAGES * kTileBytes;
@@ -76,7 +77,7 @@ __device__ __forceinline__ void epi_bar_sync(int group) {
     asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory");
 }
 
-// Advance (b-group, tile) iteration state so that tile index t lies in row group g.
+// Last row group g with prefix[g] <= t.
 __device__ __forceinline__ int find_group(const int64_t* prefix, int ngroups, int64_t t) {
     int lo = 0, hi = ngroups - 1;
     while (lo < hi) {
@@ -88,6 +89,29 @@ __device__ __forceinline__ int find_group(const int64_t* prefix, int ngroups, in
     }
     return lo;
 }
+
+// Walks the tile sequence of one CTA and keeps the current row group and its tile range in
+// registers (the prefix array is read only when the row group changes).
+struct GroupCursor {
+    int g;
+    int64_t lo, hi;
+    __device__ __forceinline__ void init(const int64_t* prefix, int ngroups, int64_t t) {
+        g = find_group(prefix, ngroups, t);
+        lo = __ldg(prefix + g);
+        hi = __ldg(prefix + g + 1);
+    }
+    // returns true when t starts a new row group
+    __device__ __forceinline__ bool advance(const int64_t* prefix, int64_t t) {
+        bool moved = false;
+        while (t >= hi) {
+            ++g;
+            lo = hi;
+            hi = __ldg(prefix + g + 1);
+            moved = true;
+        }
+        return moved;
+    }
+};
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -103,22 +127,29 @@ __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// NQ   = MMA N: G * H_I rounded up to a multiple of 16 (padding rows are ignored)
-// ESZ  = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
+// NQ     = MMA N: G * H_I rounded up to a multiple of 16 (padding columns get weight 0)
+// ESZ    = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
 // GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
-template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI>
+// TM     = 128-key halves per tile (one TMA box, TM MMA groups into adjacent TMEM columns)
+template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM>
 __global__ void __launch_bounds__(64 + 128 * EPI, 1)
     scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
-    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL>;
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
     static_assert(ACC % EPI == 0, "each epilogue group owns fixed accumulators");
-    constexpr int kKSteps = (128 * ESZ) / 32;        // 32 bytes of K per MMA instruction
-    constexpr uint32_t kHalf = kTileRows * 128;      // bytes of one 128-byte-wide K slab
+    static_assert(!GATHER || TM == 1, "gathered tiles are 128 keys");
+    constexpr int kRowsT = L::kRowsT;
+    constexpr int kKSteps = (128 * ESZ) / 32;         // 32 bytes of K per MMA instruction
+    constexpr uint32_t kSlab = kRowsT * 128;          // bytes of one 128-byte-wide K slab
     constexpr uint32_t kQHalf = NQ * 128;
-    constexpr uint32_t kAccCols = NQ;
-    constexpr uint32_t kTmemCols = (ACC * NQ <= 32) ? 32 : (ACC * NQ <= 64) ? 64
-                                 : (ACC * NQ <= 128) ? 128 : (ACC * NQ <= 256) ? 256 : 512;
+    constexpr uint32_t kAccCols = TM * NQ;
+    constexpr uint32_t kTmemCols = (ACC * kAccCols <= 32) ? 32 : (ACC * kAccCols <= 64) ? 64
+                                 : (ACC * kAccCols <= 128) ? 128 : (ACC * kAccCols <= 256) ? 256
+                                 : 512;
+    static_assert(ACC * kAccCols <= 512, "TMEM budget");
     constexpr uint32_t kIdesc = make_idesc(128, NQ, ESZ == 2 ? 1u : 0u, ESZ == 2 ? 1u : 0u);
+    constexpr int kCols = NQ / G;                     // accumulator columns per query row
+    constexpr bool kWReg = (G == 1 && NQ <= 64);      // weights kept in registers
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -149,7 +180,7 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], GATHER ? 1 : 1);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -181,30 +212,31 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int g = find_group(p.prefix, ngroups, t0);
+        GroupCursor cur;
+        cur.init(p.prefix, ngroups, t0);
         int qg = -1, qcount = 0;
         int64_t it = 0;
         const uint64_t policy = l2_policy_evict_first();
         for (int64_t t = t0; t < t1; ++t, ++it) {
             if (*abort_flag) break;
-            while (t >= __ldg(p.prefix + g + 1)) ++g;
-            const int64_t jt = t - __ldg(p.prefix + g);
-            const int r0 = g * G;
+            cur.advance(p.prefix, t);
+            const int64_t jt = t - cur.lo;
+            const int r0 = cur.g * G;
             const int b = r0 / p.T;
-            if (g != qg) {
+            if (cur.g != qg) {
                 const int qs = qcount & 1;
                 bool ok = true;
                 if (lane == 0) ok = mbar_wait(&qempty[qs], ((qcount >> 1) & 1) ^ 1, p.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) { if (lane == 0) *abort_flag = 1; break; }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&qfull[qs], 2 * 0 + (uint32_t)L::kQBytes);
+                    mbar_arrive_expect_tx(&qfull[qs], (uint32_t)L::kQBytes);
                     uint8_t* dst = q_base + qs * L::kQBytes;
                     for (int h = 0; h < ESZ; ++h)
                         tma_load_2d(dst + h * kQHalf, &tmap_q, &qfull[qs], h * 64 * (ESZ == 2),
                                     r0 * p.H_I);
                 }
-                qg = g;
+                qg = cur.g;
                 ++qcount;
             }
             const int s = (int)(it % STAGES);
@@ -217,26 +249,26 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
             if (!GATHER) {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)L::kTileBytes);
-                    const int64_t row = (int64_t)b * p.cap + jt * kTileRows;
+                    const int64_t row = (int64_t)b * p.cap + jt * kRowsT;
                     for (int h = 0; h < ESZ; ++h)
-                        tma_load_2d_hint(dst + h * kHalf, &tmap_k, &full[s], h * 64 * (ESZ == 2),
+                        tma_load_2d_hint(dst + h * kSlab, &tmap_k, &full[s], h * 64 * (ESZ == 2),
                                          (int32_t)row, policy);
                 }
             } else {
                 // pool rows of query row r0 (G == 1 in gather mode)
-                const int32_t* pl = p.pool + (int64_t)r0 * p.P + jt * kTileRows;
+                const int32_t* pl = p.pool + (int64_t)r0 * p.P + jt * kRowsT;
                 const int n_vis = __ldg(p.n_row + r0);
                 const uint32_t dst_u = smem_u32(dst);
-                for (int rr = 0; rr < kTileRows; rr += 4) {
+                for (int rr = 0; rr < kRowsT; rr += 4) {
                     const int rl = rr + (lane >> 3);       // 4 rows per pass, 8 lanes per row
-                    const int64_t slot = jt * kTileRows + rl;
+                    const int64_t slot = jt * kRowsT + rl;
                     int pos = (slot < p.P) ? __ldg(pl + rl) : -1;
                     if (pos >= n_vis) pos = -1;
                     if (pos >= 0) {
                         const uint8_t* src = p.keys + ((int64_t)b * p.cap + pos) * (128 * ESZ);
                         for (int h = 0; h < ESZ; ++h) {
                             const int c = lane & 7;         // 16-byte chunk within 128 bytes
-                            const uint32_t off = h * kHalf + rl * 128 + ((c ^ (rl & 7)) << 4);
+                            const uint32_t off = h * kSlab + rl * 128 + ((c ^ (rl & 7)) << 4);
                             cp_async16(dst_u + off, src + h * 128 + c * 16);
                         }
                     }
@@ -253,21 +285,25 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
             const int64_t n_issued = it;
             for (int64_t k = (n_issued > STAGES ? n_issued - STAGES : 0); k < n_issued; ++k)
                 mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), p.status);
+            if (qcount > 0) mbar_wait(&qfull[(qcount - 1) & 1], ((qcount - 1) >> 1) & 1, p.status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int g = find_group(p.prefix, ngroups, t0);
+            GroupCursor cur;
+            cur.init(p.prefix, ngroups, t0);
             int qg = -1, qcount = 0, qs = 0;
             int64_t it = 0;
+            const uint64_t a_desc0 = sw128_desc(smem_u32(stage_base), 16, 1024);
+            const uint64_t b_desc0 = sw128_desc(smem_u32(q_base), 16, 1024);
             for (int64_t t = t0; t < t1; ++t, ++it) {
                 if (*abort_flag) break;
-                while (t >= __ldg(p.prefix + g + 1)) ++g;
-                if (g != qg) {
+                cur.advance(p.prefix, t);
+                if (cur.g != qg) {
                     if (qg >= 0) mma_commit(&qempty[qs]);
                     qs = qcount & 1;
                     if (!mbar_wait(&qfull[qs], (qcount >> 1) & 1, p.status)) { *abort_flag = 1; break; }
-                    qg = g;
+                    qg = cur.g;
                     ++qcount;
                 }
                 const int s = (int)(it % STAGES);
@@ -275,19 +311,22 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
                 const int a = (int)(it % ACC);
                 if (!mbar_wait(&accempty[a], (uint32_t)(((it / ACC) & 1) ^ 1), p.status)) { *abort_flag = 1; break; }
                 tc_fence_after();
-                const uint32_t d = tmem_base + a * kAccCols;
-                const uint32_t a_addr = smem_u32(stage_base + s * L::kTileBytes);
-                const uint32_t b_addr = smem_u32(q_base + qs * L::kQBytes);
+                // descriptor start addresses advance in 16-byte units
+                const uint64_t a_s = a_desc0 + ((uint64_t)(s * L::kTileBytes) >> 4);
+                const uint64_t b_s = b_desc0 + ((uint64_t)(qs * L::kQBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kKSteps; ++kk) {
-                    const uint32_t koff = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    const uint32_t qoff = (kk >> 2) * kQHalf + (kk & 3) * 32;
-                    const uint64_t ad = sw128_desc(a_addr + koff, 16, 1024);
-                    const uint64_t bd = sw128_desc(b_addr + qoff, 16, 1024);
-                    if (ESZ == 1)
-                        mma_f8(d, ad, bd, kIdesc, kk > 0);
-                    else
-                        mma_f16(d, ad, bd, kIdesc, kk > 0);
+                for (int hh = 0; hh < TM; ++hh) {
+                    const uint32_t d = tmem_base + a * kAccCols + hh * NQ;
+#pragma unroll
+                    for (int kk = 0; kk < kKSteps; ++kk) {
+                        const uint64_t ad = a_s + ((uint64_t)((kk >> 2) * kSlab + hh * 128 * 128 +
+                                                              (kk & 3) * 32) >> 4);
+                        const uint64_t bd = b_s + ((uint64_t)((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
+                        if (ESZ == 1)
+                            mma_f8(d, ad, bd, kIdesc, kk > 0);
+                        else
+                            mma_f16(d, ad, bd, kIdesc, kk > 0);
+                    }
                 }
                 mma_commit(&empty[s]);
                 mma_commit(&accfull[a]);
@@ -304,28 +343,31 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
         // own histograms, weights and named barrier.
         const int e = (warp - 2) >> 2;
         const int et = threadIdx.x - 64 - 128 * e;  // 0..127 within the group
-        const int row = 32 * (warp & 3) + lane;     // TMEM lane == key row within the tile
+        const int row = 32 * (warp & 3) + lane;     // TMEM lane == key row within a half
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
         uint32_t* hist_e = hist_s + e * G * kBins;
         uint32_t* bhist_e = bhist_s + e * kBins;
         float* w_e = w_s + e * 2 * NQ;
-        int g = find_group(p.prefix, ngroups, t0);
-        int cur = -1, wslot = 0;
+        GroupCursor cur;
+        cur.init(p.prefix, ngroups, t0);
+        int gcur = -1, wslot = 0;
+        int nvis[G];
+        float wr[kWReg ? NQ : 1];
         bool aborted = false;
         for (int64_t it = e; t0 + it < t1; it += EPI) {
             const int64_t t = t0 + it;
-            while (t >= __ldg(p.prefix + g + 1)) ++g;
-            const int64_t jt = t - __ldg(p.prefix + g);
-            const int r0 = g * G;
-            if (g != cur) {
+            cur.advance(p.prefix, t);
+            const int64_t jt = t - cur.lo;
+            const int r0 = cur.g * G;
+            if (cur.g != gcur) {
                 // flush the previous row group's histograms, then load the new weights
                 epi_bar_sync(e);
-                if (cur >= 0) {
+                if (gcur >= 0) {
                     for (int gg = 0; gg < G; ++gg)
                         for (int i = et; i < kBins; i += 128) {
                             const uint32_t v = hist_e[gg * kBins + i];
                             if (v) {
-                                atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
+                                atomicAdd(p.hist + (int64_t)(gcur * G + gg) * kBins + i, v);
                                 hist_e[gg * kBins + i] = 0;
                             }
                         }
@@ -333,7 +375,7 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
                         for (int i = et; i < kBins; i += 128) {
                             const uint32_t v = bhist_e[i];
                             if (v) {
-                                atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
+                                atomicAdd(p.bhist + (int64_t)(gcur * G) * kBins + i, v);
                                 bhist_e[i] = 0;
                             }
                         }
@@ -342,7 +384,13 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
                 for (int i = et; i < NQ; i += 128)
                     w_e[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
                 epi_bar_sync(e);
-                cur = g;
+                if (kWReg) {
+#pragma unroll
+                    for (int h = 0; h < (kWReg ? NQ : 1); ++h) wr[h] = w_e[wslot * NQ + h];
+                }
+#pragma unroll
+                for (int gg = 0; gg < G; ++gg) nvis[gg] = __ldg(p.n_row + r0 + gg);
+                gcur = cur.g;
             }
             const int a = (int)(it % ACC);
             aborted = aborted || *abort_flag;
@@ -354,89 +402,85 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
             }
             if (aborted) continue;
             tc_fence_after();
-            float sc[G];
+            float sc[TM][G];
             const float* wv = w_e + wslot * NQ;
-            constexpr int kChunks = NQ / 16 / G;      // 16-column TMEM loads per query row
-            const int nch = (p.H_I + 15) >> 4;        // chunks actually holding heads
 #pragma unroll
-            for (int gg = 0; gg < G; ++gg) {
-                // columns [gg*H_I, gg*H_I + H_I) of this accumulator; all loads in flight
-                // before one wait
-                uint32_t v[kChunks][16];
-                const uint32_t col = tmem_base + lane_addr + a * kAccCols + gg * p.H_I;
+            for (int hh = 0; hh < TM; ++hh) {
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c)
-                    if (c < nch) tmem_ld16(col + c * 16, v[c]);
-                tmem_ld_wait();
-                // four independent accumulation chains (heads h = 4m + j go to chain j)
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
-                const float* wg = wv + gg * p.H_I;
+                for (int gg = 0; gg < G; ++gg) {
+                    // this query row's kCols columns of half hh; all loads before one wait
+                    uint32_t v[kCols];
+                    const uint32_t col = tmem_base + lane_addr + a * kAccCols + hh * NQ + gg * kCols;
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    if (c < nch) {
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const float4 w4 = *reinterpret_cast<const float4*>(wg + c * 16 + k4 * 4);
-                            // heads past H_I carry weight 0 (the weights are zero-padded)
-                            s4[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[c][4 * k4 + 0]), 0.f), s4[0]);
-                            s4[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[c][4 * k4 + 1]), 0.f), s4[1]);
-                            s4[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[c][4 * k4 + 2]), 0.f), s4[2]);
-                            s4[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[c][4 * k4 + 3]), 0.f), s4[3]);
-                        }
+                    for (int c = 0; c < kCols / 16; ++c) {
+                        uint32_t (&vc)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16 * c);
+                        tmem_ld16(col + c * 16, vc);
                     }
+                    tmem_ld_wait();
+                    // four independent accumulation chains; padding columns have weight 0
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int h = 0; h < kCols; ++h) {
+                        const float wh = kWReg ? wr[kWReg ? h : 0] : wv[gg * kCols + h];
+                        s4[h & 3] = fmaf(wh, fmaxf(__uint_as_float(v[h]), 0.f), s4[h & 3]);
+                    }
+                    sc[hh][gg] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + 0.0f;
                 }
-                sc[gg] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + 0.0f;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[a]);
 
-            const int64_t j = jt * kTileRows + row;   // entry (or pool slot) index
 #pragma unroll
-            for (int gg = 0; gg < G; ++gg) {
-                const int r = r0 + gg;
-                bool vis;
-                if (!GATHER) {
-                    vis = j < __ldg(p.n_row + r);
-                } else {
-                    int pos = (j < p.P) ? __ldg(p.pool + (int64_t)r * p.P + j) : -1;
-                    vis = pos >= 0 && pos < __ldg(p.n_row + r);
-                }
-                const uint32_t key = score_key(sc[gg]);
-                if (vis) p.scores[(int64_t)r * p.ld_scores + j] = sc[gg];
-                {
-                    // scores cluster in a few bins: one shared atomic per distinct bin
-                    const uint32_t bin = vis ? (key >> 20) : 0xFFFFFFFFu;
-                    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                    if (vis && (lane == __ffs(peers) - 1))
-                        atomicAdd(&hist_e[gg * kBins + bin], (uint32_t)__popc(peers));
-                }
-                if (POOL) {
-                    uint32_t bk = vis ? key : 0u;
-                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
-                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
-                    bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
-                    const bool lead = (row & 7) == 0 && j < __ldg(p.n_row + r);
-                    if (lead) p.bkey[(int64_t)r * p.ld_bkey + (j >> 3)] = bk;
-                    const uint32_t bbin = lead ? (bk >> 20) : 0xFFFFFFFFu;
-                    const uint32_t peers = __match_any_sync(0xffffffffu, bbin);
-                    if (lead && (lane == __ffs(peers) - 1))
-                        atomicAdd(&bhist_e[bbin], (uint32_t)__popc(peers));
+            for (int hh = 0; hh < TM; ++hh) {
+                const int64_t j = jt * kRowsT + hh * 128 + row;   // entry (or pool slot)
+#pragma unroll
+                for (int gg = 0; gg < G; ++gg) {
+                    const int r = r0 + gg;
+                    bool vis;
+                    if (!GATHER) {
+                        vis = j < nvis[gg];
+                    } else {
+                        int pos = (j < p.P) ? __ldg(p.pool + (int64_t)r * p.P + j) : -1;
+                        vis = pos >= 0 && pos < nvis[gg];
+                    }
+                    const float scv = sc[hh][gg];
+                    const uint32_t key = score_key(scv);
+                    if (vis) p.scores[(int64_t)r * p.ld_scores + j] = scv;
+                    {
+                        // scores cluster in a few bins: one shared atomic per distinct bin
+                        const uint32_t bin = vis ? (key >> 20) : 0xFFFFFFFFu;
+                        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                        if (vis && (lane == __ffs(peers) - 1))
+                            atomicAdd(&hist_e[gg * kBins + bin], (uint32_t)__popc(peers));
+                    }
+                    if (POOL) {
+                        uint32_t bk = vis ? key : 0u;
+                        bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
+                        bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
+                        bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
+                        const bool lead = (row & 7) == 0 && j < nvis[gg];
+                        if (lead) p.bkey[(int64_t)r * p.ld_bkey + (j >> 3)] = bk;
+                        const uint32_t bbin = lead ? (bk >> 20) : 0xFFFFFFFFu;
+                        const uint32_t peers = __match_any_sync(0xffffffffu, bbin);
+                        if (lead && (lane == __ffs(peers) - 1))
+                            atomicAdd(&bhist_e[bbin], (uint32_t)__popc(peers));
+                    }
                 }
             }
         }
         // final flush
         epi_bar_sync(e);
-        if (cur >= 0) {
+        if (gcur >= 0) {
             for (int gg = 0; gg < G; ++gg)
                 for (int i = et; i < kBins; i += 128) {
                     const uint32_t v = hist_e[gg * kBins + i];
-                    if (v) atomicAdd(p.hist + (int64_t)(cur * G + gg) * kBins + i, v);
+                    if (v) atomicAdd(p.hist + (int64_t)(gcur * G + gg) * kBins + i, v);
                 }
             if (POOL)
                 for (int i = et; i < kBins; i += 128) {
                     const uint32_t v = bhist_e[i];
-                    if (v) atomicAdd(p.bhist + (int64_t)(cur * G) * kBins + i, v);
+                    if (v) atomicAdd(p.bhist + (int64_t)(gcur * G) * kBins + i, v);
                 }
         }
     }
@@ -452,7 +496,8 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
 // mode counts pool slots instead of entries for the tile prefix.
 __global__ void __launch_bounds__(1024) prep_rows_kernel(
     int rows, int T, int G, const int32_t* n_vis0, const int32_t* q_pos0, int ratio,
-    int64_t cap, int P_gather, int32_t* n_row, int64_t* prefix, int32_t* status) {
+    int64_t cap, int P_gather, int tile_rows, int32_t* n_row, int64_t* prefix,
+    int32_t* status) {
     __shared__ int64_t warp_sums[32];
     __shared__ int64_t carry;
     if (threadIdx.x == 0) carry = 0;
@@ -480,7 +525,7 @@ __global__ void __launch_bounds__(1024) prep_rows_kernel(
         int64_t tiles = 0;
         if (gi < ngroups) {
             const int64_t n = P_gather > 0 ? P_gather : n_row[gi * G + G - 1];
-            tiles = (n + kTileRows - 1) / kTileRows;
+            tiles = (n + tile_rows - 1) / tile_rows;
         }
         // block-wide exclusive scan of `tiles`
         int64_t v = tiles;
@@ -552,14 +597,28 @@ static int num_sms() {
     return n;
 }
 
-template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL>
+// Largest stage count (<= 8) whose shared-memory plan fits in one SM.
+template <int NQ, int ESZ, int ACC, int G, int EPI, bool POOL, int TM>
+constexpr int pick_stages() {
+    return ScanSmem<NQ, ESZ, 8, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 8
+         : ScanSmem<NQ, ESZ, 6, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 6
+         : ScanSmem<NQ, ESZ, 4, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 4
+         : ScanSmem<NQ, ESZ, 3, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 3 : 2;
+}
+
+template <int NQ, int ESZ, int G, bool GATHER, bool POOL>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
-    // two epilogue groups when the per-tile epilogue is short (one query row per tile)
+    // one query row per tile: two epilogue groups and 256-key tiles
     constexpr int EPI = (G == 1) ? 2 : 1;
-    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL>;
+    constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 2 : 1;
+    constexpr int kAccCols = TM * NQ;
+    constexpr int ACC = kAccCols <= 128 ? 4 : kAccCols <= 256 ? 2 : 1;
+    static_assert(ACC % EPI == 0, "accumulators per epilogue group");
+    constexpr int STAGES = pick_stages<NQ, ESZ, ACC, G, EPI, POOL, TM>();
+    using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
-    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL, EPI>;
+    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL, EPI, TM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kAlloc);
     if (e != cudaSuccess) return e;
@@ -576,7 +635,8 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     memset(&mk, 0, sizeof mk);
     memset(&mq, 0, sizeof mq);
     if (!make_map(&mq, a.q, (int64_t)a.rows * a.H_I, esz, NQ)) return cudaErrorInvalidValue;
-    if (!a.gather && !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, kTileRows))
+    if (!a.gather &&
+        !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, scan_tile_rows(a.G, a.gather, esz)))
         return cudaErrorInvalidValue;
     ScanParams p;
     p.rows = a.rows;
@@ -598,59 +658,46 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     p.keys = reinterpret_cast<const uint8_t*>(a.k);
     p.status = a.status;
 
-#define CSA2_SCAN(NQv, ESZv, STv, ACCv, Gv, GA, PO) \
-    return launch_scan_t<NQv, ESZv, STv, ACCv, Gv, GA, PO>(mk, mq, p, st)
+#define CSA2_SCAN(NQv, ESZv, Gv, GA, PO) return launch_scan_t<NQv, ESZv, Gv, GA, PO>(mk, mq, p, st)
+#define CSA2_SCAN_NQ(ESZv, GA, PO)                    \
+    do {                                              \
+        if (NQ <= 16) CSA2_SCAN(16, ESZv, 1, GA, PO); \
+        if (NQ <= 32) CSA2_SCAN(32, ESZv, 1, GA, PO); \
+        if (NQ <= 64) CSA2_SCAN(64, ESZv, 1, GA, PO); \
+        CSA2_SCAN(128, ESZv, 1, GA, PO);              \
+    } while (0)
 
     if (a.G == 1) {
         if (a.gather) {
-            if (esz == 1) {
-                if (NQ <= 32) CSA2_SCAN(32, 1, 4, 4, 1, true, false);
-                if (NQ <= 64) CSA2_SCAN(64, 1, 4, 4, 1, true, false);
-                CSA2_SCAN(128, 1, 4, 2, 1, true, false);
-            } else {
-                if (NQ <= 32) CSA2_SCAN(32, 2, 2, 4, 1, true, false);
-                if (NQ <= 64) CSA2_SCAN(64, 2, 2, 4, 1, true, false);
-                CSA2_SCAN(128, 2, 2, 2, 1, true, false);
-            }
+            if (esz == 1) CSA2_SCAN_NQ(1, true, false);
+            CSA2_SCAN_NQ(2, true, false);
         }
         if (esz == 1) {
-            if (a.pool_build) {
-                if (NQ <= 16) CSA2_SCAN(16, 1, 8, 4, 1, false, true);
-                if (NQ <= 32) CSA2_SCAN(32, 1, 8, 4, 1, false, true);
-                if (NQ <= 64) CSA2_SCAN(64, 1, 8, 4, 1, false, true);
-                CSA2_SCAN(128, 1, 6, 2, 1, false, true);
-            }
-            if (NQ <= 16) CSA2_SCAN(16, 1, 8, 4, 1, false, false);
-            if (NQ <= 32) CSA2_SCAN(32, 1, 8, 4, 1, false, false);
-            if (NQ <= 64) CSA2_SCAN(64, 1, 8, 4, 1, false, false);
-            CSA2_SCAN(128, 1, 6, 2, 1, false, false);
-        } else {
-            if (a.pool_build) {
-                if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, true);
-                if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, true);
-                if (NQ <= 64) CSA2_SCAN(64, 2, 3, 4, 1, false, true);
-                CSA2_SCAN(128, 2, 2, 2, 1, false, true);
-            }
-            if (NQ <= 16) CSA2_SCAN(16, 2, 4, 4, 1, false, false);
-            if (NQ <= 32) CSA2_SCAN(32, 2, 4, 4, 1, false, false);
-            if (NQ <= 64) CSA2_SCAN(64, 2, 4, 4, 1, false, false);
-            CSA2_SCAN(128, 2, 3, 2, 1, false, false);
+            if (a.pool_build) CSA2_SCAN_NQ(1, false, true);
+            CSA2_SCAN_NQ(1, false, false);
         }
+        if (a.pool_build) CSA2_SCAN_NQ(2, false, true);
+        CSA2_SCAN_NQ(2, false, false);
     } else if (a.G == 4 && NQ == 256 && esz == 1 && !a.gather && !a.pool_build) {
-        CSA2_SCAN(256, 1, 4, 2, 4, false, false);
+        CSA2_SCAN(256, 1, 4, false, false);
     } else if (a.G == 2 && NQ <= 128 && esz == 1 && !a.gather && !a.pool_build) {
-        CSA2_SCAN(128, 1, 6, 2, 2, false, false);
+        CSA2_SCAN(128, 1, 2, false, false);
     }
+#undef CSA2_SCAN_NQ
 #undef CSA2_SCAN
     return cudaErrorNotSupported;
 }
 
+int scan_tile_rows(int G, bool gather, int esz) {
+    return (G == 1 && !gather && esz == 1) ? 2 * kTileRows : kTileRows;
+}
+
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
                              const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
-                             int32_t* n_row, int64_t* prefix, int32_t* status,
+                             int tile_rows, int32_t* n_row, int64_t* prefix, int32_t* status,
                              cudaStream_t st) {
     prep_rows_kernel<<<1, 1024, 0, st>>>(rows, T, G, n_vis0, q_pos0, ratio, cap, P_gather,
-                                         n_row, prefix, status);
+                                         tile_rows, n_row, prefix, status);
     return cudaGetLastError();
 }
 
