@@ -109,11 +109,12 @@ __device__ __forceinline__ uint32_t e2m1x2_to_h2_tc(uint32_t byte) {
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// Transposed logit tile S[h][r] (fp32, 128 rows per head): within each 32-row quarter q the
-// row is rotated by 8q + (h mod 8), so both the row-per-thread writes and the
-// (head, quarter)-per-thread reads touch 32 distinct banks.
+// Logit tile S[r][h] (fp32, 64 heads per row) with the 16-byte chunk (4 heads) index XOR-ed
+// by ((r / 32) * 2) ^ (r mod 8): one thread per row writes it with 16-byte stores, and the
+// (head, 32-row quarter)-per-thread reads of the softmax touch 32 distinct banks.
+__device__ __forceinline__ int s_swz(int r) { return ((r >> 5) << 1) ^ (r & 7); }
 __device__ __forceinline__ int s_idx(int h, int r) {
-    return h * kRows + (r & ~31) + (((r & 31) + 8 * (r >> 5) + (h & 7)) & 31);
+    return r * kHeads + ((((h >> 2) ^ s_swz(r)) & 15) << 2) + (h & 3);
 }
 
 // Gather + dequantise rows [ch*128, ch*128+128) of query row `qrow` into X (all 256 threads:
@@ -268,54 +269,63 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
     if (tid < kHeads) m_s[tid] = -INFINITY;
 
     // ---- query: per-head power-of-two rescale into fp16, K-major swizzled slabs --------
-    auto load_q = [&]() {
-        uint4 raw[8][2];   // this warp's 8 heads, all loads in flight before use
+    // (1) the raw bf16 rows [64 heads x 1 KiB] are fetched asynchronously into the Q tile,
+    // overlapping the row gather; (2) every thread reads its (head, 128-channel quarter) into
+    // registers, the block syncs, and the scaled fp16 values are written back swizzled.
+    auto q_prefetch = [&]() {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int h = warp + 8 * k;
-            if (h < a.H) {
-                const uint4* src = reinterpret_cast<const uint4*>(
-                    a.q + ((int64_t)qrow * a.H + h) * kD + lane * 16);
-                raw[k][0] = __ldg(src);
-                raw[k][1] = __ldg(src + 1);
-            } else {
-                raw[k][0] = raw[k][1] = make_uint4(0, 0, 0, 0);
-            }
+        for (int k = 0; k < 16; ++k) {
+            const int c = tid + 256 * k;          // 16-byte chunk of the 64 KiB tile
+            const int h = c >> 6, off = (c & 63) * 16;
+            const uint32_t dst = sQ + h * 1024 + off;
+            if (h < a.H)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                             "l"(reinterpret_cast<const uint8_t*>(a.q + ((int64_t)qrow * a.H + h) * kD) + off)
+                             : "memory");
+            else
+                st_shared_v4(dst, 0u, 0u, 0u, 0u);
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto q_convert = [&]() {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        const int h = tid >> 2, qq = tid & 3;   // channels [128 qq, 128 qq + 128) of head h
+        uint4 raw[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int h = warp + 8 * k;
-            float v[16];
-            const uint32_t w8[8] = {raw[k][0].x, raw[k][0].y, raw[k][0].z, raw[k][0].w,
-                                    raw[k][1].x, raw[k][1].y, raw[k][1].z, raw[k][1].w};
+        for (int k = 0; k < 16; ++k)
+            raw[k] = *reinterpret_cast<const uint4*>(sm + L::kQ + h * 1024 + qq * 256 + k * 16);
+        float amax = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                v[2 * e] = __uint_as_float(w8[e] << 16);
-                v[2 * e + 1] = __uint_as_float(w8[e] & 0xFFFF0000u);
-            }
-            float amax = 0.f;
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
 #pragma unroll
-            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            int shift = 0;
-            if (amax > 0.f) {
-                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                shift = min(126, max(-126, 14 - ex));
-            }
-            const float mul = __int_as_float((127 + shift) << 23);   // 2^shift, exact
-            uint32_t hw[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                hw[e] = h2_bits(__floats2half2_rn(v[2 * e] * mul, v[2 * e + 1] * mul));
-            // lane owns channels [16 lane, 16 lane + 16): slab lane/4, chunks 2(lane%4), +1
-            const uint32_t slab = sQ + (lane >> 2) * L::kQSlab;
-            const int cc = (lane & 3) * 2;
-            st_shared_v4(slab + slab_off(h, cc), hw[0], hw[1], hw[2], hw[3]);
-            st_shared_v4(slab + slab_off(h, cc + 1), hw[4], hw[5], hw[6], hw[7]);
-            if (lane == 0) qf[h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
+            for (int e = 0; e < 4; ++e)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
+                                         fabsf(__uint_as_float(w4[e] & 0xFFFF0000u))));
         }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int shift = 0;
+        if (amax > 0.f) {
+            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+            shift = min(126, max(-126, 14 - ex));
+        }
+        const float mul = __int_as_float((127 + shift) << 23);   // 2^shift, exact
+        __syncthreads();   // every raw read is done before the swizzled writes begin
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+            uint32_t hw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                hw[e] = h2_bits(__floats2half2_rn(__uint_as_float(w4[e] << 16) * mul,
+                                                  __uint_as_float(w4[e] & 0xFFFF0000u) * mul));
+            // channels 128 qq + 8 k .. +8: slab 2 qq + k / 8, chunk k % 8
+            st_shared_v4(sQ + (2 * qq + (k >> 3)) * L::kQSlab + slab_off(h, k & 7), hw[0], hw[1],
+                         hw[2], hw[3]);
+        }
+        if (qq == 0) qf[h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
     };
 
     tc_fence_before();
@@ -334,8 +344,9 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
 
     // S^T for chunk ch -> transposed logits Ssm[h][r] (log2 domain, -inf for empty rows)
     auto scores = [&](int ch) {
+        q_prefetch();
         load_chunk(a, qrow, b, t, ch, sX, rvalid);
-        load_q();
+        q_convert();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
         if (tid == 0) {
@@ -353,12 +364,15 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
             for (int c = 0; c < 4; ++c) tmem_ld16(tmem + quad + 16 * c, v[c]);
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int h = 16 * c + k;
-                    Ssm[s_idx(h, r)] = valid ? __uint_as_float(v[c][k]) * qf[h] : -INFINITY;
-                }
+            for (int c4 = 0; c4 < 16; ++c4) {   // heads 4 c4 .. 4 c4 + 3
+                float4 o;
+                const float4 f = *reinterpret_cast<const float4*>(qf + 4 * c4);
+                o.x = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 0]) * f.x : -INFINITY;
+                o.y = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 1]) * f.y : -INFINITY;
+                o.z = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 2]) * f.z : -INFINITY;
+                o.w = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 3]) * f.w : -INFINITY;
+                *reinterpret_cast<float4*>(Ssm + r * kHeads + (((c4 ^ s_swz(r)) & 15) << 2)) = o;
+            }
         }
         tc_fence_before();
         __syncthreads();
@@ -455,8 +469,8 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
                         const int hh = 16 * k + e;
                         if (hh < a.H) {
                             const float l = l_s[hh];
-                            a.out[((int64_t)qrow * a.H + hh) * kD + c] =
-                                l > 0.f ? __uint_as_float(v[k][e]) / l : 0.f;
+                            const float inv = l > 0.f ? 1.f / l : 0.f;
+                            a.out[((int64_t)qrow * a.H + hh) * kD + c] = __uint_as_float(v[k][e]) * inv;
                         }
                     }
             } else {
