@@ -225,6 +225,32 @@ class Decode:
         return tot, scan
 
 
+def flush_l2(buf, k):
+    """Evict L2 between timed steps: write a buffer twice the size of L2, then read it back
+    so that the dirty lines are written to HBM here and not during the next step."""
+    buf.fill_(k & 0xFF)
+    torch.sum(buf.view(torch.int64))
+
+
+def capture_steps(state, events, stream):
+    """One CUDA graph per timed step: the step's library calls, with that step's pair of
+    scan events recorded inside (as external event nodes)."""
+    graphs = []
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        state.step()                      # warm the side stream
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    for ev in events:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            state.step(scan_events=ev, stream=side)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
 def max_over_ranks(ms, pg, dev):
     """Device-timed milliseconds of this rank -> the slowest rank's (every rank gets it)."""
     if pg is None:
@@ -242,6 +268,127 @@ def job_throughput(batch_per_rank, world, steps, total_ms):
 def rank_seed(seed, rank):
     """Each rank draws its own independent batch."""
     return seed + 7919 * rank
+
+
+class Prefill:
+    """Device-resident state of the chunked-prefill workload plus its per-step inputs."""
+
+    def __init__(self, w, seed, dev):
+        self.w = w
+        self.dev = dev
+        self.seed = seed
+        B, T, cap, K = w.B, w.T, w.cap, w.K
+        self.tau = 1.0 / math.sqrt(synth.D_MAIN)
+        self.L = synth.layer_inputs(w, 0, seed, dev)
+        self.k_I, _ = synth.indexer_keys(w, seed, dev)
+        self.n_old = w.ctx // w.ratio
+        self.codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
+        src = torch.stack([_main_rows(w, seed, b, dev) for b in range(B)])
+        csa2.quantize_kv(src[:, :self.n_old], torch.zeros(B, dtype=torch.int32, device=dev),
+                         self.codes, self.scales)
+        self.kv_new = src[:, self.n_old:].contiguous()
+        del src
+        self.dst = torch.full((B,), self.n_old, dtype=torch.int32, device=dev)
+        self.q_pos0 = synth.prefill_positions(w, dev)
+        self.idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, T, w.H, synth.D_MAIN), dtype=torch.float32, device=dev)
+        self.ws = csa2.new_workspace(csa2.workspace_bytes(0, B, T, w.H_I, cap, K))
+        self.wsa = csa2.new_workspace(csa2.workspace_bytes(2, B, T, w.H, cap, K))
+        torch.cuda.synchronize()
+
+    def step(self, scan_events=None, attn_events=None, stream=None):
+        w = self.w
+        csa2.quantize_kv(self.kv_new, self.dst, self.codes, self.scales,
+                         status=self.ws[:4].view(torch.int32), stream=stream)
+        if scan_events is not None:
+            csa2.set_stage_events(*scan_events)
+        csa2.index_score_topk("full", self.L["q_I"], self.L["w"], self.k_I, w.K, self.idx,
+                              self.ws, q_pos0=self.q_pos0, ratio=w.ratio, stream=stream)
+        if attn_events is not None:
+            attn_events[0].record(stream or torch.cuda.current_stream())
+        csa2.sparse_attn_prefill(self.L["q"], self.codes, self.scales, self.idx, self.L["swa"],
+                                 self.out, self.wsa, synth.WINDOW, q_pos0=self.q_pos0,
+                                 scale=self.tau, stream=stream)
+        if attn_events is not None:
+            attn_events[1].record(stream or torch.cuda.current_stream())
+
+    def flops(self):
+        """Algorithmic FLOPs of one step: the indexer over every causally visible
+        (token, entry) pair and the attention (S and P x V) over K + W rows per token."""
+        w = self.w
+        vis = sum((w.ctx + t + 1) // w.ratio for t in range(w.T))
+        scan = w.B * vis * w.H_I * synth.D_IDX * 2
+        attn = w.B * w.T * w.H * (w.K + synth.WINDOW) * synth.D_MAIN * 2 * 2
+        return scan, attn
+
+
+def prefill_main(args, w, dev, rank, world):
+    state = Prefill(w, rank_seed(args.seed, rank), dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        state.step()
+    torch.cuda.synchronize()
+    assert csa2.read_device_status(state.ws) == 0 and csa2.read_device_status(state.wsa) == 0
+    mk = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ev = [mk() for _ in range(args.steps)]
+    sev = [mk() for _ in range(args.steps)]
+    aev = [mk() for _ in range(args.steps)]
+    for pair in sev + aev:
+        pair[0].record(stream)
+        pair[1].record(stream)
+    torch.cuda.synchronize()
+    clocks = Clocks(local_rank())
+    clocks.start()
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        state.step(scan_events=sev[k], attn_events=aev[k])
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    scan_ms = sum(a.elapsed_time(b) for a, b in sev) / args.steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in aev) / args.steps
+    scan_f, attn_f = state.flops()
+    bf16 = measured_bf16_tflops()
+    tokens = w.B * w.T * args.steps
+    line = {
+        "metric": "CSA2 chunked prefill tokens/s (FP8 indexer + sparse attention), 1 B200",
+        "value": tokens / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 indexer / fp16 attention (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "new_tokens": w.T, "cached_tokens": w.ctx,
+                   "ratio": w.ratio, "topk": w.K, "indexer_heads": w.H_I, "query_heads": w.H,
+                   "window": synth.WINDOW, "l2": "inputs larger than L2"},
+        "roofline": {"kernel": "csa2 indexer scan (tcgen05 kind::f8f6f4)", "bound": "tensor",
+                     "achieved": scan_f / (scan_ms / 1e3) / 1e12,
+                     "peak": 2 * bf16, "unit": "TFLOP/s",
+                     "frac": scan_f / (scan_ms / 1e3) / 1e12 / (2 * bf16),
+                     "peak_source": "measured bf16 x 2 (FP8/bf16 nominal ratio)",
+                     "flops_per_launch": scan_f, "avg_launch_ms": scan_ms, "traffic": None},
+        "attention": {"bound": "tensor", "achieved": attn_f / (attn_ms / 1e3) / 1e12,
+                      "peak": bf16, "unit": "TFLOP/s",
+                      "frac": attn_f / (attn_ms / 1e3) / 1e12 / bf16,
+                      "flops_per_call": attn_f, "avg_call_ms": attn_ms},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def local_rank():
+    return int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def measured_bf16_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
 
 
 def csa2_attn_splits(w):
@@ -326,6 +473,8 @@ def main():
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -343,8 +492,12 @@ def main():
                                 device_id=dev)
         pg = dist
     w = synth.WORKLOADS[args.workload]
-    if w.kind != "decode":
-        raise SystemExit("bench.py times the decode path; prefill is covered by the tests")
+    if w.kind == "prefill":
+        prefill_main(args, w, dev, rank, world)
+        if pg:
+            pg.barrier()
+            pg.destroy_process_group()
+        return
     state = Decode(w, rank_seed(args.seed, rank), dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -363,14 +516,20 @@ def main():
     for a, b in sev:           # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
+    # Each timed step is one CUDA-graph replay of the whole step (captured once per step so
+    # that every replay records its own scan events): launches reach the GPU back to back.
+    graphs = capture_steps(state, sev, stream) if not args.eager else None
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     clocks.start()
     for k in range(args.steps):
-        flush.fill_(k & 0xFF)                   # evict L2 between steps (outside the events)
+        flush_l2(flush, k)                      # evict L2 between steps (outside the events)
         ev[k][0].record(stream)
-        state.step(scan_events=sev[k])
+        if graphs:
+            graphs[k].replay()
+        else:
+            state.step(scan_events=sev[k])
         ev[k][1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -389,12 +548,23 @@ def main():
     bo = sum(x.numel() * x.element_size() for x in h_out)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+    g_plain = None
+    if graphs:
+        g_plain = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.graph(g_plain, stream=side):
+            state.step(stream=side)
+        torch.cuda.synchronize()
     for k in range(args.steps):
-        flush.fill_(k & 0xFF)
+        flush_l2(flush, k)
         e2e_ev[k][0].record(stream)
         for d, h in zip(ins, h_in):
             d.copy_(h, non_blocking=True)
-        state.step()
+        if g_plain:
+            g_plain.replay()
+        else:
+            state.step()
         for h, o in zip(h_out, outs):
             h.copy_(o, non_blocking=True)
         e2e_ev[k][1].record(stream)
@@ -428,11 +598,12 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3/fp4/fp16 (fp32 accumulate)", "data": "synthetic",
             "config": {"workload": args.workload, "batch_per_gpu": w.B, "context_tokens": w.ctx,
+                       "launch": "eager" if args.eager else "cuda graph replay per step",
                        "ratio": w.ratio, "compressed_entries": w.N, "topk": w.K,
                        "indexer_heads": w.H_I, "indexer_dtype": w.idx_dtype, "query_heads": w.H,
                        "window": synth.WINDOW, "layers": list(w.layers),
                        "parallelism": f"dp{world} (independent batches)",
-                       "l2": "flushed between steps (256 MiB write)"},
+                       "l2": "flushed between steps (256 MiB write + read, outside the timed events)"},
             "hbm_gbs_step": alg_bytes / (per_step_ms / 1e3) / 1e9,
             "roofline": {"kernel": "csa2 indexer scan (tcgen05, FP8 keys)", "bound": "hbm",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -37,9 +37,10 @@ struct TopkPlan {
     size_t total;
 };
 
+// Query rows sharing one key tile in prefill: two rows of 64 heads fill an N = 128 MMA
+// (full tensor rate) and leave the epilogue two groups of warps.
 static int choose_group(int T, int H_I, int esz, bool prefill, bool pool) {
     if (!prefill || pool || esz != 1) return 1;
-    if (H_I == 64 && T % 4 == 0) return 4;
     if (2 * H_I <= 128 && H_I % 16 == 0 && T % 2 == 0) return 2;
     return 1;
 }
@@ -294,9 +295,14 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
     sl.status = status;
     const cudaEvent_t ev0 = g_stage_ev[0], ev1 = g_stage_ev[1];
     g_stage_ev[0] = g_stage_ev[1] = nullptr;
-    if (ev0 && cudaEventRecord(ev0, st) != cudaSuccess) return CSA2_ERR_CUDA;
+    // inside a stream capture the events become external record nodes (usable for timing)
+    cudaStreamCaptureStatus capst = cudaStreamCaptureStatusNone;
+    if ((ev0 || ev1) && cudaStreamIsCapturing(st, &capst) != cudaSuccess) return CSA2_ERR_CUDA;
+    const unsigned ev_flags =
+        capst == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    if (ev0 && cudaEventRecordWithFlags(ev0, st, ev_flags) != cudaSuccess) return CSA2_ERR_CUDA;
     e = launch_index_scan(sl, st);
-    if (ev1 && e == cudaSuccess) e = cudaEventRecord(ev1, st);
+    if (ev1 && e == cudaSuccess) e = cudaEventRecordWithFlags(ev1, st, ev_flags);
     if (e == cudaErrorNotSupported) return CSA2_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
 

@@ -601,7 +601,9 @@ static int num_sms() {
 template <int NQ, int ESZ, int ACC, int G, int EPI, bool POOL, int TM>
 constexpr int pick_stages() {
     return ScanSmem<NQ, ESZ, 8, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 8
+         : ScanSmem<NQ, ESZ, 7, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 7
          : ScanSmem<NQ, ESZ, 6, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 6
+         : ScanSmem<NQ, ESZ, 5, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 5
          : ScanSmem<NQ, ESZ, 4, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 4
          : ScanSmem<NQ, ESZ, 3, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 3 : 2;
 }
@@ -609,11 +611,12 @@ constexpr int pick_stages() {
 template <int NQ, int ESZ, int G, bool GATHER, bool POOL>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
-    // one query row per tile: two epilogue groups and 256-key tiles
-    constexpr int EPI = (G == 1) ? 2 : 1;
+    // 256-key tiles for one FP8 query row per tile; two epilogue groups whenever the TMEM
+    // accumulators split evenly between them
     constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 2 : 1;
     constexpr int kAccCols = TM * NQ;
     constexpr int ACC = kAccCols <= 128 ? 4 : kAccCols <= 256 ? 2 : 1;
+    constexpr int EPI = (ACC % 2 == 0 && G <= 2) ? 2 : 1;
     static_assert(ACC % EPI == 0, "accumulators per epilogue group");
     constexpr int STAGES = pick_stages<NQ, ESZ, ACC, G, EPI, POOL, TM>();
     using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;

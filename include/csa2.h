@@ -247,7 +247,9 @@ CSA2_API int csa2_version(void);
 /* Benchmark hook: when set, the next csa2_index_score_topk() issued from the calling host
  * thread records `ev_start` (a cudaEvent_t passed as void*) on its stream right before
  * its indexer-scan kernel launch and `ev_stop` right after it, then forgets both. The
- * setting is per host thread and consumed by one call; NULL, NULL clears it. */
+ * setting is per host thread and consumed by one call; NULL, NULL clears it. During a stream
+ * capture the two records become external event nodes of the graph, so replays of the graph
+ * can be timed with them. */
 CSA2_API csa2_status_t csa2_set_stage_events(void* ev_start, void* ev_stop);
 
 /* Test hook for the bounded waits: launches one block that waits on an mbarrier that is
