@@ -185,13 +185,14 @@ class Decode:
                                     stream=stream)
 
     def launches_per_step(self):
+        """Kernels of this library per step (memsets excluded)."""
         n = 1  # quantize
         for m in self.w.layers:
             if m == "full":
-                n += 4 + (2 if self.w.pool else 0)   # prep, scan, collect, finalize (+ pool)
+                n += 3 + (1 if self.w.pool else 0)   # prep, scan, Top-K (+ pool Top-K)
             elif m == "reindex":
-                n += 4
-            n += 1 + (1 if csa2_attn_splits(self.w) > 1 else 0)
+                n += 3
+            n += 2 + (1 if csa2_attn_splits(self.w) > 1 else 0)   # stage, attention (+ merge)
         return n
 
     def step_inputs(self):
@@ -372,7 +373,7 @@ def prefill_main(args, w, dev, rank, world):
                       "peak": bf16, "unit": "TFLOP/s",
                       "frac": attn_f / (attn_ms / 1e3) / 1e12 / bf16,
                       "flops_per_call": attn_f, "avg_call_ms": attn_ms},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": 5 * args.steps,   # quantize, prep, scan, Top-K, attention
         "clocks": clk,
     }
     if rank == 0:
@@ -393,7 +394,7 @@ def measured_bf16_tflops():
 
 def csa2_attn_splits(w):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    nch = (w.K + synth.WINDOW + 63) // 64
+    nch = (w.K + synth.WINDOW + 127) // 128
     ns = min(nch, (2 * sms + w.B - 1) // w.B)
     cps = (nch + ns - 1) // ns
     return (nch + cps - 1) // cps

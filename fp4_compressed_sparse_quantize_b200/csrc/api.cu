@@ -88,9 +88,15 @@ static TopkPlan plan_topk(int B, int T, int H_I, int esz, int64_t row_len, int K
     return p;
 }
 
-static size_t attn_ws_bytes(int Q, int H, int nsplit) {
-    size_t b = kStatusBytes;
-    if (nsplit > 1) b += sizeof(float) * (size_t)Q * nsplit * H * (CSA2_D_MAIN + 2);
+// Attention workspace: status word, split partials (decode with nsplit > 1), and for decode
+// the staging area of the dequantised rows (`rows` = K + W per query).
+static size_t attn_partial_bytes(int Q, int H, int nsplit) {
+    return nsplit > 1 ? align_up(sizeof(float) * (size_t)Q * nsplit * H * (CSA2_D_MAIN + 2), 256)
+                      : 0;
+}
+static size_t attn_ws_bytes(int Q, int H, int nsplit, int stage_rows) {
+    size_t b = kStatusBytes + attn_partial_bytes(Q, H, nsplit);
+    if (stage_rows > 0) b += attention_stage_bytes(Q, stage_rows);
     return b;
 }
 
@@ -195,9 +201,10 @@ size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t cap, int 
             return std::max(p.total, p2.total);
         }
         case CSA2_OP_SPARSE_ATTN_DECODE:
-            return attn_ws_bytes(B, H, attn_split_bound(B, K));
+            // sized for windows of up to 1024 rows
+            return attn_ws_bytes(B, H, attn_split_bound(B, K), K + 1024);
         case CSA2_OP_SPARSE_ATTN_PREFILL:
-            return attn_ws_bytes(B * T, H, 1);
+            return attn_ws_bytes(B * T, H, 1, 0);
     }
     return 0;
 }
@@ -372,7 +379,8 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
     const int64_t Q = (int64_t)B * T;
     if (Q > 2147483647) return CSA2_ERR_UNSUPPORTED;
     const int nsplit = attention_splits((int)Q, K, W, prefill);
-    if (ws_bytes < attn_ws_bytes((int)Q, H, nsplit)) return CSA2_ERR_WORKSPACE;
+    const int stage_rows = prefill ? 0 : K + W;
+    if (ws_bytes < attn_ws_bytes((int)Q, H, nsplit, stage_rows)) return CSA2_ERR_WORKSPACE;
     AttnLaunch l;
     memset(&l, 0, sizeof l);
     l.Q = (int)Q;
@@ -393,6 +401,9 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
     l.out = out;
     l.nsplit = nsplit;
     l.partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kStatusBytes);
+    l.stage = stage_rows > 0 ? reinterpret_cast<uint8_t*>(ws) + kStatusBytes +
+                                   attn_partial_bytes((int)Q, H, nsplit)
+                             : nullptr;
     l.status = reinterpret_cast<int32_t*>(ws);
     return cuda_status(launch_attention(l, reinterpret_cast<cudaStream_t>(stream)));
 }

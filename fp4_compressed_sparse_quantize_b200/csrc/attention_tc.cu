@@ -37,6 +37,9 @@
 //      were split over several CTAs.
 // A CTA with several chunks (prefill) first sweeps them for the exact per-head maximum,
 // then sweeps again to accumulate P x V, so no accumulator is ever rescaled.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "csa2_common.cuh"
 #include "csa2_internal.h"
 
@@ -64,6 +67,9 @@ struct TcAttnDev {
     float* partial;
     int nsplit, nchunks, chunks_per_split;
     int32_t* status;
+    // staged decode: rows / query already dequantised by attn_stage_kernel
+    const int32_t* st_valid;   // [Q][K + W] row kinds (0 = empty)
+    const float* st_qf;        // [Q][64] logit factors
 };
 
 struct TcSmem {
@@ -80,8 +86,8 @@ struct TcSmem {
     static constexpr int kM = kQf + 256;                  // 64 floats
     static constexpr int kL = kM + 256;                   // 64 floats
     static constexpr int kValid = kL + 256;               // 128 ints
-    static constexpr int kBar = kValid + 512;             // 2 mbarriers
-    static constexpr int kTmem = kBar + 16;
+    static constexpr int kBar = kValid + 512;             // 3 mbarriers
+    static constexpr int kTmem = kBar + 24;
     static constexpr int kBytes = kTmem + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
@@ -239,7 +245,102 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sX, uint32_t sP
     }
 }
 
-__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
+// Decode pre-pass: every selected main-KV row and window row of every query, dequantised to
+// fp16 rows [Q][K + W][512] (exact), plus each query's heads rescaled to fp16 [Q][64][512] and
+// their logit factors. One warp per row or head, 16 channels per lane, coalesced 1 KiB stores.
+__global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __half* __restrict__ xg,
+                                                         __half* __restrict__ qg,
+                                                         float* __restrict__ qfg,
+                                                         int32_t* __restrict__ validg,
+                                                         int row_blocks) {
+    const int b = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = a.K + a.W;
+    if ((int)blockIdx.y < row_blocks) {
+        const int r = blockIdx.y * 8 + warp;
+        if (r >= rows) return;
+        int kind = 0;
+        uint32_t hv[8];
+        if (r < a.K) {
+            const int32_t e = __ldg(a.idx + (int64_t)b * a.K + r);
+            if (e >= 0 && e < a.cap) {
+                kind = 1;
+                const int64_t ent = (int64_t)b * a.cap + e;
+                const uint2 cb = __ldg(reinterpret_cast<const uint2*>(a.codes + ent * CSA2_ENTRY_CODE_BYTES) + lane);
+                const uint8_t sb = __ldg(a.scales + ent * CSA2_ENTRY_SCALE_BYTES + lane);
+                const __half2 s2 = __half2half2(__float2half_rn(e4m3_to_float(sb)));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t byte = ((k < 4 ? cb.x : cb.y) >> (8 * (k & 3))) & 0xFFu;
+                    uint32_t h2 = e2m1x2_to_h2_tc(byte);
+                    hv[k] = h2_bits(__hmul2(*reinterpret_cast<__half2*>(&h2), s2));
+                }
+            } else if (e != -1 && lane == 0) {
+                set_status(a.status, CSA2_DEV_BAD_INDEX);
+            }
+        } else {
+            const int v = r - a.K;   // window row 0..W-1, oldest first
+            const int nv = a.swa_valid ? __ldg(a.swa_valid + b) : a.W;
+            if (v >= a.W - nv) {
+                kind = 2;
+                const uint4 eb = __ldg(reinterpret_cast<const uint4*>(a.swa + ((int64_t)b * a.W + v) * kD) + lane);
+                const uint32_t ew[4] = {eb.x, eb.y, eb.z, eb.w};
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    hv[k] = h2_bits(e4m3x2_to_half2((uint16_t)(ew[k >> 1] >> (16 * (k & 1)))));
+            }
+        }
+        if (kind == 0) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) hv[k] = 0u;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(xg + ((int64_t)b * rows + r) * kD + lane * 16);
+        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        if (lane == 0) validg[(int64_t)b * rows + r] = kind;
+        return;
+    }
+    // heads: per-head power-of-two rescale into fp16
+    const int h = ((int)blockIdx.y - row_blocks) * 8 + warp;
+    if (h >= kHeads) return;
+    float v[16];
+    float amax = 0.f;
+    if (h < a.H) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.H + h) * kD + lane * 16);
+        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+        const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            v[2 * e] = __uint_as_float(w8[e] << 16);
+            v[2 * e + 1] = __uint_as_float(w8[e] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int shift = 0;
+    if (amax > 0.f) {
+        const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+        shift = min(126, max(-126, 14 - ex));
+    }
+    const float mul = __int_as_float((127 + shift) << 23);   // 2^shift, exact
+    uint32_t hw[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hw[e] = h2_bits(__floats2half2_rn(v[2 * e] * mul, v[2 * e + 1] * mul));
+    uint4* dst = reinterpret_cast<uint4*>(qg + ((int64_t)b * kHeads + h) * kD + lane * 16);
+    dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    if (lane == 0) qfg[b * kHeads + h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
+}
+
+template <bool STAGED>
+__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                         const __grid_constant__ CUtensorMap tmap_q,
+                                                         const TcAttnDev a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -263,6 +364,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
+        mbar_init(&bar[2], 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tmem_holder, 512);
@@ -333,7 +435,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint32_t quad = (uint32_t)(32 * (warp & 3)) << 16;
-    uint32_t phase[2] = {0u, 0u};
+    uint32_t phase[3] = {0u, 0u, 0u};
     bool ok = true;
 
     // wait on barrier i (all threads), bounded
@@ -344,11 +446,31 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
 
     // S^T for chunk ch -> transposed logits Ssm[h][r] (log2 domain, -inf for empty rows)
     auto scores = [&](int ch) {
-        q_prefetch();
-        load_chunk(a, qrow, b, t, ch, sX, rvalid);
-        q_convert();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
+        if constexpr (STAGED) {
+            // rows and query already in fp16: 8 + 8 TMA boxes of [rows x 64 channels]
+            if (tid == 0) {
+                mbar_arrive_expect_tx(&bar[2], 8u * L::kXSlab + 8u * L::kQSlab);
+                const int32_t xrow = qrow * (a.K + a.W) + ch * kRows;
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j) {
+                    tma_load_2d(sm + L::kX + j * L::kXSlab, &tmap_x, &bar[2], 64 * j, xrow);
+                    tma_load_2d(sm + L::kQ + j * L::kQSlab, &tmap_q, &bar[2], 64 * j, qrow * kHeads);
+                }
+            }
+            if (tid < kRows) {
+                const int r = ch * kRows + tid;
+                rvalid[tid] = (r < a.K + a.W) ? __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
+            }
+            if (tid < kHeads) qf[tid] = __ldg(a.st_qf + qrow * kHeads + tid);
+            wait_bar(2);
+            __syncthreads();
+        } else {
+            q_prefetch();
+            load_chunk(a, qrow, b, t, ch, sX, rvalid);
+            q_convert();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+        }
         if (tid == 0) {
             tc_fence_after();
             issue_s(tmem, sX, sQ);
@@ -497,8 +619,41 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const TcAttnDev a) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [rows][512] fp16 matrix, box = 64 channels x box_rows, 128-byte swizzle
+static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(kD * 2)};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t attention_stage_bytes(int Q, int rows) {
+    return (size_t)Q * rows * kD * 2 + (size_t)Q * kHeads * kD * 2 + (size_t)Q * kHeads * 4 +
+           (size_t)Q * rows * 4 + 4 * 256;
+}
+
 cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
     TcAttnDev a;
+    memset(&a, 0, sizeof a);
     a.Q = l.Q;
     a.T = l.T;
     a.H = l.H;
@@ -522,11 +677,42 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
     a.chunks_per_split = (a.nchunks + l.nsplit - 1) / l.nsplit;
     a.status = l.status;
     const int smem = TcSmem::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
+    dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
+    CUtensorMap mx, mq;
+    memset(&mx, 0, sizeof mx);
+    memset(&mq, 0, sizeof mq);
+    if (!l.prefill && l.stage && l.K + l.W > 0) {
+        // staged decode: pre-pass, then the TMA-fed tensor-core kernel
+        const int rows = l.K + l.W;
+        uint8_t* base = reinterpret_cast<uint8_t*>(l.stage);
+        __half* xg = reinterpret_cast<__half*>(base);
+        base += (size_t)l.Q * rows * kD * 2;
+        base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 255) & ~(uintptr_t)255);
+        __half* qg = reinterpret_cast<__half*>(base);
+        base += (size_t)l.Q * kHeads * kD * 2;
+        float* qfg = reinterpret_cast<float*>(base);
+        base += (size_t)l.Q * kHeads * 4;
+        base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 255) & ~(uintptr_t)255);
+        int32_t* validg = reinterpret_cast<int32_t*>(base);
+        if (!fp16_rows_map(&mx, xg, (int64_t)l.Q * rows, kRows)) return cudaErrorInvalidValue;
+        if (!fp16_rows_map(&mq, qg, (int64_t)l.Q * kHeads, kHeads)) return cudaErrorInvalidValue;
+        a.st_valid = validg;
+        a.st_qf = qfg;
+        const int row_blocks = (rows + 7) / 8;
+        attn_stage_kernel<<<dim3((unsigned)l.Q, (unsigned)(row_blocks + kHeads / 8)), 256, 0, st>>>(
+            a, xg, qg, qfg, validg, row_blocks);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem);
+        if (e != cudaSuccess) return e;
+        attn_tc_kernel<true><<<grid, 256, smem, st>>>(mx, mq, a);
+        return cudaGetLastError();
+    }
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
-    attn_tc_kernel<<<grid, 256, smem, st>>>(a);
+    attn_tc_kernel<false><<<grid, 256, smem, st>>>(mx, mq, a);
     return cudaGetLastError();
 }
 

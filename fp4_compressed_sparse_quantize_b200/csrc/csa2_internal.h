@@ -88,10 +88,12 @@ struct AttnLaunch {
     float* out;              // [Q][H][512]
     float* partial;          // workspace for split rows
     int nsplit;
+    void* stage;             // decode staging area (attention_stage_bytes), or null
     int32_t* status;
 };
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+size_t attention_stage_bytes(int Q, int rows);
 int attention_splits(int Q, int K, int W, bool prefill);
 
 int device_sm_count();
