@@ -100,12 +100,15 @@ static size_t attn_ws_bytes(int Q, int H, int nsplit, int stage_rows) {
     return b;
 }
 
-// Upper bound of attention_splits() over every window size the API accepts (W <= 1024).
+// Upper bound of attention_splits() over every window size the API accepts (W <= 1024):
+// its unrounded split count, which grows with the row count.
 static int attn_split_bound(int Q, int K) {
     const int sms = device_sm_count();
-    const int ns = (2 * sms + Q - 1) / Q;
-    const int nch = (K + 1024 + 63) / 64;
-    return std::max(1, std::min(ns, nch));
+    const int rows = K + 1024;
+    int ns = sms / std::max(Q, 1);
+    ns = std::max(ns, (rows + kAttnDecodeRows - 1) / kAttnDecodeRows);
+    ns = std::min(ns, (rows + 31) / 32);
+    return std::max(1, ns);
 }
 
 __global__ void bounded_wait_probe_kernel(int32_t* status, uint64_t limit_ns) {

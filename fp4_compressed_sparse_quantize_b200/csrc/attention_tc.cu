@@ -64,7 +64,8 @@ struct TcAttnDev {
     bool prefill;
     float scale;
     float* out;
-    float* partial;
+    float* partial;          // O [Q * nsplit][H][512]
+    float* partial_ml;       // (m, l) [Q * nsplit][2][H]
     int nsplit, nchunks, chunks_per_split;
     int32_t* status;
     // staged decode: rows / query already dequantised by attn_stage_kernel
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
 template <bool STAGED>
 __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                          const __grid_constant__ CUtensorMap tmap_q,
+                                                         const __grid_constant__ CUtensorMap tmap_o,
                                                          const TcAttnDev a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -361,12 +363,33 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
     const int c_begin = split * a.chunks_per_split;
     const int c_end = min(a.nchunks, c_begin + a.chunks_per_split);
 
+    // staged rows and query of chunk ch: 8 + 8 TMA boxes of [rows x 64 channels] on bar[2]
+    auto issue_loads = [&](int ch) {
+        mbar_arrive_expect_tx(&bar[2], 8u * L::kXSlab + 8u * L::kQSlab);
+        const int32_t xrow = qrow * (a.K + a.W) + ch * kRows;
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+            tma_load_2d(sm + L::kX + j * L::kXSlab, &tmap_x, &bar[2], 64 * j, xrow);
+            tma_load_2d(sm + L::kQ + j * L::kQSlab, &tmap_q, &bar[2], 64 * j, qrow * kHeads);
+        }
+    };
     if (tid == 0) {
         mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         mbar_init(&bar[2], 1);
         fence_mbar_init();
+        if constexpr (STAGED) issue_loads(c_begin);   // overlaps the TMEM allocation below
     }
+    // the first chunk's row kinds and logit factors, fetched before the setup barrier
+    int pre_valid = 0;
+    float pre_qf = 0.f;
+    if constexpr (STAGED) {
+        const int r0 = c_begin * kRows + tid;
+        if (tid < kRows && r0 < a.K + a.W)
+            pre_valid = __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r0);
+        if (tid < kHeads) pre_qf = __ldg(a.st_qf + qrow * kHeads + tid);
+    }
+    bool first_chunk = true;
     if (warp == 0) tmem_alloc(tmem_holder, 512);
     if (tid < kHeads) m_s[tid] = -INFINITY;
 
@@ -447,21 +470,20 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
     // S^T for chunk ch -> transposed logits Ssm[h][r] (log2 domain, -inf for empty rows)
     auto scores = [&](int ch) {
         if constexpr (STAGED) {
-            // rows and query already in fp16: 8 + 8 TMA boxes of [rows x 64 channels]
-            if (tid == 0) {
-                mbar_arrive_expect_tx(&bar[2], 8u * L::kXSlab + 8u * L::kQSlab);
-                const int32_t xrow = qrow * (a.K + a.W) + ch * kRows;
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    tma_load_2d(sm + L::kX + j * L::kXSlab, &tmap_x, &bar[2], 64 * j, xrow);
-                    tma_load_2d(sm + L::kQ + j * L::kQSlab, &tmap_q, &bar[2], 64 * j, qrow * kHeads);
+            // rows and query already in fp16 (the first chunk's loads went out at the start)
+            if (first_chunk) {
+                if (tid < kRows) rvalid[tid] = pre_valid;
+                if (tid < kHeads) qf[tid] = pre_qf;
+                first_chunk = false;
+            } else {
+                if (tid == 0) issue_loads(ch);
+                if (tid < kRows) {
+                    const int r = ch * kRows + tid;
+                    rvalid[tid] =
+                        (r < a.K + a.W) ? __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
                 }
+                if (tid < kHeads) qf[tid] = __ldg(a.st_qf + qrow * kHeads + tid);
             }
-            if (tid < kRows) {
-                const int r = ch * kRows + tid;
-                rvalid[tid] = (r < a.K + a.W) ? __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
-            }
-            if (tid < kHeads) qf[tid] = __ldg(a.st_qf + qrow * kHeads + tid);
             wait_bar(2);
             __syncthreads();
         } else {
@@ -570,51 +592,318 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
         tc_fence_after();
         __syncthreads();   // X and the Q region may be rewritten by the next chunk
     }
-    if (qq == 0) l_s[h] = l_acc;
+    if (qq == 0) {
+        l_s[h] = l_acc;
+        qf[h] = l_acc > 0.f ? 1.f / l_acc : 0.f;   // the logit factors are no longer needed
+    }
     __syncthreads();
 
-    // ---- epilogue: O^T tiles (warps 0-3: tiles 0,1; warps 4-7: tiles 2,3) ---------------
+    // ---- epilogue: O^T tiles (warps 0-3: tiles 0,1; warps 4-7: tiles 2,3) -> shared memory
+    // as [heads][128 channels] fp32 per tile (the X region is free), then one bulk tensor
+    // store per tile: the normalised output (one split) or the partial output of this split
+    float* osm = reinterpret_cast<float*>(sm + L::kX);
+    const int oblk = a.nsplit == 1 ? qrow : qrow * a.nsplit + split;
     if (ok) {
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
             const int tile = 2 * (warp >> 2) + tt;
-            const int c = 128 * tile + 32 * (warp & 3) + lane;   // channel of this thread
+            const int cl = 32 * (warp & 3) + lane;   // channel within the tile
             uint32_t v[4][16];
 #pragma unroll
             for (int k = 0; k < 4; ++k) tmem_ld16(tmem + quad + kHeads + 64 * tile + 16 * k, v[k]);
             tmem_ld_wait();
-            if (a.nsplit == 1) {
+            float* dst = osm + tile * (kHeads * 128) + cl;
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k)
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int hh = 16 * k + e;
-                        if (hh < a.H) {
-                            const float l = l_s[hh];
-                            const float inv = l > 0.f ? 1.f / l : 0.f;
-                            a.out[((int64_t)qrow * a.H + hh) * kD + c] = __uint_as_float(v[k][e]) * inv;
-                        }
-                    }
-            } else {
-                float* base = a.partial + ((int64_t)qrow * a.nsplit + split) * ((int64_t)a.H * (kD + 2));
+                for (int e = 0; e < 16; ++e) {
+                    const int hh = 16 * k + e;
+                    float x = __uint_as_float(v[k][e]);
+                    if (a.nsplit == 1) x *= qf[hh];
+                    dst[hh * 128] = x;
+                }
+        }
+        if (a.nsplit > 1 && warp == 0) {
+            float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
+            for (int hh = lane; hh < a.H; hh += 32) {
+                ml[hh] = m_s[hh];
+                ml[a.H + hh] = l_s[hh];
+            }
+        }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && ok) {
+#pragma unroll 1
+        for (int tile = 0; tile < 4; ++tile)
+            tma_store_3d(&tmap_o, osm + tile * (kHeads * 128), 128 * tile, 0, oblk);
+        bulk_commit();
+        bulk_wait_all();
+    }
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---- decode: one CTA per (query, split of at most 160 rows) ------------------------------
+// The rows of a decode query are split evenly (a multiple of 32 per split, at most
+// kDecRows) so that all splits of all queries fit in one wave of CTAs.
+//
+// Logits: S = Q X^T with the 64 heads as the MMA M dimension (M = 64) and rows as N, in two
+// halves of the split's rows: half 0 into TMEM lanes 0-15 of every 32-lane subpartition,
+// half 1 into lanes 16-31 (the M = 64 accumulator layout: head h in lane (h mod 16) +
+// 32 (h / 16), row n in column n; a second accumulator may sit 16 lanes lower). The MMAs
+// of each 64-channel slab start as soon as that slab of X and Q has landed.
+// Softmax: thread (warp w, lane l) owns head 16 (w mod 4) + (l mod 16), row half l / 16 and
+// column half w / 4 of it; maxima and sums are combined with one shuffle and one
+// shared-memory exchange.
+// Output: P is written as the stacked A operand [P_hi; P_lo] of [O_hi; O_lo] = P X with
+// M = 128 rows ordered so that the high and low parts of head h are 16 TMEM lanes apart in
+// the same subpartition (row 32 (h / 16) + (h mod 16) high, +16 low); X is the MN-major B
+// operand (N = 256 channels, two halves). The epilogue adds the two parts with one shuffle.
+constexpr int kDecRows = kAttnDecodeRows;
+
+struct DecSmem {
+    int xslab;   // bytes per X slab: rows x 128 B
+    __device__ __host__ explicit DecSmem(int rps) : xslab(rps * 128) {}
+    // the X region also takes the 128 KiB output tile of the epilogue
+    __device__ __host__ int q() const { return 8 * xslab > 131072 ? 8 * xslab : 131072; }
+    // after S: P (3 slabs of [128 stacked heads x 64 rows], 16 KiB each) and the tail
+    __device__ __host__ int phi() const { return q(); }
+    __device__ __host__ int tail() const { return q() + 6 * TcSmem::kQSlab; }   // 16 KiB
+    __device__ __host__ int bytes() const { return q() + 8 * TcSmem::kQSlab; }
+};
+
+// exact split of p into p_hi + p_lo with p_hi representable in fp16 (p in the fp16 normal
+// range; below it the pair carries p to within 2^-25): p_hi keeps 11 significant bits
+__device__ __forceinline__ float hi11(float p) {
+    return __uint_as_float((__float_as_uint(p) + 0x1000u) & 0xFFFFE000u);
+}
+
+__global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                             const __grid_constant__ CUtensorMap tmap_q,
+                                                             const __grid_constant__ CUtensorMap tmap_o,
+                                                             const TcAttnDev a, int rps) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar[10];   // 0-7: slab j of X and Q landed; 8: S done; 9: P X done
+    __shared__ uint32_t tmem_holder;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const DecSmem L(rps);
+    const uint32_t sX = smem_u32(sm), sQ = smem_u32(sm + L.q()), sP = smem_u32(sm + L.phi());
+    float* tail = reinterpret_cast<float*>(sm + L.tail());
+    float* qf = tail;              // [64]
+    float* m_s = tail + 64;        // [64]
+    float* l_s = tail + 128;       // [64]
+    float* inv_s = tail + 192;     // [64]
+    float* redm = tail + 256;      // [2][64]
+    float* redl = tail + 384;      // [2][64]
+    uint32_t* vmask = reinterpret_cast<uint32_t*>(tail + 512);   // row validity bits [8]
+
+    const int qrow = blockIdx.x, split = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rows = a.K + a.W;
+    const int r0 = split * rps;    // first row of this split
+    const int half_rows = rps >> 1;
+
+    if (tid == 0) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
+        for (int j = 0; j < 10; ++j) mbar_init(&bar[j], 1);
+        fence_mbar_init();
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+            mbar_arrive_expect_tx(&bar[j], (uint32_t)L.xslab + TcSmem::kQSlab);
+            tma_load_2d(sm + j * L.xslab, &tmap_x, &bar[j], 64 * j, qrow * rows + r0);
+            tma_load_2d(sm + L.q() + j * TcSmem::kQSlab, &tmap_q, &bar[j], 64 * j, qrow * kHeads);
+        }
+    }
+    // row kinds and logit factors, held in registers until the Q tile is dead
+    int pre_valid = 0;
+    float pre_qf = 0.f;
+    if (tid < rps && r0 + tid < rows) pre_valid = __ldg(a.st_valid + (int64_t)qrow * rows + r0 + tid);
+    if (tid < kHeads) pre_qf = __ldg(a.st_qf + qrow * kHeads + tid);
+    if (warp == 0) tmem_alloc(&tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_holder;
+    bool ok = true;
+    bool loads_ok = true;
+
+    // ---- S = Q X^T, M = 64, N = rps / 2 per half, K = 512: slab by slab as it lands ------------
+    if (tid == 0) {
+        const uint32_t idesc = make_idesc(64, half_rows, 0u, 0u);
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+            if (!mbar_wait(&bar[j], 0, a.status)) ok = loads_ok = false;
+            tc_fence_after();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int hh = 16 * k + e;
-                        if (hh < a.H) base[(int64_t)hh * kD + c] = __uint_as_float(v[k][e]);
-                    }
-                if (tile == 0 && warp == 0 && lane < 32) {
-                    for (int hh = lane; hh < a.H; hh += 32) {
-                        base[(int64_t)a.H * kD + hh] = m_s[hh];
-                        base[(int64_t)a.H * kD + a.H + hh] = l_s[hh];
-                    }
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int kk = 4 * j + k4;
+                const uint64_t ad = sw128_desc(sQ + j * TcSmem::kQSlab + k4 * 32, 16, 1024);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint64_t bd = sw128_desc(sX + j * L.xslab + part * half_rows * 128 + k4 * 32, 16, 1024);
+                    mma_f16(tmem + ((uint32_t)(16 * part) << 16) + 256u, ad, bd, idesc, kk > 0);
+                }
+            }
+        }
+        mma_commit(&bar[8]);
+    }
+    if (!mbar_wait(&bar[8], 0, a.status)) ok = false;
+    tc_fence_after();
+    // the Q tile is dead: its tail takes the row validity bits and the logit factors
+    {
+        const uint32_t vb = __ballot_sync(0xffffffffu, pre_valid != 0);
+        if (lane == 0) vmask[warp] = vb;   // rows 32 warp .. +31 (rows >= rps are 0)
+    }
+    if (tid < kHeads) qf[tid] = pre_qf;
+    __syncthreads();
+
+    // ---- softmax over this split's rows ------------------------------------------------------
+    const int quad = warp & 3, wh = warp >> 2;
+    const int hl = lane & 15, rh = lane >> 4;
+    const int h = 16 * quad + hl;                    // head of this thread
+    const int ncol = rps >> 2;                       // columns per thread: multiple of 8, <= 40
+    const int cstart = rh * half_rows + wh * ncol;   // first row (of the split) of the thread
+    const uint32_t sbase = tmem + ((uint32_t)(32 * quad) << 16) + 256u + (uint32_t)(wh * ncol);
+    const float f = qf[h];
+    uint32_t sv[kDecRows / 4];
+#pragma unroll
+    for (int g = 0; g < kDecRows / 32; ++g)
+        if (8 * g < ncol) tmem_ld8(sbase + 8 * g, *reinterpret_cast<uint32_t(*)[8]>(sv + 8 * g));
+    uint32_t vm[2];                                  // validity bits of rows cstart .. +63
+    {
+        const int wi = cstart >> 5, sh = cstart & 31;
+        vm[0] = __funnelshift_r(vmask[wi], vmask[wi + 1], sh);
+        vm[1] = __funnelshift_r(vmask[wi + 1], vmask[wi + 2], sh);
+    }
+    tmem_ld_wait();
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kDecRows / 4; ++j) {
+        const float x = __uint_as_float(sv[j]) * f;
+        sv[j] = __float_as_uint(x);
+        if (j < ncol && ((vm[j >> 5] >> (j & 31)) & 1u)) mx = fmaxf(mx, x);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (rh == 0) redm[wh * 64 + h] = mx;
+    __syncthreads();
+    const float m = fmaxf(redm[h], redm[64 + h]);
+    const float base = (m == -INFINITY) ? 0.f : m;
+    float ls = 0.f;
+    const int prow = 32 * quad + hl;                 // stacked P row of the high part
+#pragma unroll
+    for (int g = 0; g < kDecRows / 32; ++g) {
+        if (8 * g < ncol) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 8 * g + 2 * e;
+                const float p0 = ((vm[j >> 5] >> (j & 31)) & 1u) ? exp2f(__uint_as_float(sv[j]) - base) : 0.f;
+                const float p1 = ((vm[(j + 1) >> 5] >> ((j + 1) & 31)) & 1u) ? exp2f(__uint_as_float(sv[j + 1]) - base) : 0.f;
+                ls += p0 + p1;
+                const float h0 = hi11(p0), h1 = hi11(p1);
+                hi[e] = h2_bits(__floats2half2_rn(h0, h1));
+                lo[e] = h2_bits(__floats2half2_rn(p0 - h0, p1 - h1));
+            }
+            const int c = cstart + 8 * g;            // 8 rows: one 16-byte chunk per part
+            const uint32_t sl = sP + (uint32_t)((c >> 6) * 2 * TcSmem::kQSlab);
+            st_shared_v4(sl + slab_off(prow, (c & 63) >> 3), hi[0], hi[1], hi[2], hi[3]);
+            st_shared_v4(sl + slab_off(prow + 16, (c & 63) >> 3), lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+    ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+    if (rh == 0) redl[wh * 64 + h] = ls;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    if (rh == 0 && wh == 0) {
+        const float l = redl[h] + redl[64 + h];
+        m_s[h] = m;
+        l_s[h] = l;
+        inv_s[h] = l > 0.f ? 1.f / l : 0.f;
+    }
+
+    // ---- [O_hi; O_lo] = P X: M = 128, N = 256 channels (two halves), K = rps rows ------------
+    // X (rows x channels, channels contiguous) is the MN-major B operand: 64-channel slabs
+    // apart by one X slab (LBO), 8-row groups 1 KiB apart (SBO). D fills TMEM columns
+    // [0, 512); the logits there were all read above.
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = make_idesc(128, 256, 0u, 0u, 0u, /*b MN-major*/ 1u);
+        const int nk = rps >> 4;
+#pragma unroll 1
+        for (int nh = 0; nh < 2; ++nh)
+#pragma unroll 1
+            for (int kk = 0; kk < nk; ++kk) {
+                const uint64_t ad =
+                    sw128_desc(sP + (kk >> 2) * 2 * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = sw128_desc(sX + (4 * nh) * L.xslab + kk * 16 * 128,
+                                               (uint32_t)L.xslab, 1024);
+                mma_f16(tmem + 256 * nh, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+        mma_commit(&bar[9]);
+    }
+    if (!mbar_wait(&bar[9], 0, a.status)) ok = false;
+    tc_fence_after();
+    __syncthreads();
+
+    // ---- epilogue: O = O_hi + O_lo (lanes l and l ^ 16) into shared memory as 16 boxes of
+    // [64 heads][32 channels] (128-byte rows, 16-byte chunks XOR-swizzled by head), then one
+    // bulk tensor store per box
+    float* osm = reinterpret_cast<float*>(sm);
+    const int oblk = a.nsplit == 1 ? qrow : qrow * a.nsplit + split;
+    const uint32_t tq = (uint32_t)(32 * quad) << 16;
+    const int cbase = 256 * wh;                // channels of this warp
+    const float oscale = a.nsplit == 1 ? inv_s[h] : 1.f;
+    if (ok) {
+#pragma unroll 1
+        for (int cc = 0; cc < 256; cc += 64) {
+            uint32_t v[4][16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tmem_ld16(tmem + tq + cbase + cc + 16 * k, v[k]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float o[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float x = __uint_as_float(v[k][e]);
+                    o[e] = (x + __shfl_xor_sync(0xffffffffu, x, 16)) * oscale;
+                }
+                // lanes 0-15 store channels +0..7, lanes 16-31 channels +8..15
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int c = cbase + cc + 16 * k + 8 * rh + 4 * j;
+                    float* dst = osm + (c >> 5) * (kHeads * 32) + h * 32 + ((((c & 31) >> 2) ^ (h & 7)) << 2);
+                    const int e0 = 4 * j;   // of this lane's half: o[e0 + 8 rh ..]
+                    *reinterpret_cast<float4*>(dst) =
+                        rh ? make_float4(o[e0 + 8], o[e0 + 9], o[e0 + 10], o[e0 + 11])
+                           : make_float4(o[e0], o[e0 + 1], o[e0 + 2], o[e0 + 3]);
                 }
             }
         }
     }
+    if (ok && a.nsplit > 1 && warp == 0) {
+        float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
+        for (int x = lane; x < a.H; x += 32) {
+            ml[x] = m_s[x];
+            ml[a.H + x] = l_s[x];
+        }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && ok) {
+#pragma unroll 1
+        for (int b = 0; b < 16; ++b)
+            tma_store_3d(&tmap_o, osm + b * (kHeads * 32), 32 * b, 0, oblk);
+        bulk_commit();
+        bulk_wait_all();
+    }
+    if (tid == 0 && !loads_ok)   // a load that timed out may still be in flight: bounded
+        for (int j = 0; j < 8; ++j) mbar_wait(&bar[j], 0, a.status);
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
@@ -646,6 +935,32 @@ static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int bo
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [blocks][H][512] fp32 output or partial output, box = 128 channels x H heads x 1 block
+static bool out_map(CUtensorMap* m, void* base, int H, int64_t blocks) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)(kD * 4), (cuuint64_t)H * kD * 4};
+    cuuint32_t box[3] = {128u, (cuuint32_t)H, 1u};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [blocks][H][512] fp32, box = 32 channels x H heads x 1 block, 128-byte swizzle
+static bool out_map_sw(CUtensorMap* m, void* base, int H, int64_t blocks) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)blocks};
+    cuuint64_t strides[2] = {(cuuint64_t)(kD * 4), (cuuint64_t)H * kD * 4};
+    cuuint32_t box[3] = {32u, (cuuint32_t)H, 1u};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t attention_stage_bytes(int Q, int rows) {
     return (size_t)Q * rows * kD * 2 + (size_t)Q * kHeads * kD * 2 + (size_t)Q * kHeads * 4 +
            (size_t)Q * rows * 4 + 4 * 256;
@@ -671,6 +986,7 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
     a.scale = l.scale;
     a.out = l.out;
     a.partial = l.partial;
+    a.partial_ml = l.nsplit > 1 ? l.partial + (int64_t)l.Q * l.nsplit * l.H * kD : nullptr;
     a.nsplit = l.nsplit;
     a.nchunks = (l.K + l.W + kRows - 1) / kRows;
     if (a.nchunks < 1) a.nchunks = 1;
@@ -678,12 +994,17 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
     a.status = l.status;
     const int smem = TcSmem::kAlloc;
     dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
-    CUtensorMap mx, mq;
+    CUtensorMap mx, mq, mo;
     memset(&mx, 0, sizeof mx);
     memset(&mq, 0, sizeof mq);
+    if (l.nsplit > 1 ? !out_map(&mo, l.partial, l.H, (int64_t)l.Q * l.nsplit)
+                     : !out_map(&mo, l.out, l.H, l.Q))
+        return cudaErrorInvalidValue;
     if (!l.prefill && l.stage && l.K + l.W > 0) {
-        // staged decode: pre-pass, then the TMA-fed tensor-core kernel
+        // staged decode: pre-pass, then one CTA per (query, split)
         const int rows = l.K + l.W;
+        const int rps = attention_rows_per_split(rows, l.nsplit);
+        if (rps > kDecRows || (int64_t)rps * l.nsplit < rows) return cudaErrorInvalidValue;
         uint8_t* base = reinterpret_cast<uint8_t*>(l.stage);
         __half* xg = reinterpret_cast<__half*>(base);
         base += (size_t)l.Q * rows * kD * 2;
@@ -694,7 +1015,7 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
         base += (size_t)l.Q * kHeads * 4;
         base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(base) + 255) & ~(uintptr_t)255);
         int32_t* validg = reinterpret_cast<int32_t*>(base);
-        if (!fp16_rows_map(&mx, xg, (int64_t)l.Q * rows, kRows)) return cudaErrorInvalidValue;
+        if (!fp16_rows_map(&mx, xg, (int64_t)l.Q * rows, rps)) return cudaErrorInvalidValue;
         if (!fp16_rows_map(&mq, qg, (int64_t)l.Q * kHeads, kHeads)) return cudaErrorInvalidValue;
         a.st_valid = validg;
         a.st_qf = qfg;
@@ -703,16 +1024,22 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
             a, xg, qg, qfg, validg, row_blocks);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem);
+        CUtensorMap mos;
+        memset(&mos, 0, sizeof mos);
+        if (l.nsplit > 1 ? !out_map_sw(&mos, l.partial, l.H, (int64_t)l.Q * l.nsplit)
+                         : !out_map_sw(&mos, l.out, l.H, l.Q))
+            return cudaErrorInvalidValue;
+        const int dsmem = DecSmem(rps).bytes() + 1024;
+        e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsmem);
         if (e != cudaSuccess) return e;
-        attn_tc_kernel<true><<<grid, 256, smem, st>>>(mx, mq, a);
+        attn_decode_kernel<<<grid, 256, dsmem, st>>>(mx, mq, mos, a, rps);
         return cudaGetLastError();
     }
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<false><<<grid, 256, smem, st>>>(mx, mq, a);
+    attn_tc_kernel<false><<<grid, 256, smem, st>>>(mx, mq, mo, a);
     return cudaGetLastError();
 }
 

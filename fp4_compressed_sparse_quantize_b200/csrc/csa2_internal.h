@@ -94,7 +94,11 @@ struct AttnLaunch {
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
 size_t attention_stage_bytes(int Q, int rows);
+// Decode splits the K + W rows of a query into equal runs of at most kAttnDecodeRows rows
+// (a multiple of 32), as many as fill one wave of CTAs; prefill never splits.
+constexpr int kAttnDecodeRows = 160;
 int attention_splits(int Q, int K, int W, bool prefill);
+int attention_rows_per_split(int rows, int nsplit);
 
 int device_sm_count();
 

@@ -11,7 +11,9 @@
 //
 // Radix select on an order-preserving 32-bit key of the fp32 score, extended to a unique
 // 64-bit composite  (key << 32) | ~id  so that "larger composite" is the required order.
-// One kernel, grid = chunks x rows:
+// Rows of up to 262,144 elements take one 1024-thread CTA each (topk_row_kernel: the steps
+// below, all in shared memory). Longer rows (the 1M-entry Full layer) are split over CTAs,
+// grid = chunks x rows:
 //   1. the scan kernel already histogrammed the top 12 key bits of every row, which fixes
 //      the threshold digit d0: fewer than K elements lie above it;
 //   2. every CTA classifies its chunk: elements above d0 are sure winners, elements on d0
@@ -422,6 +424,478 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
     for (int i = npick * mult + tid; i < K * mult; i += kThreads) o[i] = -1;
 }
 
+// ---- one CTA per row ----------------------------------------------------------------------
+// For rows of up to kRowMaxN elements a single 1024-thread CTA owns the row: the threshold
+// digit, the winners, the candidates and the refinement all stay in shared memory, so
+// there is no cross-CTA hand-off. Without ids the row's histogram and scores (or keys) are
+// streamed into shared memory by bulk asynchronous copies (64 KiB chunks, two buffers): a
+// single SM keeps far more bytes in flight that way than with per-thread loads. With ids
+// (Reindex: short rows) the elements are read 8 per thread per batch.
+constexpr int kRowThreads = 1024;
+constexpr int kRowPer = 16;                  // elements per thread per chunk (no ids)
+constexpr int kRowChunk = kRowThreads * kRowPer;   // 16384 elements = 64 KiB
+constexpr int kRowPerIds = 8;                // elements per thread per batch (ids)
+constexpr int kRowCands = 4096;
+constexpr int64_t kRowMaxN = 262144;
+constexpr size_t kRowOffHist = 0;                                   // u32[4096]
+constexpr size_t kRowOffCand = kRowOffHist + 4 * kBinsT;            // u64[kRowCands]
+constexpr size_t kRowOffWin = kRowOffCand + 8 * kRowCands;          // u32[kMaxK]
+constexpr size_t kRowOffBar = kRowOffWin + 4 * kMaxK;               // 3 mbarriers
+constexpr size_t kRowOffBm = kRowOffBar + 64;                       // bitmap or pick list
+// after the bitmap (no ids): two chunk buffers, 64 KiB each, 128-byte aligned
+constexpr size_t kRowChunkBytes = (size_t)kRowChunk * 4;
+__host__ __device__ constexpr size_t row_chunk_offset(int bitmap_words) {
+    return (kRowOffBm + (bitmap_words > 0 ? (size_t)bitmap_words * 4 : (size_t)kMaxK * 4) + 127) &
+           ~(size_t)127;
+}
+
+// Exclusive prefix sum of v over the 1024 threads (thread order); `total` gets the sum.
+// Uses wsum[0..32); ends with a barrier, so wsum may be reused right away.
+__device__ __forceinline__ uint32_t row_excl_scan(uint32_t v, uint32_t* wsum, uint32_t& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t x = wsum[lane], xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += u;
+        }
+        wsum[lane] = xi - x;   // exclusive over warps
+        if (lane == 31) wsum[32] = xi;
+    }
+    __syncthreads();
+    const uint32_t r = wsum[warp] + incl - v;
+    total = wsum[32];
+    __syncthreads();
+    return r;
+}
+
+// Warp 0 only: over bins h[0..256) (counts), find d with above(d) < rem <= above(d) + h[d],
+// above(d) = sum of h[e] for e > d. Writes d (or -1 when the total is < rem), above(d) and
+// h[d] into out[0..3).
+__device__ __forceinline__ void warp_find_digit256(const uint32_t* h, uint32_t rem, int* out) {
+    const int lane = threadIdx.x & 31;
+    uint32_t b[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {   // lane 0 owns the 8 highest bins, highest first
+        b[j] = h[255 - 8 * lane - j];
+        sum += b[j];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    const uint32_t excl = incl - sum;
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0 && total < rem) {
+        out[0] = -1;
+        out[1] = (int)total;
+        out[2] = 0;
+    }
+    if (excl < rem && incl >= rem) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (acc < rem && acc + b[j] >= rem) {
+                out[0] = 255 - 8 * lane - j;
+                out[1] = (int)acc;
+                out[2] = (int)b[j];
+            }
+            acc += b[j];
+        }
+    }
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t elem_key(const TopkDev& a, int r, int64_t i) {
+    return a.scores ? score_key(__ldg(a.scores + (int64_t)r * a.ld + i))
+                    : __ldg(a.keys + (int64_t)r * a.ld + i);
+}
+
+// Shared-memory state of one row's selection.
+struct RowState {
+    uint32_t* hist;     // 4096 bins (the histogram, later 256-bin refinement counts)
+    uint64_t* cand_s;   // candidates (composites), first kRowCands
+    uint32_t* win_s;    // winner ids
+    uint32_t* bm;       // bitmap of picked ids, or the pick list
+    uint32_t* wsum;
+    int* dig_s;
+    uint32_t* tot_s;    // running winner / candidate counts
+};
+
+// Classify PER elements per thread against d0 and append them to the winner / candidate
+// lists. Element k has key[k] and id ID(k) and takes part when bit k of `valid` is set.
+// Block-wide (contains barriers).
+template <int PER, class IdOf>
+__device__ __forceinline__ void row_classify(const TopkDev& a, const RowState& S, int r,
+                                             const uint32_t (&key)[PER], IdOf ID,
+                                             uint32_t valid, bool many, int d0) {
+    uint32_t wmask = 0, cmask = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const bool ok = (valid >> k) & 1u;
+        const int dig = (int)(key[k] >> 20);
+        if (ok && (!many || dig > d0)) wmask |= 1u << k;
+        if (ok && many && dig == d0) cmask |= 1u << k;
+    }
+    const uint32_t cw = __popc(wmask), cc = __popc(cmask);
+    uint32_t tot;
+    const uint32_t ex = row_excl_scan(cw | (cc << 16), S.wsum, tot);
+    uint32_t pw = S.tot_s[0] + (ex & 0xFFFFu), pc = S.tot_s[1] + (ex >> 16);
+    uint64_t* gcand = a.cands + (int64_t)r * a.ccap;
+    uint32_t wm = wmask, cm = cmask;
+    // only the (few) selected elements are visited
+    while (wm | cm) {
+        const int k = __ffs(wm | cm) - 1;
+        const uint32_t bit = 1u << k;
+        uint32_t kk = 0;
+#pragma unroll
+        for (int j = 0; j < PER; ++j)
+            if (j == k) kk = key[j];
+        const uint32_t id = ID(k);
+        if (wm & bit) {
+            if (pw < (uint32_t)a.K) S.win_s[pw] = id;
+            ++pw;
+        } else {
+            const uint64_t c = ((uint64_t)kk << 32) | (uint64_t)(~id);
+            if (pc < (uint32_t)kRowCands) S.cand_s[pc] = c;
+            else if (pc < (uint32_t)a.ccap) gcand[pc] = c;
+            ++pc;
+        }
+        wm &= ~bit;
+        cm &= ~bit;
+    }
+    __syncthreads();   // every thread has read tot_s
+    if (threadIdx.x == 0) {
+        S.tot_s[0] += tot & 0xFFFFu;
+        S.tot_s[1] += tot >> 16;
+    }
+    __syncthreads();
+}
+
+// d0 (the digit holding the K-th best element) from this thread's four bins, highest first
+// (thread 0 owns the top bins). Sets many / d0 / above for every thread.
+__device__ __forceinline__ void row_threshold(const RowState& S, const uint32_t (&b4)[4], int K,
+                                              bool& many, int& d0, uint32_t& above) {
+    const int tid = threadIdx.x;
+    const uint32_t local = b4[0] + b4[1] + b4[2] + b4[3];
+    uint32_t total;
+    const uint32_t excl = row_excl_scan(local, S.wsum, total);
+    if (excl < (uint32_t)K && excl + local >= (uint32_t)K) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (acc < (uint32_t)K && acc + b4[j] >= (uint32_t)K) {
+                S.dig_s[0] = 4 * (kRowThreads - 1 - tid) + 3 - j;
+                S.dig_s[1] = (int)acc;
+            }
+            acc += b4[j];
+        }
+    }
+    __syncthreads();
+    many = total >= (uint32_t)K;
+    d0 = many ? S.dig_s[0] : -1;
+    above = many ? (uint32_t)S.dig_s[1] : total;
+    __syncthreads();
+}
+
+// Refinement, picks and the ordered output of one row, after every element was classified.
+template <bool GATHER>
+__device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t n,
+                             uint32_t id_lim, bool many, int d0, uint32_t above) {
+    const int tid = threadIdx.x;
+    const int K = a.K;
+    const bool use_bm = a.bitmap_words > 0;
+    const int nwords = a.bitmap_words;
+    const uint32_t nwin_all = S.tot_s[0], ncand = S.tot_s[1];
+    const uint32_t nwin = min(nwin_all, (uint32_t)K);
+    if (tid == 0 && (nwin_all > (uint32_t)K || (many && nwin_all != above)))
+        set_status(a.status, CSA2_DEV_BAD_COUNT);
+    __syncthreads();
+    uint64_t* gcand = a.cands + (int64_t)r * a.ccap;
+
+    if (many) {
+        const uint32_t need = (uint32_t)K - above;
+        const bool from_row = ncand > (uint32_t)max(a.ccap, kRowCands);
+        const int64_t nsrc = from_row ? n : (int64_t)ncand;
+        // candidate i of the source (false: not a candidate)
+        auto cand = [&](int64_t i, uint64_t& c) -> bool {
+            if (from_row) {
+                const uint32_t kk = elem_key(a, r, i);
+                uint32_t id = (uint32_t)i;
+                if (GATHER) {
+                    const int32_t v = __ldg(a.ids + (int64_t)r * a.ld + i);
+                    if (v < 0 || (uint32_t)v >= id_lim) return false;
+                    id = (uint32_t)v;
+                }
+                c = ((uint64_t)kk << 32) | (uint64_t)(~id);
+                return (int)(kk >> 20) == d0;
+            }
+            c = i < kRowCands ? S.cand_s[i] : __ldcg(gcand + i);
+            return true;
+        };
+        uint64_t prefix = (uint64_t)d0;
+        int shift = 52;
+        uint32_t rem = need;
+        while (shift > 0) {
+            const int nb = shift < 8 ? shift : 8;
+            if (tid < 256) S.hist[tid] = 0u;
+            __syncthreads();
+            for (int64_t i = tid; i < nsrc; i += kRowThreads) {
+                uint64_t c;
+                if (cand(i, c) && (c >> shift) == prefix)
+                    atomicAdd(&S.hist[(c >> (shift - nb)) & ((1u << nb) - 1u)], 1u);
+            }
+            __syncthreads();
+            if (tid < 32) warp_find_digit256(S.hist, rem, S.dig_s);
+            __syncthreads();
+            const int d = S.dig_s[0];
+            const uint32_t ab = (uint32_t)S.dig_s[1], inbin = (uint32_t)S.dig_s[2];
+            __syncthreads();   // dig_s is rewritten by the next pass
+            if (d < 0) {
+                if (tid == 0) set_status(a.status, CSA2_DEV_BAD_COUNT);
+                prefix = 0;
+                shift = 0;
+                break;
+            }
+            rem -= ab;
+            prefix = (prefix << nb) | (uint64_t)d;
+            shift -= nb;
+            if (inbin == rem) break;   // the whole bin is taken
+        }
+        const uint64_t T = prefix << shift;
+        // mark the chosen candidates
+        for (int64_t i = tid; i < nsrc; i += kRowThreads) {
+            uint64_t c;
+            if (cand(i, c) && c >= T) {
+                const uint32_t id = ~(uint32_t)(c & 0xFFFFFFFFu);
+                if (use_bm) {
+                    if ((int)(id >> 5) < nwords) atomicOr(&S.bm[id >> 5], 1u << (id & 31));
+                } else {
+                    const uint32_t pos = atomicAdd(&S.tot_s[0], 1u);
+                    if (pos < (uint32_t)K) S.bm[pos] = id;
+                }
+            }
+        }
+    }
+    // winners
+    for (uint32_t i = tid; i < nwin; i += kRowThreads) {
+        const uint32_t id = S.win_s[i];
+        if (use_bm) {
+            if ((int)(id >> 5) < nwords) atomicOr(&S.bm[id >> 5], 1u << (id & 31));
+        } else {
+            S.bm[i] = id;   // slots [0, nwin) of the pick list; candidates were appended after
+        }
+    }
+    __syncthreads();
+
+    // ---- emit in ascending id order ----------------------------------------------------------
+    const int32_t lim = a.expand8 ? __ldg(a.expand_limit + r) : 0;
+    int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
+    auto emit = [&](uint32_t slot, int64_t id) {
+        if (slot >= (uint32_t)K) return;
+        if (!a.expand8) {
+            o[slot] = (int32_t)id;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int64_t pos = id * 8 + e;
+                o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
+            }
+        }
+    };
+    int npick;
+    if (use_bm) {
+        const int per = (nwords + kRowThreads - 1) / kRowThreads;
+        const int w0 = tid * per, w1 = min(nwords, w0 + per);
+        uint32_t cntb = 0;
+        for (int wi = w0; wi < w1; ++wi) cntb += __popc(S.bm[wi]);
+        uint32_t tot;
+        uint32_t off = row_excl_scan(cntb, S.wsum, tot);
+        npick = (int)min(tot, (uint32_t)K);
+        for (int wi = w0; wi < w1; ++wi) {
+            uint32_t m = S.bm[wi];
+            while (m) {
+                const int b = __ffs(m) - 1;
+                m &= m - 1;
+                emit(off++, (int64_t)wi * 32 + b);
+            }
+        }
+    } else {
+        // winners occupy [0, nwin), candidates were appended from tot_s[0] = nwin_all on
+        npick = (int)min(many ? S.tot_s[0] : nwin, (uint32_t)K);
+        for (int i = tid; i < npick; i += kRowThreads) {
+            const uint32_t v = S.bm[i];
+            int rank = 0;
+            for (int j = 0; j < npick; ++j) {
+                const uint32_t u = S.bm[j];
+                rank += (u < v) | ((u == v) & (j < i));
+            }
+            emit((uint32_t)rank, v);
+        }
+    }
+    const int mult = a.expand8 ? 8 : 1;
+    for (int i = npick * mult + tid; i < K * mult; i += kRowThreads) o[i] = -1;
+}
+
+template <bool GATHER>
+__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ uint32_t wsum[40];
+    __shared__ int dig_s[4];
+    __shared__ uint32_t tot_s[2];
+    RowState S;
+    S.hist = reinterpret_cast<uint32_t*>(dsm + kRowOffHist);
+    S.cand_s = reinterpret_cast<uint64_t*>(dsm + kRowOffCand);
+    S.win_s = reinterpret_cast<uint32_t*>(dsm + kRowOffWin);
+    S.bm = reinterpret_cast<uint32_t*>(dsm + kRowOffBm);
+    S.wsum = wsum;
+    S.dig_s = dig_s;
+    S.tot_s = tot_s;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + kRowOffBar);
+    const int r = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t n = row_len(a, r);
+    const int K = a.K;
+    const uint32_t id_lim = GATHER ? (uint32_t)max(0, __ldg(a.id_limit + r)) : 0xFFFFFFFFu;
+    const bool use_bm = a.bitmap_words > 0;
+    const int nwords = a.bitmap_words;
+    if (tid == 0) {
+        tot_s[0] = tot_s[1] = 0u;
+        dig_s[0] = -1;
+        dig_s[1] = 0;
+    }
+    bool many;
+    int d0;
+    uint32_t above;
+
+    if constexpr (GATHER) {
+        // ---- ids: plain loads, 8 elements per thread per batch ------------------------------
+        constexpr int PER = kRowPerIds;
+        constexpr int BATCH = kRowThreads * PER;
+        uint32_t key[PER], id[PER];
+        auto load = [&](int64_t base) {
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int64_t i = base + (int64_t)k * kRowThreads + tid;
+                key[k] = i < n ? elem_key(a, r, i) : 0u;
+                id[k] = i < n ? (uint32_t)__ldg(a.ids + (int64_t)r * a.ld + i) : 0xFFFFFFFFu;
+            }
+        };
+        load(0);
+        const uint4 h4 = reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kBinsT)[kRowThreads - 1 - tid];
+        if (use_bm)
+            for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
+        const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
+        row_threshold(S, b4, K, many, d0, above);
+        for (int64_t base = 0; base < n; base += BATCH) {
+            if (base > 0) load(base);
+            uint32_t valid = 0;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int64_t i = base + (int64_t)k * kRowThreads + tid;
+                if (i < n && (int32_t)id[k] >= 0 && id[k] < id_lim) valid |= 1u << k;
+            }
+            row_classify<PER>(a, S, r, key, [&](int k) { 
+                uint32_t v = 0;
+#pragma unroll
+                for (int j = 0; j < PER; ++j)
+                    if (j == k) v = id[j];
+                return v;
+            }, valid, many, d0);
+        }
+    } else {
+        // ---- positions: histogram and elements through bulk copies -------------------------
+        // Elements [h0, h0 + nbulk) arrive in 64 KiB chunks (16-byte aligned source, whole
+        // 16-byte units); the few before h0 and after the last unit are read directly.
+        uint8_t* cbuf = dsm + row_chunk_offset(nwords);
+        const uint8_t* rowp = a.scores ? reinterpret_cast<const uint8_t*>(a.scores + (int64_t)r * a.ld)
+                                       : reinterpret_cast<const uint8_t*>(a.keys + (int64_t)r * a.ld);
+        const int64_t lead = (int64_t)(((16u - (reinterpret_cast<uintptr_t>(rowp) & 15u)) & 15u) >> 2);
+        const int h0 = (int)(lead < n ? lead : n);
+        const int64_t nbulk = ((n - h0) >> 2) << 2;       // whole 16-byte units
+        const int64_t ntail = n - h0 - nbulk;              // < 4
+        const int nch = (int)((nbulk + kRowChunk - 1) / kRowChunk);
+        bool ok = true;
+        auto issue = [&](int c) {
+            const int64_t e0 = (int64_t)c * kRowChunk;
+            const int64_t left = nbulk - e0;
+            const uint32_t bytes = (uint32_t)((left < kRowChunk ? left : (int64_t)kRowChunk) * 4);
+            mbar_arrive_expect_tx(&bar[1 + (c & 1)], bytes);
+            bulk_load(cbuf + (size_t)(c & 1) * kRowChunkBytes, rowp + (h0 + e0) * 4, bytes,
+                      &bar[1 + (c & 1)]);
+        };
+        if (tid == 0) {
+            mbar_init(&bar[0], 1);
+            mbar_init(&bar[1], 1);
+            mbar_init(&bar[2], 1);
+            fence_mbar_init();
+            mbar_arrive_expect_tx(&bar[0], 4u * kBinsT);
+            bulk_load(S.hist, a.hist + (int64_t)r * kBinsT, 4u * kBinsT, &bar[0]);
+            for (int c = 0; c < min(nch, 2); ++c) issue(c);
+        }
+        // the stray head / tail elements: one per thread among the first few threads
+        uint32_t xkey = 0u;
+        int64_t xi = -1;
+        if (tid < h0) xi = tid;
+        else if (tid - h0 < ntail) xi = h0 + nbulk + (tid - h0);
+        if (xi >= 0) xkey = elem_key(a, r, xi);
+        if (use_bm)
+            for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
+        __syncthreads();   // barrier initialisation is visible to every waiting thread
+        if (!mbar_wait(&bar[0], 0, a.status)) ok = false;
+        const uint4 h4 = reinterpret_cast<const uint4*>(S.hist)[kRowThreads - 1 - tid];
+        const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
+        row_threshold(S, b4, K, many, d0, above);   // ends with a barrier: hist is free again
+        for (int c = 0; c < max(nch, 1); ++c) {
+            uint32_t key[kRowPer + 1];
+            uint32_t valid = 0;
+            const int64_t e0 = (int64_t)c * kRowChunk;
+            if (c < nch) {
+                if (!mbar_wait(&bar[1 + (c & 1)], (uint32_t)((c >> 1) & 1), a.status)) ok = false;
+                const uint32_t* buf = reinterpret_cast<const uint32_t*>(cbuf + (size_t)(c & 1) * kRowChunkBytes);
+#pragma unroll
+                for (int k = 0; k < kRowPer; ++k) {
+                    const int64_t e = e0 + (int64_t)k * kRowThreads + tid;
+                    const uint32_t raw = e < nbulk ? buf[k * kRowThreads + tid] : 0u;
+                    key[k] = a.scores ? score_key(__uint_as_float(raw)) : raw;
+                    if (e < nbulk) valid |= 1u << k;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < kRowPer; ++k) key[k] = 0u;
+            }
+            key[kRowPer] = xkey;
+            if (c == 0 && xi >= 0) valid |= 1u << kRowPer;
+            const uint32_t idb = (uint32_t)(h0 + e0 + tid);
+            row_classify<kRowPer + 1>(a, S, r, key, [&](int k) {
+                return k < kRowPer ? idb + (uint32_t)k * kRowThreads : (uint32_t)xi;
+            }, valid, many, d0);
+            // every thread has read buffer (c & 1): refill it with chunk c + 2
+            if (tid == 0 && ok && c + 2 < nch) issue(c + 2);
+        }
+    }
+    row_finalize<GATHER>(a, S, r, n, id_lim, many, d0, above);
+}
+
 cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     if (l.K > kMaxK || l.K <= 0) return cudaErrorInvalidValue;
     TopkDev a;
@@ -443,13 +917,27 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     a.cands = l.cands;
     a.ccap = l.ccap;
     a.status = l.status;
-    // ids are < id_bound: a bitmap of that many bits orders the picks when it is small
+    // ids are < id_bound: a bitmap of that many bits orders the picks when it fits
     const int64_t words = (l.id_bound + 31) / 32;
+    cudaError_t e;
+    if (l.max_n <= kRowMaxN) {
+        // ids: the bitmap may cover up to 2^20 ids; positions: ids < max_n <= 2^18, and the
+        // two 64 KiB chunk buffers follow the bitmap
+        a.bitmap_words = (l.id_bound > 0 && words * 4 <= 128 * 1024) ? (int)words : 0;
+        size_t rsmem = kRowOffBm + (a.bitmap_words > 0 ? (size_t)a.bitmap_words * 4
+                                                        : (size_t)kMaxK * 4);
+        if (!l.ids) rsmem = row_chunk_offset(a.bitmap_words) + 2 * kRowChunkBytes;
+        if (rsmem > 227 * 1024) return cudaErrorInvalidValue;
+        auto kern = l.ids ? topk_row_kernel<true> : topk_row_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)l.R, kRowThreads, rsmem, st>>>(a);
+        return cudaGetLastError();
+    }
     a.bitmap_words = (l.id_bound > 0 && words * 4 <= 64 * 1024) ? (int)words : 0;
     const size_t smem = (size_t)kSmemCands * 8 +
                         (a.bitmap_words > 0 ? (size_t)a.bitmap_words * 4 : (size_t)kMaxK * 4);
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int64_t chunks = (l.max_n + kCollectChunk - 1) / kCollectChunk;
     if (chunks < 1) chunks = 1;
