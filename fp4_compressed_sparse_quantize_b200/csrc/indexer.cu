@@ -12,15 +12,20 @@
 // Score (reading adopted; the pages print no formula):
 //     s[r, j] = sum_{h < H_I} w[r, h] * max(0, <q_I[r, h, :], k_I[j, :]>)
 //
-// Design (one persistent CTA per SM, 6 warps):
-//   warp 0      producer: TMA tiles of 128 indexer keys (contiguous, 128-byte swizzle) into
-//               an S-stage ring; in gather mode (Reindex) cp.async of the pool's rows into
-//               the same swizzled layout; plus the query-group operand per row group.
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128 keys,
-//               N = G queries x H_I heads, K = 128 channels) into a TMEM accumulator ring.
-//   warps 2..5  epilogue: tcgen05.ld of one key row per thread, ReLU-weighted head sum in
-//               fp32, coalesced score stores, shared-memory histogram of the top 12 key
-//               bits per query row (first radix-select digit), 8-entry block maxima.
+// Design (one persistent CTA per SM):
+//   warp 0      producer: TMA tiles of 128 (or 256) indexer keys (contiguous, 128-byte
+//               swizzle) into an S-stage ring; in gather mode (Reindex) cp.async of the
+//               pool's rows into the same swizzled layout; plus the query-group operand per
+//               row group.
+//   warps 1, 2  MMA issuers (alternate tiles; warp 1 also allocates TMEM): one thread each
+//               issues tcgen05.mma (M = 128 keys, N = G queries x H_I heads, K = 128
+//               channels) into a TMEM accumulator ring. A single issuing thread spends a few
+//               hundred cycles per tile in barrier waits and per-instruction issue, which
+//               alone would cap the tile rate below the HBM rate; two issuers share it.
+//   then EPI    epilogue groups of 4 warps: tcgen05.ld of one key row per thread,
+//               ReLU-weighted head sum in fp32, coalesced score stores, shared-memory
+//               histogram of the top 12 key bits per query row (first radix-select digit),
+//               8-entry block maxima.
 // Every wait is bounded (2 s) and sets CSA2_DEV_TIMEOUT instead of hanging.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -131,8 +136,11 @@ __device__ __forceinline__ void fence_proxy_async() {
 // ESZ    = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
 // GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
 // TM     = 128-key halves per tile (one TMA box, TM MMA groups into adjacent TMEM columns)
+constexpr int kIssuers = 2;                       // MMA-issuing warps
+constexpr int kEpiWarp0 = 1 + kIssuers;           // first epilogue warp
+
 template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM>
-__global__ void __launch_bounds__(64 + 128 * EPI, 1)
+__global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
@@ -185,20 +193,20 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qfull[s], 1);
-            mbar_init(&qempty[s], 1);
+            mbar_init(&qempty[s], kIssuers);   // every issuer releases the query slot
         }
         for (int s = 0; s < ACC; ++s) {
             mbar_init(&accfull[s], 1);
             mbar_init(&accempty[s], 4);
         }
-        mbar_init(done_bar, 1);
+        mbar_init(done_bar, kIssuers);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < EPI * G * kBins; i += 128 * EPI) hist_s[i] = 0;
+    if (warp >= kEpiWarp0) {
+        for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * G * kBins; i += 128 * EPI) hist_s[i] = 0;
         if (POOL)
-            for (int i = threadIdx.x - 64; i < EPI * kBins; i += 128 * EPI) bhist_s[i] = 0;
+            for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * kBins; i += 128 * EPI) bhist_s[i] = 0;
     }
     if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
     if (warp == 0 && lane == 0 && !GATHER) {
@@ -287,8 +295,11 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
                 mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), p.status);
             if (qcount > 0) mbar_wait(&qfull[(qcount - 1) & 1], ((qcount - 1) >> 1) & 1, p.status);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp <= kIssuers) {
+        // ------------------------------------------------------------ MMA issuers
+        // issuer m issues the tiles it == m (mod kIssuers) but follows every row-group
+        // change, so that each issuer releases every query slot
+        const int m = warp - 1;
         if (lane == 0) {
             GroupCursor cur;
             cur.init(p.prefix, ngroups, t0);
@@ -306,6 +317,7 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
                     qg = cur.g;
                     ++qcount;
                 }
+                if ((int)(it % kIssuers) != m) continue;
                 const int s = (int)(it % STAGES);
                 if (!mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), p.status)) { *abort_flag = 1; break; }
                 const int a = (int)(it % ACC);
@@ -341,8 +353,8 @@ __global__ void __launch_bounds__(64 + 128 * EPI, 1)
         // EPI groups of 4 warps take alternate tiles (group e owns iterations it = e mod
         // EPI and therefore TMEM accumulators a = it mod ACC of that residue), each with its
         // own histograms, weights and named barrier.
-        const int e = (warp - 2) >> 2;
-        const int et = threadIdx.x - 64 - 128 * e;  // 0..127 within the group
+        const int e = (warp - kEpiWarp0) >> 2;
+        const int et = threadIdx.x - 32 * kEpiWarp0 - 128 * e;  // 0..127 within the group
         const int row = 32 * (warp & 3) + lane;     // TMEM lane == key row within a half
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
         uint32_t* hist_e = hist_s + e * G * kBins;
@@ -625,7 +637,7 @@ static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms(), 64 + 128 * EPI, L::kAlloc, st>>>(mk, mq, p);
+    kern<<<num_sms(), 32 * kEpiWarp0 + 128 * EPI, L::kAlloc, st>>>(mk, mq, p);
     return cudaGetLastError();
 }
 
