@@ -266,16 +266,21 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
     const int R = pl.R;
 
     cudaError_t e;
-    e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)R * kBins, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(cnt, 0, sizeof(uint32_t) * 4 * (size_t)R, st);
-    if (e == cudaSuccess && pool_blocks > 0) {
-        e = cudaMemsetAsync(wb + pl.off_bhist, 0, sizeof(uint32_t) * (size_t)R * kBins, st);
-        if (e == cudaSuccess)
-            e = cudaMemsetAsync(wb + pl.off_pcnt, 0, sizeof(uint32_t) * 4 * (size_t)R, st);
+    // histograms and counters start at zero: cleared by the prep kernel
+    ZeroList zl;
+    memset(&zl, 0, sizeof zl);
+    zl.p[0] = reinterpret_cast<uint4*>(hist);
+    zl.n16[0] = (int64_t)R * kBins * 4 / 16;
+    zl.p[1] = reinterpret_cast<uint4*>(cnt);
+    zl.n16[1] = (int64_t)R * 4 * 4 / 16;
+    if (pool_blocks > 0) {
+        zl.p[2] = reinterpret_cast<uint4*>(wb + pl.off_bhist);
+        zl.n16[2] = (int64_t)R * kBins * 4 / 16;
+        zl.p[3] = reinterpret_cast<uint4*>(wb + pl.off_pcnt);
+        zl.n16[3] = (int64_t)R * 4 * 4 / 16;
     }
-    if (e != cudaSuccess) return CSA2_ERR_CUDA;
     e = launch_prep_rows(R, T, pl.G, n_vis0, q_pos0, ratio, cap, reindex ? P_in : 0,
-                         scan_tile_rows(pl.G, reindex, esz), n_row, prefix, status, st);
+                         scan_tile_rows(pl.G, reindex, esz), n_row, prefix, status, zl, st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
 
     ScanLaunch sl;

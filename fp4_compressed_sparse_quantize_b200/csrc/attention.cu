@@ -22,6 +22,8 @@ constexpr int kDm = 512;      // latent channels
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ partial,
                                                            int nsplit, int H,
                                                            float* __restrict__ out) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int qrow = blockIdx.x, h = blockIdx.y;
     const int64_t stride = (int64_t)H * kDm;            // between splits of one row
     const float* base = partial + (int64_t)qrow * nsplit * stride;
@@ -88,9 +90,8 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st);
 cudaError_t launch_attention(const AttnLaunch& l, cudaStream_t st) {
     cudaError_t e = launch_attention_tc(l, st);
     if (e != cudaSuccess || l.nsplit == 1) return e;
-    attn_combine_kernel<<<dim3((unsigned)l.Q, (unsigned)l.H), 128, 0, st>>>(l.partial, l.nsplit,
-                                                                          l.H, l.out);
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel, dim3((unsigned)l.Q, (unsigned)l.H), dim3(128), 0, st,
+                      (const float*)l.partial, l.nsplit, l.H, l.out);
 }
 
 }  // namespace csa2

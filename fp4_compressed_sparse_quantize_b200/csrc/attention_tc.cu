@@ -254,6 +254,8 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
                                                          float* __restrict__ qfg,
                                                          int32_t* __restrict__ validg,
                                                          int row_blocks) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = a.K + a.W;
@@ -357,6 +359,8 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::kTmem);
 
+    grid_dep_launch();
+    grid_dep_wait();
     const int qrow = blockIdx.x, split = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = qrow / a.T, t = qrow - b * a.T;
@@ -706,10 +710,15 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     const int r0 = split * rps;    // first row of this split
     const int half_rows = rps >> 1;
 
+    grid_dep_launch();
     if (tid == 0) {
 #pragma unroll
         for (int j = 0; j < 10; ++j) mbar_init(&bar[j], 1);
         fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_holder, 512);
+    grid_dep_wait();   // the staged rows and query come from the pre-pass
+    if (tid == 0) {
 #pragma unroll 1
         for (int j = 0; j < 8; ++j) {
             mbar_arrive_expect_tx(&bar[j], (uint32_t)L.xslab + TcSmem::kQSlab);
@@ -722,7 +731,6 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     float pre_qf = 0.f;
     if (tid < rps && r0 + tid < rows) pre_valid = __ldg(a.st_valid + (int64_t)qrow * rows + r0 + tid);
     if (tid < kHeads) pre_qf = __ldg(a.st_qf + qrow * kHeads + tid);
-    if (warp == 0) tmem_alloc(&tmem_holder, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1020,9 +1028,9 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
         a.st_valid = validg;
         a.st_qf = qfg;
         const int row_blocks = (rows + 7) / 8;
-        attn_stage_kernel<<<dim3((unsigned)l.Q, (unsigned)(row_blocks + kHeads / 8)), 256, 0, st>>>(
-            a, xg, qg, qfg, validg, row_blocks);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(attn_stage_kernel,
+                                   dim3((unsigned)l.Q, (unsigned)(row_blocks + kHeads / 8)),
+                                   dim3(256), 0, st, a, xg, qg, qfg, validg, row_blocks);
         if (e != cudaSuccess) return e;
         CUtensorMap mos;
         memset(&mos, 0, sizeof mos);
@@ -1033,14 +1041,12 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
         e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsmem);
         if (e != cudaSuccess) return e;
-        attn_decode_kernel<<<grid, 256, dsmem, st>>>(mx, mq, mos, a, rps);
-        return cudaGetLastError();
+        return launch_pdl(attn_decode_kernel, grid, dim3(256), (size_t)dsmem, st, mx, mq, mos, a, rps);
     }
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<false><<<grid, 256, smem, st>>>(mx, mq, mo, a);
-    return cudaGetLastError();
+    return launch_pdl(attn_tc_kernel<false>, grid, dim3(256), (size_t)smem, st, mx, mq, mo, a);
 }
 
 }  // namespace csa2

@@ -80,6 +80,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     }
 }
 
+// ---- programmatic dependent launch -----------------------------------------------------
+// Every library kernel is launched so that it may start while the previous kernel on the
+// stream is still finishing. It announces at once that the next kernel may begin its own
+// prologue, and it waits for the previous grids (complete, memory visible) before its first
+// access to global memory that another kernel reads or writes. Both are no-ops for a plain
+// launch.
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- TMA (no multicast anywhere in this library) --------------------------------------
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar,

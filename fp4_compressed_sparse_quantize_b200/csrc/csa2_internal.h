@@ -5,7 +5,27 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <utility>
+
 namespace csa2 {
+
+// Launch with programmatic stream serialisation (see grid_dep_wait / grid_dep_launch).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct ScanLaunch {
     int B, T, rows, G, H_I, esz;
@@ -33,10 +53,16 @@ cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
                                uint8_t* scales, int64_t cap, int32_t* status,
                                cudaStream_t stream);
 
+// Up to four workspace buffers that the prep kernel clears (16-byte units).
+struct ZeroList {
+    uint4* p[4];
+    int64_t n16[4];
+};
+
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
                              const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
                              int tile_rows, int32_t* n_row, int64_t* prefix, int32_t* status,
-                             cudaStream_t st);
+                             const ZeroList& zero, cudaStream_t st);
 
 // keys per scan tile for a query-group size and mode
 int scan_tile_rows(int G, bool gather, int esz);

@@ -181,10 +181,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int ngroups = p.rows / G;
-    const int64_t total = __ldg(p.prefix + ngroups);
-    const int64_t t0 = total * blockIdx.x / gridDim.x;
-    const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
-    if (t0 >= t1) return;  // uniform across the CTA
+    grid_dep_launch();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -217,8 +214,15 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // the tile prefix (and everything else in global memory) comes from earlier kernels
+    grid_dep_wait();
+    const int64_t total = __ldg(p.prefix + ngroups);
+    const int64_t t0 = total * blockIdx.x / gridDim.x;
+    const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
 
-    if (warp == 0) {
+    if (t0 >= t1) {
+        // no tiles for this CTA (uniform): release TMEM below
+    } else if (warp == 0) {
         // ------------------------------------------------------------ producer
         GroupCursor cur;
         cur.init(p.prefix, ngroups, t0);
@@ -505,13 +509,23 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
 // ---- per-row visible counts and tile prefix ---------------------------------------------
 // decode: n_row[r] = n_vis0[r]; prefill: n_row[b*T+t] = floor((q_pos0[b]+t+1)/ratio).
 // Counts are clamped to [0, cap] (CSA2_DEV_BAD_COUNT when clamping was needed); gather
-// mode counts pool slots instead of entries for the tile prefix.
+// mode counts pool slots instead of entries for the tile prefix. Every CTA also clears its
+// share of the histograms and counters that the scan and Top-K accumulate into; CTA 0
+// computes the counts and the prefix.
 __global__ void __launch_bounds__(1024) prep_rows_kernel(
     int rows, int T, int G, const int32_t* n_vis0, const int32_t* q_pos0, int ratio,
     int64_t cap, int P_gather, int tile_rows, int32_t* n_row, int64_t* prefix,
-    int32_t* status) {
+    int32_t* status, const ZeroList zero) {
     __shared__ int64_t warp_sums[32];
     __shared__ int64_t carry;
+    grid_dep_launch();
+    grid_dep_wait();
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero.n16[k];
+             i += (int64_t)gridDim.x * blockDim.x)
+            zero.p[k][i] = make_uint4(0u, 0u, 0u, 0u);
+    if (blockIdx.x != 0) return;
     if (threadIdx.x == 0) carry = 0;
     const int ngroups = rows / G;
     for (int base = 0; base < rows; base += blockDim.x) {
@@ -637,8 +651,8 @@ static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms(), 32 * kEpiWarp0 + 128 * EPI, L::kAlloc, st>>>(mk, mq, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(num_sms()), dim3(32 * kEpiWarp0 + 128 * EPI), L::kAlloc, st,
+                      mk, mq, p);
 }
 
 // Dispatch on (padded query columns, element size, group size, mode).
@@ -710,10 +724,15 @@ int scan_tile_rows(int G, bool gather, int esz) {
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
                              const int32_t* q_pos0, int ratio, int64_t cap, int P_gather,
                              int tile_rows, int32_t* n_row, int64_t* prefix, int32_t* status,
-                             cudaStream_t st) {
-    prep_rows_kernel<<<1, 1024, 0, st>>>(rows, T, G, n_vis0, q_pos0, ratio, cap, P_gather,
-                                         tile_rows, n_row, prefix, status);
-    return cudaGetLastError();
+                             const ZeroList& zero, cudaStream_t st) {
+    int64_t n16 = 0;
+    for (int k = 0; k < 4; ++k) n16 += zero.n16[k];
+    int64_t blocks = (n16 + 4 * 1024 - 1) / (4 * 1024);
+    if (blocks < 1) blocks = 1;
+    if (blocks > 64) blocks = 64;
+    return launch_pdl(prep_rows_kernel, dim3((unsigned)blocks), dim3(1024), 0, st, rows, T, G,
+                      n_vis0, q_pos0, ratio, cap, P_gather, tile_rows, n_row, prefix, status,
+                      zero);
 }
 
 }  // namespace csa2

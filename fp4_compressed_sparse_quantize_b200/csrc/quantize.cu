@@ -17,6 +17,7 @@
 // value with at most 4) leaves a non-dyadic quotient far from every dyadic midpoint, and
 // a dyadic quotient is exact in fp32. A reciprocal-multiply would not have that property.
 #include "csa2_common.cuh"
+#include "csa2_internal.h"
 
 namespace csa2 {
 
@@ -24,6 +25,8 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(
     const __nv_bfloat16* __restrict__ kv, int B, int n_new, int64_t ld_kv, int64_t bstride_kv,
     const int32_t* __restrict__ dst_off, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int64_t cap, int32_t* status) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int lane = threadIdx.x & 31;
     const int64_t entry = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (entry >= (int64_t)B * n_new) return;
@@ -89,10 +92,9 @@ cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
     if (entries == 0) return cudaSuccess;
     const int warps = 8;
     const int64_t grid = (entries + warps - 1) / warps;
-    quantize_kv_kernel<<<(unsigned)grid, warps * 32, 0, stream>>>(
-        reinterpret_cast<const __nv_bfloat16*>(kv), B, n_new, ld_kv, bstride_kv, dst_off, codes,
-        scales, cap, status);
-    return cudaGetLastError();
+    return launch_pdl(quantize_kv_kernel, dim3((unsigned)grid), dim3(warps * 32), 0, stream,
+                      reinterpret_cast<const __nv_bfloat16*>(kv), B, n_new, ld_kv, bstride_kv,
+                      dst_off, codes, scales, cap, status);
 }
 
 }  // namespace csa2

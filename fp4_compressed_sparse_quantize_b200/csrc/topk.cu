@@ -211,6 +211,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
     __shared__ uint32_t npick_s;
     const int r = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    grid_dep_launch();
+    grid_dep_wait();
     const int64_t n = row_len(a, r);
     const int64_t start = (int64_t)blockIdx.x * kCollectChunk;
     const int64_t end = min(n, start + kCollectChunk);
@@ -773,6 +775,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
     uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + kRowOffBar);
     const int r = blockIdx.x;
     const int tid = threadIdx.x;
+    grid_dep_launch();
+    grid_dep_wait();
     const int64_t n = row_len(a, r);
     const int K = a.K;
     const uint32_t id_lim = GATHER ? (uint32_t)max(0, __ldg(a.id_limit + r)) : 0xFFFFFFFFu;
@@ -931,8 +935,7 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
         auto kern = l.ids ? topk_row_kernel<true> : topk_row_kernel<false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
         if (e != cudaSuccess) return e;
-        kern<<<(unsigned)l.R, kRowThreads, rsmem, st>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(kern, dim3((unsigned)l.R), dim3(kRowThreads), rsmem, st, a);
     }
     a.bitmap_words = (l.id_bound > 0 && words * 4 <= 64 * 1024) ? (int)words : 0;
     const size_t smem = (size_t)kSmemCands * 8 +
@@ -942,8 +945,7 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     int64_t chunks = (l.max_n + kCollectChunk - 1) / kCollectChunk;
     if (chunks < 1) chunks = 1;
     dim3 grid((unsigned)chunks, (unsigned)l.R);
-    topk_kernel<<<grid, kThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel, grid, dim3(kThreads), smem, st, a);
 }
 
 }  // namespace csa2
