@@ -17,11 +17,8 @@
 //               swizzle) into an S-stage ring; in gather mode (Reindex) cp.async of the
 //               pool's rows into the same swizzled layout; plus the query-group operand per
 //               row group.
-//   warps 1, 2  MMA issuers (alternate tiles; warp 1 also allocates TMEM): one thread each
-//               issues tcgen05.mma (M = 128 keys, N = G queries x H_I heads, K = 128
-//               channels) into a TMEM accumulator ring. A single issuing thread spends a few
-//               hundred cycles per tile in barrier waits and per-instruction issue, which
-//               alone would cap the tile rate below the HBM rate; two issuers share it.
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128 keys,
+//               N = G queries x H_I heads, K = 128 channels) into a TMEM accumulator ring.
 //   then EPI    epilogue groups of 4 warps: tcgen05.ld of one key row per thread,
 //               ReLU-weighted head sum in fp32, coalesced score stores, shared-memory
 //               histogram of the top 12 key bits per query row (first radix-select digit),
@@ -136,7 +133,10 @@ __device__ __forceinline__ void fence_proxy_async() {
 // ESZ    = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
 // GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
 // TM     = 128-key halves per tile (one TMA box, TM MMA groups into adjacent TMEM columns)
-constexpr int kIssuers = 2;                       // MMA-issuing warps
+// One thread issues every tcgen05.mma of the CTA. (Issuing from two warps on alternate
+// tiles was faster but intermittently never completed an MMA commit on the 256K-context
+// workload, so the MMA issue stays with a single thread.)
+constexpr int kIssuers = 1;                       // MMA-issuing warps
 constexpr int kEpiWarp0 = 1 + kIssuers;           // first epilogue warp
 
 template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM>

@@ -439,6 +439,7 @@ constexpr int kRowChunk = kRowThreads * kRowPer;   // 16384 elements = 64 KiB
 constexpr int kRowPerIds = 8;                // elements per thread per batch (ids)
 constexpr int kRowCands = 4096;
 constexpr int64_t kRowMaxN = 262144;
+constexpr int kRowCluster = 4;               // CTAs per row for few long rows
 constexpr size_t kRowOffHist = 0;                                   // u32[4096]
 constexpr size_t kRowOffCand = kRowOffHist + 4 * kBinsT;            // u64[kRowCands]
 constexpr size_t kRowOffWin = kRowOffCand + 8 * kRowCands;          // u32[kMaxK]
@@ -758,8 +759,41 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
     for (int i = npick * mult + tid; i < K * mult; i += kRowThreads) o[i] = -1;
 }
 
-template <bool GATHER>
-__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a) {
+// ---- cluster helpers (distributed shared memory) -------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// shared::cluster address of `p` (this CTA's shared memory) in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_peer_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t ld_peer_u64(uint32_t addr) {
+    uint64_t v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// CL > 1: a cluster of CL CTAs shares one row. Every CTA finds d0 and classifies its own
+// contiguous part of the row into its own lists; CTA 0 then gathers the other CTAs' lists
+// through distributed shared memory and finishes the row alone.
+template <bool GATHER, int CL>
+__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a_in) {
+    static_assert(!GATHER || CL == 1, "gather rows are short: one CTA each");
+    TopkDev a = a_in;
+    if (CL > 1) a.ccap = 0;   // per-CTA candidate lists live in shared memory only
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ uint32_t wsum[40];
     __shared__ int dig_s[4];
@@ -773,14 +807,15 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
     S.dig_s = dig_s;
     S.tot_s = tot_s;
     uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + kRowOffBar);
-    const int r = blockIdx.x;
+    const int r = CL > 1 ? (int)blockIdx.y : (int)blockIdx.x;
+    const uint32_t crank = CL > 1 ? cluster_rank() : 0u;
     const int tid = threadIdx.x;
     grid_dep_launch();
     grid_dep_wait();
     const int64_t n = row_len(a, r);
     const int K = a.K;
     const uint32_t id_lim = GATHER ? (uint32_t)max(0, __ldg(a.id_limit + r)) : 0xFFFFFFFFu;
-    const bool use_bm = a.bitmap_words > 0;
+    const bool use_bm = a.bitmap_words > 0 && crank == 0;
     const int nwords = a.bitmap_words;
     if (tid == 0) {
         tot_s[0] = tot_s[1] = 0u;
@@ -835,8 +870,12 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
                                        : reinterpret_cast<const uint8_t*>(a.keys + (int64_t)r * a.ld);
         const int64_t lead = (int64_t)(((16u - (reinterpret_cast<uintptr_t>(rowp) & 15u)) & 15u) >> 2);
         const int h0 = (int)(lead < n ? lead : n);
-        const int64_t nbulk = ((n - h0) >> 2) << 2;       // whole 16-byte units
-        const int64_t ntail = n - h0 - nbulk;              // < 4
+        const int64_t nbulk_all = ((n - h0) >> 2) << 2;   // whole 16-byte units
+        const int64_t ntail = n - h0 - nbulk_all;          // < 4
+        // this CTA's part [pb, pb + nbulk) of the bulk elements (4-element granularity)
+        const int64_t part = (((nbulk_all >> 2) + CL - 1) / CL) << 2;
+        const int64_t pb = (int64_t)crank * part < nbulk_all ? (int64_t)crank * part : nbulk_all;
+        const int64_t nbulk = (pb + part < nbulk_all ? pb + part : nbulk_all) - pb;
         const int nch = (int)((nbulk + kRowChunk - 1) / kRowChunk);
         bool ok = true;
         auto issue = [&](int c) {
@@ -844,7 +883,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
             const int64_t left = nbulk - e0;
             const uint32_t bytes = (uint32_t)((left < kRowChunk ? left : (int64_t)kRowChunk) * 4);
             mbar_arrive_expect_tx(&bar[1 + (c & 1)], bytes);
-            bulk_load(cbuf + (size_t)(c & 1) * kRowChunkBytes, rowp + (h0 + e0) * 4, bytes,
+            bulk_load(cbuf + (size_t)(c & 1) * kRowChunkBytes, rowp + (h0 + pb + e0) * 4, bytes,
                       &bar[1 + (c & 1)]);
         };
         if (tid == 0) {
@@ -859,8 +898,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
         // the stray head / tail elements: one per thread among the first few threads
         uint32_t xkey = 0u;
         int64_t xi = -1;
-        if (tid < h0) xi = tid;
-        else if (tid - h0 < ntail) xi = h0 + nbulk + (tid - h0);
+        if (crank == 0) {
+            if (tid < h0) xi = tid;
+            else if (tid - h0 < ntail) xi = h0 + nbulk_all + (tid - h0);
+        }
         if (xi >= 0) xkey = elem_key(a, r, xi);
         if (use_bm)
             for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
@@ -889,13 +930,42 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
             }
             key[kRowPer] = xkey;
             if (c == 0 && xi >= 0) valid |= 1u << kRowPer;
-            const uint32_t idb = (uint32_t)(h0 + e0 + tid);
+            const uint32_t idb = (uint32_t)(h0 + pb + e0 + tid);
             row_classify<kRowPer + 1>(a, S, r, key, [&](int k) {
                 return k < kRowPer ? idb + (uint32_t)k * kRowThreads : (uint32_t)xi;
             }, valid, many, d0);
             // every thread has read buffer (c & 1): refill it with chunk c + 2
             if (tid == 0 && ok && c + 2 < nch) issue(c + 2);
         }
+    }
+    if constexpr (CL > 1) {
+        // every CTA's lists are complete; CTA 0 appends the others' lists to its own
+        cluster_sync_all();
+        if (crank == 0) {
+            uint32_t wbase = tot_s[0], cbase = tot_s[1];
+            __syncthreads();
+#pragma unroll 1
+            for (uint32_t k = 1; k < (uint32_t)CL; ++k) {
+                const uint32_t nw = ld_peer_u32(peer_addr(&tot_s[0], k));
+                const uint32_t nc = ld_peer_u32(peer_addr(&tot_s[1], k));
+                const uint32_t rw = peer_addr(S.win_s, k), rc = peer_addr(S.cand_s, k);
+                for (uint32_t i = tid; i < nw; i += kRowThreads)
+                    if (wbase + i < (uint32_t)K && i < (uint32_t)K) S.win_s[wbase + i] = ld_peer_u32(rw + 4 * i);
+                for (uint32_t i = tid; i < nc; i += kRowThreads)
+                    if (cbase + i < (uint32_t)kRowCands && i < (uint32_t)kRowCands)
+                        S.cand_s[cbase + i] = ld_peer_u64(rc + 8 * i);
+                wbase += nw;
+                cbase += nc;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                tot_s[0] = wbase;
+                tot_s[1] = cbase;
+            }
+            __syncthreads();
+        }
+        cluster_sync_all();   // the other CTAs' lists have been read: they may exit
+        if (crank != 0) return;
     }
     row_finalize<GATHER>(a, S, r, n, id_lim, many, d0, above);
 }
@@ -932,7 +1002,29 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
                                                         : (size_t)kMaxK * 4);
         if (!l.ids) rsmem = row_chunk_offset(a.bitmap_words) + 2 * kRowChunkBytes;
         if (rsmem > 227 * 1024) return cudaErrorInvalidValue;
-        auto kern = l.ids ? topk_row_kernel<true> : topk_row_kernel<false>;
+        // few long rows: a cluster of kRowCluster CTAs per row spreads the classification
+        if (!l.ids && l.max_n >= 4 * kRowChunk / 2 && l.R * kRowCluster <= 2 * device_sm_count()) {
+            auto kern = topk_row_kernel<false, kRowCluster>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+            if (e != cudaSuccess) return e;
+            cudaLaunchConfig_t cfg;
+            memset(&cfg, 0, sizeof cfg);
+            cfg.gridDim = dim3(kRowCluster, (unsigned)l.R);
+            cfg.blockDim = dim3(kRowThreads);
+            cfg.dynamicSmemBytes = rsmem;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = kRowCluster;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 2;
+            return cudaLaunchKernelEx(&cfg, kern, a);
+        }
+        auto kern = l.ids ? topk_row_kernel<true, 1> : topk_row_kernel<false, 1>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3((unsigned)l.R), dim3(kRowThreads), rsmem, st, a);

@@ -157,6 +157,22 @@ def test_full_decode_scores_and_topk(dtype, H_I, K, n_list):
         check_topk(idx[b, 0], s, np.arange(n), K, f"b={b} n={n}")
 
 
+def test_topk_long_rows_odd_stride():
+    """Rows long enough for the multi-CTA row selection, an odd row stride (rows start at
+    every 4-byte alignment) and ragged lengths."""
+    g = _gen(77)
+    n_list = [40003, 33000, 65537]
+    B, cap, H_I, K = len(n_list), max(n_list), 64, 512
+    k_I = _keys(B, cap, torch.float8_e4m3fn, g)
+    q_I = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn)
+    w = torch.rand((B, 1, H_I), generator=g)
+    idx, scores, _, st = _full_decode(q_I, w, k_I, n_list, K)
+    assert st == 0
+    for b, n in enumerate(n_list):
+        s = O.index_scores(raw_qk(q_I[b, 0]), w[b, 0].numpy(), raw_qk(k_I[b, :n]), O.E4M3)
+        check_topk(idx[b, 0], s, np.arange(n), K, f"b={b} n={n}")
+
+
 def test_topk_degenerate_all_equal_scores():
     """w = 0: every score is +0, the K lowest positions must win (slow exact path)."""
     g = _gen(7)
