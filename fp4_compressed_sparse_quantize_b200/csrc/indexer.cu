@@ -262,9 +262,13 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)L::kTileBytes);
                     const int64_t row = (int64_t)b * p.cap + jt * kRowsT;
-                    for (int h = 0; h < ESZ; ++h)
-                        tma_load_2d_hint(dst + h * kSlab, &tmap_k, &full[s], h * 64 * (ESZ == 2),
-                                         (int32_t)row, policy);
+                    // one box of 128 rows per 128-key half (and per 64-channel half for bf16)
+#pragma unroll
+                    for (int hh = 0; hh < TM; ++hh)
+                        for (int h = 0; h < ESZ; ++h)
+                            tma_load_2d_hint(dst + h * kSlab + hh * kTileRows * 128, &tmap_k,
+                                             &full[s], h * 64 * (ESZ == 2),
+                                             (int32_t)(row + hh * kTileRows), policy);
                 }
             } else {
                 // pool rows of query row r0 (G == 1 in gather mode)
@@ -637,9 +641,10 @@ constexpr int pick_stages() {
 template <int NQ, int ESZ, int G, bool GATHER, bool POOL>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
-    // 256-key tiles for one FP8 query row per tile; two epilogue groups whenever the TMEM
-    // accumulators split evenly between them
-    constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 2 : 1;
+    // 384-key tiles for one FP8 query row per tile (fewer barrier waits and commits per key
+    // for the single MMA-issuing thread); two epilogue groups whenever the TMEM accumulators
+    // split evenly between them
+    constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 3 : 1;
     constexpr int kAccCols = TM * NQ;
     constexpr int ACC = kAccCols <= 128 ? 4 : kAccCols <= 256 ? 2 : 1;
     constexpr int EPI = (ACC % 2 == 0 && G <= 2) ? 2 : 1;
@@ -665,7 +670,7 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     memset(&mq, 0, sizeof mq);
     if (!make_map(&mq, a.q, (int64_t)a.rows * a.H_I, esz, NQ)) return cudaErrorInvalidValue;
     if (!a.gather &&
-        !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, scan_tile_rows(a.G, a.gather, esz)))
+        !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, kTileRows))
         return cudaErrorInvalidValue;
     ScanParams p;
     p.rows = a.rows;
@@ -718,7 +723,7 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
 }
 
 int scan_tile_rows(int G, bool gather, int esz) {
-    return (G == 1 && !gather && esz == 1) ? 2 * kTileRows : kTileRows;
+    return (G == 1 && !gather && esz == 1) ? 3 * kTileRows : kTileRows;
 }
 
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
