@@ -23,6 +23,9 @@
 //               ReLU-weighted head sum in fp32, coalesced score stores, shared-memory
 //               histogram of the top 12 key bits per query row (first radix-select digit),
 //               8-entry block maxima.
+//               The histograms hold two 16-bit bins per word (half the shared memory, one
+//               more stage in the ring) and are added to global memory before a bin could
+//               pass 65,535.
 // Every wait is bounded (2 s) and sets CSA2_DEV_TIMEOUT instead of hanging.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -34,6 +37,7 @@ namespace csa2 {
 
 constexpr int kTileRows = 128;  // keys per tile (MMA M, TMEM lanes)
 constexpr int kBins = 4096;     // first radix digit: key >> 20
+constexpr int kHW = kBins / 2;  // histogram words in shared memory (two 16-bit bins each)
 
 struct ScanParams {
     int rows;               // query rows R (B*T)
@@ -64,9 +68,10 @@ struct ScanSmem {
     static constexpr int kQBytes = NQ * 128 * ESZ;
     static constexpr int kStageOff = 0;
     static constexpr int kQOff = kStageOff + STAGES * kTileBytes;
+    // histograms: two 16-bit bins per 32-bit word (flushed before a bin can overflow)
     static constexpr int kHistOff = kQOff + 2 * kQBytes;
-    static constexpr int kBHistOff = kHistOff + EPI * G * kBins * 4;
-    static constexpr int kWOff = kBHistOff + (POOL ? EPI * kBins * 4 : 0);
+    static constexpr int kBHistOff = kHistOff + EPI * G * kBins * 2;
+    static constexpr int kWOff = kBHistOff + (POOL ? EPI * kBins * 2 : 0);
     static constexpr int kBarOff = kWOff + EPI * 2 * NQ * 4;
     static constexpr int kNumBars = 2 * STAGES + 4 + 2 * ACC + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
@@ -201,9 +206,9 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         fence_mbar_init();
     }
     if (warp >= kEpiWarp0) {
-        for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * G * kBins; i += 128 * EPI) hist_s[i] = 0;
+        for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * G * kHW; i += 128 * EPI) hist_s[i] = 0;
         if (POOL)
-            for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * kBins; i += 128 * EPI) bhist_s[i] = 0;
+            for (int i = threadIdx.x - 32 * kEpiWarp0; i < EPI * kHW; i += 128 * EPI) bhist_s[i] = 0;
     }
     if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
     if (warp == 0 && lane == 0 && !GATHER) {
@@ -365,8 +370,34 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         const int et = threadIdx.x - 32 * kEpiWarp0 - 128 * e;  // 0..127 within the group
         const int row = 32 * (warp & 3) + lane;     // TMEM lane == key row within a half
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
-        uint32_t* hist_e = hist_s + e * G * kBins;
-        uint32_t* bhist_e = bhist_s + e * kBins;
+        uint32_t* hist_e = hist_s + e * G * kHW;
+        uint32_t* bhist_e = bhist_s + e * kHW;
+        // adds the group's shared histograms of row group g into global memory and clears them
+        auto flush = [&](int g) {
+            for (int gg = 0; gg < G; ++gg)
+                for (int i = et; i < kHW; i += 128) {
+                    const uint32_t v = hist_e[gg * kHW + i];
+                    if (v) {
+                        uint32_t* dst = p.hist + (int64_t)(g * G + gg) * kBins + 2 * i;
+                        if (v & 0xFFFFu) atomicAdd(dst, v & 0xFFFFu);
+                        if (v >> 16) atomicAdd(dst + 1, v >> 16);
+                        hist_e[gg * kHW + i] = 0;
+                    }
+                }
+            if (POOL)
+                for (int i = et; i < kHW; i += 128) {
+                    const uint32_t v = bhist_e[i];
+                    if (v) {
+                        uint32_t* dst = p.bhist + (int64_t)(g * G) * kBins + 2 * i;
+                        if (v & 0xFFFFu) atomicAdd(dst, v & 0xFFFFu);
+                        if (v >> 16) atomicAdd(dst + 1, v >> 16);
+                        bhist_e[i] = 0;
+                    }
+                }
+        };
+        // a bin gains at most kRowsT per iteration: flush before 65,535 could be passed
+        constexpr int kFlushEvery = 65535 / kRowsT;
+        int since_flush = 0;
         float* w_e = w_s + e * 2 * NQ;
         GroupCursor cur;
         cur.init(p.prefix, ngroups, t0);
@@ -382,24 +413,8 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             if (cur.g != gcur) {
                 // flush the previous row group's histograms, then load the new weights
                 epi_bar_sync(e);
-                if (gcur >= 0) {
-                    for (int gg = 0; gg < G; ++gg)
-                        for (int i = et; i < kBins; i += 128) {
-                            const uint32_t v = hist_e[gg * kBins + i];
-                            if (v) {
-                                atomicAdd(p.hist + (int64_t)(gcur * G + gg) * kBins + i, v);
-                                hist_e[gg * kBins + i] = 0;
-                            }
-                        }
-                    if (POOL)
-                        for (int i = et; i < kBins; i += 128) {
-                            const uint32_t v = bhist_e[i];
-                            if (v) {
-                                atomicAdd(p.bhist + (int64_t)(gcur * G) * kBins + i, v);
-                                bhist_e[i] = 0;
-                            }
-                        }
-                }
+                if (gcur >= 0) flush(gcur);
+                since_flush = 0;
                 wslot ^= 1;
                 for (int i = et; i < NQ; i += 128)
                     w_e[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
@@ -412,6 +427,13 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                 for (int gg = 0; gg < G; ++gg) nvis[gg] = __ldg(p.n_row + r0 + gg);
                 gcur = cur.g;
             }
+            if (since_flush == kFlushEvery) {
+                epi_bar_sync(e);
+                flush(gcur);
+                epi_bar_sync(e);
+                since_flush = 0;
+            }
+            ++since_flush;
             const int a = (int)(it % ACC);
             aborted = aborted || *abort_flag;
             if (!aborted) {
@@ -472,7 +494,8 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                         const uint32_t bin = vis ? (key >> 20) : 0xFFFFFFFFu;
                         const uint32_t peers = __match_any_sync(0xffffffffu, bin);
                         if (vis && (lane == __ffs(peers) - 1))
-                            atomicAdd(&hist_e[gg * kBins + bin], (uint32_t)__popc(peers));
+                            atomicAdd(&hist_e[gg * kHW + (bin >> 1)],
+                                      (uint32_t)__popc(peers) << (16 * (bin & 1)));
                     }
                     if (POOL) {
                         uint32_t bk = vis ? key : 0u;
@@ -484,25 +507,14 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                         const uint32_t bbin = lead ? (bk >> 20) : 0xFFFFFFFFu;
                         const uint32_t peers = __match_any_sync(0xffffffffu, bbin);
                         if (lead && (lane == __ffs(peers) - 1))
-                            atomicAdd(&bhist_e[bbin], (uint32_t)__popc(peers));
+                            atomicAdd(&bhist_e[bbin >> 1], (uint32_t)__popc(peers) << (16 * (bbin & 1)));
                     }
                 }
             }
         }
         // final flush
         epi_bar_sync(e);
-        if (gcur >= 0) {
-            for (int gg = 0; gg < G; ++gg)
-                for (int i = et; i < kBins; i += 128) {
-                    const uint32_t v = hist_e[gg * kBins + i];
-                    if (v) atomicAdd(p.hist + (int64_t)(gcur * G + gg) * kBins + i, v);
-                }
-            if (POOL)
-                for (int i = et; i < kBins; i += 128) {
-                    const uint32_t v = bhist_e[i];
-                    if (v) atomicAdd(p.bhist + (int64_t)(gcur * G) * kBins + i, v);
-                }
-        }
+        if (gcur >= 0) flush(gcur);
     }
     tc_fence_before();
     __syncthreads();
