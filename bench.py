@@ -195,7 +195,7 @@ class Decode:
                 n += 3 + (1 if self.w.pool else 0)   # prep, scan, Top-K (+ pool Top-K)
             elif m == "reindex":
                 n += 3
-            n += 2 + (1 if csa2_attn_splits(self.w) > 1 else 0)   # stage, attention (+ merge)
+            n += csa2.sparse_attn_decode_launches(self.w.B, self.w.K, synth.WINDOW)
         return n
 
     def step_inputs(self):
@@ -393,14 +393,6 @@ def measured_bf16_tflops():
         with open(p) as f:
             return float(json.load(f)["bf16_tflops"])
     return 1590.0
-
-
-def csa2_attn_splits(w):
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    nch = (w.K + synth.WINDOW + 127) // 128
-    ns = min(nch, (2 * sms + w.B - 1) // w.B)
-    cps = (nch + ns - 1) // ns
-    return (nch + cps - 1) // cps
 
 
 def _main_rows(w, seed, b, dev):

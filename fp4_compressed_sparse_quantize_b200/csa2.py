@@ -23,7 +23,7 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_sparse_attn_prefill", "csa2_workspace_bytes", "csa2_status_string",
            "csa2_read_device_status", "csa2_reset_device_status", "csa2_version",
            "csa2_debug_bounded_wait", "csa2_set_stage_events",
-           "csa2_index_score_topk_noalloc")
+           "csa2_index_score_topk_noalloc", "csa2_sparse_attn_decode_launches")
 
 
 class Csa2Error(RuntimeError):
@@ -61,6 +61,7 @@ def lib():
         L.csa2_set_stage_events.argtypes = [P, P]
         L.csa2_index_score_topk_noalloc.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P,
                                                     i32, P, i32, P, i32, P, i32, P, P, P, P]
+        L.csa2_sparse_attn_decode_launches.argtypes = [i32, i32, i32]
         for name in EXPORTS:
             if name not in ("csa2_workspace_bytes", "csa2_status_string"):
                 getattr(L, name).restype = i32
@@ -105,6 +106,11 @@ def _need(t, dtype, name, dev=True):
 def workspace_bytes(op, B, T, H, cap, K, pool_blocks=0):
     return int(lib().csa2_workspace_bytes(int(op), int(B), int(T), int(H), int(cap), int(K),
                                           int(pool_blocks)))
+
+
+def sparse_attn_decode_launches(B, K, W):
+    """Kernels one sparse_attn_decode call launches on the current device (see csa2.h)."""
+    return int(lib().csa2_sparse_attn_decode_launches(int(B), int(K), int(W)))
 
 
 def new_workspace(nbytes, device="cuda"):

@@ -193,6 +193,11 @@ csa2_status_t csa2_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
                                           cap, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int csa2_sparse_attn_decode_launches(int B, int K, int W) {
+    if (B < 1 || K < 0 || W < 0 || W > 1024 || K > 65536) return -1;
+    return attention_decode_launches(B, K, W);
+}
+
 size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t cap, int K,
                             int pool_blocks) {
     if (B < 1 || T < 1 || H < 1 || cap < 1 || K < 0) return 0;

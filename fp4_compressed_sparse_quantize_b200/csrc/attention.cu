@@ -85,11 +85,12 @@ int attention_splits(int Q, int K, int W, bool prefill) {
     return (rows + rps - 1) / rps;
 }
 
-cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st);
+cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merged);
 
 cudaError_t launch_attention(const AttnLaunch& l, cudaStream_t st) {
-    cudaError_t e = launch_attention_tc(l, st);
-    if (e != cudaSuccess || l.nsplit == 1) return e;
+    bool merged = false;
+    cudaError_t e = launch_attention_tc(l, st, &merged);
+    if (e != cudaSuccess || l.nsplit == 1 || merged) return e;
     return launch_pdl(attn_combine_kernel, dim3((unsigned)l.Q, (unsigned)l.H), dim3(128), 0, st,
                       (const float*)l.partial, l.nsplit, l.H, l.out);
 }

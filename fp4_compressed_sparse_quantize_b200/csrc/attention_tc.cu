@@ -38,6 +38,8 @@
 // A CTA with several chunks (prefill) first sweeps them for the exact per-head maximum,
 // then sweeps again to accumulate P x V, so no accumulator is ever rescaled.
 #include <cuda.h>
+#include <map>
+#include <mutex>
 #include <cudaTypedefs.h>
 
 #include "csa2_common.cuh"
@@ -684,6 +686,9 @@ __device__ __forceinline__ float hi11(float p) {
     return __uint_as_float((__float_as_uint(p) + 0x1000u) & 0xFFFFE000u);
 }
 
+// CL: the nsplit CTAs of one query form a thread-block cluster and merge their partial
+// results through distributed shared memory (no partials in global memory, no merge kernel).
+template <bool CL>
 __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                              const __grid_constant__ CUtensorMap tmap_q,
                                                              const __grid_constant__ CUtensorMap tmap_o,
@@ -893,22 +898,93 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
             }
         }
     }
-    if (ok && a.nsplit > 1 && warp == 0) {
-        float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
-        for (int x = lane; x < a.H; x += 32) {
-            ml[x] = m_s[x];
-            ml[a.H + x] = l_s[x];
+    if constexpr (CL) {
+        // every split of this query has its (max, sum) and unnormalised output tile in shared
+        // memory; CTA k of the cluster finishes the 32-channel boxes b = k (mod nsplit): it
+        // reads box b of every split, weights them by 2^(m_s - M) and divides by the merged
+        // sum. Box b of this CTA is read by this CTA only, so it is overwritten in place.
+        const uint32_t ns = (uint32_t)a.nsplit, k = cluster_rank();
+        float* wgt = tail + 1024;    // [8 splits][64 heads]
+        float* ginv = tail + 1536;   // [64 heads]
+        cluster_sync_all();
+        if (tid < kHeads) {
+            float mv[8], lv[8], M = -INFINITY;
+#pragma unroll
+            for (uint32_t sp = 0; sp < 8; ++sp) {
+                mv[sp] = -INFINITY;
+                lv[sp] = 0.f;
+                if (sp < ns) {
+                    mv[sp] = __uint_as_float(ld_peer_u32(peer_addr(&m_s[tid], sp)));
+                    lv[sp] = __uint_as_float(ld_peer_u32(peer_addr(&l_s[tid], sp)));
+                    M = fmaxf(M, mv[sp]);
+                }
+            }
+            const float Mb = (M == -INFINITY) ? 0.f : M;
+            float L = 0.f;
+#pragma unroll
+            for (uint32_t sp = 0; sp < 8; ++sp) {
+                if (sp < ns) {
+                    const float wv = exp2f(mv[sp] - Mb);
+                    L += wv * lv[sp];
+                    wgt[sp * kHeads + tid] = wv;
+                }
+            }
+            ginv[tid] = L > 0.f ? 1.f / L : 0.f;
         }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && ok) {
+        __syncthreads();
 #pragma unroll 1
-        for (int b = 0; b < 16; ++b)
-            tma_store_3d(&tmap_o, osm + b * (kHeads * 32), 32 * b, 0, oblk);
-        bulk_commit();
-        bulk_wait_all();
+        for (uint32_t bx = k; bx < 16; bx += ns) {
+#pragma unroll
+            for (int u0 = 0; u0 < 512; u0 += 256) {
+                const int u = u0 + tid, hh = u >> 3, ch = u & 7;
+                const int off = (int)bx * (kHeads * 32) + hh * 32 + ((ch ^ (hh & 7)) << 2);
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (uint32_t sp = 0; sp < 8; ++sp) {
+                    if (sp < ns) {
+                        const float4 v = sp == k ? *reinterpret_cast<const float4*>(osm + off)
+                                                 : ld_peer_f4(peer_addr(osm + off, sp));
+                        const float wv = wgt[sp * kHeads + hh];
+                        acc.x += wv * v.x;
+                        acc.y += wv * v.y;
+                        acc.z += wv * v.z;
+                        acc.w += wv * v.w;
+                    }
+                }
+                const float iv = ginv[hh];
+                *reinterpret_cast<float4*>(osm + off) =
+                    make_float4(acc.x * iv, acc.y * iv, acc.z * iv, acc.w * iv);
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+#pragma unroll 1
+            for (uint32_t bx = k; bx < 16; bx += ns)
+                tma_store_3d(&tmap_o, osm + bx * (kHeads * 32), 32 * (int)bx, 0, qrow);
+            bulk_commit();
+            bulk_wait_all();
+        }
+        cluster_sync_all();   // the other splits have finished reading this CTA's tiles
+    } else {
+        if (ok && a.nsplit > 1 && warp == 0) {
+            float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
+            for (int x = lane; x < a.H; x += 32) {
+                ml[x] = m_s[x];
+                ml[a.H + x] = l_s[x];
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+#pragma unroll 1
+            for (int b = 0; b < 16; ++b)
+                tma_store_3d(&tmap_o, osm + b * (kHeads * 32), 32 * b, 0, oblk);
+            bulk_commit();
+            bulk_wait_all();
+        }
     }
     if (tid == 0 && !loads_ok)   // a load that timed out may still be in flight: bounded
         for (int j = 0; j < 8; ++j) mbar_wait(&bar[j], 0, a.status);
@@ -974,7 +1050,50 @@ size_t attention_stage_bytes(int Q, int rows) {
            (size_t)Q * rows * 4 + 4 * 256;
 }
 
-cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
+// Whether the decode splits of every query can run as clusters in one wave (the merge then
+// happens in distributed shared memory). Looked up once per (splits, shared memory) shape.
+static bool cluster_merge_fits(int Q, int nsplit, int dsmem) {
+    if (nsplit < 2 || nsplit > 8) return false;
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(nsplit, dsmem);
+    auto it = cache.find(key);
+    if (it == cache.end()) {
+        int n = 0;
+        if (cudaFuncSetAttribute(attn_decode_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem) == cudaSuccess) {
+            cudaLaunchConfig_t cfg;
+            memset(&cfg, 0, sizeof cfg);
+            cfg.gridDim = dim3(1, (unsigned)nsplit);
+            cfg.blockDim = dim3(256);
+            cfg.dynamicSmemBytes = dsmem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = (unsigned)nsplit;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, attn_decode_kernel<true>, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();   // a refused query leaves no sticky error
+        it = cache.emplace(key, n).first;
+    }
+    return it->second >= Q;
+}
+
+int attention_decode_launches(int Q, int K, int W) {
+    const int rows = K + W;
+    if (rows <= 0) return 1;
+    const int nsplit = attention_splits(Q, K, W, false);
+    if (nsplit == 1) return 2;   // stage + attention
+    const int rps = attention_rows_per_split(rows, nsplit);
+    return cluster_merge_fits(Q, nsplit, DecSmem(rps).bytes() + 1024) ? 2 : 3;
+}
+
+cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merged) {
+    *merged = false;
     TcAttnDev a;
     memset(&a, 0, sizeof a);
     a.Q = l.Q;
@@ -1032,16 +1151,42 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st) {
                                    dim3((unsigned)l.Q, (unsigned)(row_blocks + kHeads / 8)),
                                    dim3(256), 0, st, a, xg, qg, qfg, validg, row_blocks);
         if (e != cudaSuccess) return e;
+        const int dsmem = DecSmem(rps).bytes() + 1024;
         CUtensorMap mos;
         memset(&mos, 0, sizeof mos);
+        if (l.nsplit > 1 && cluster_merge_fits(l.Q, l.nsplit, dsmem)) {
+            // the splits of a query form one cluster and write the final output themselves
+            if (!out_map_sw(&mos, l.out, l.H, l.Q)) return cudaErrorInvalidValue;
+            e = cudaFuncSetAttribute(attn_decode_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem);
+            if (e != cudaSuccess) return e;
+            cudaLaunchConfig_t cfg;
+            memset(&cfg, 0, sizeof cfg);
+            cfg.gridDim = grid;
+            cfg.blockDim = dim3(256);
+            cfg.dynamicSmemBytes = dsmem;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = (unsigned)l.nsplit;
+            attr[0].val.clusterDim.z = 1;
+            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 2;
+            e = cudaLaunchKernelEx(&cfg, attn_decode_kernel<true>, mx, mq, mos, a, rps);
+            if (e == cudaSuccess) *merged = true;
+            return e;
+        }
         if (l.nsplit > 1 ? !out_map_sw(&mos, l.partial, l.H, (int64_t)l.Q * l.nsplit)
                          : !out_map_sw(&mos, l.out, l.H, l.Q))
             return cudaErrorInvalidValue;
-        const int dsmem = DecSmem(rps).bytes() + 1024;
-        e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsmem);
+        e = cudaFuncSetAttribute(attn_decode_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(attn_decode_kernel, grid, dim3(256), (size_t)dsmem, st, mx, mq, mos, a, rps);
+        return launch_pdl(attn_decode_kernel<false>, grid, dim3(256), (size_t)dsmem, st, mx, mq,
+                          mos, a, rps);
     }
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

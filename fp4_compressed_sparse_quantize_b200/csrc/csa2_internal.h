@@ -124,6 +124,8 @@ size_t attention_stage_bytes(int Q, int rows);
 // (a multiple of 32), as many as fill one wave of CTAs; prefill never splits.
 constexpr int kAttnDecodeRows = 160;
 int attention_splits(int Q, int K, int W, bool prefill);
+// kernels one decode attention call launches for Q queries (stage, attention, merge or not)
+int attention_decode_launches(int Q, int K, int W);
 int attention_rows_per_split(int rows, int nsplit);
 
 int device_sm_count();

@@ -759,33 +759,6 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
     for (int i = npick * mult + tid; i < K * mult; i += kRowThreads) o[i] = -1;
 }
 
-// ---- cluster helpers (distributed shared memory) -------------------------------------
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
-}
-// shared::cluster address of `p` (this CTA's shared memory) in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t ld_peer_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint64_t ld_peer_u64(uint32_t addr) {
-    uint64_t v;
-    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 // CL > 1: a cluster of CL CTAs shares one row. Every CTA finds d0 and classifies its own
 // contiguous part of the row into its own lists; CTA 0 then gathers the other CTAs' lists
 // through distributed shared memory and finishes the row alone.

@@ -231,6 +231,14 @@ CSA2_API csa2_status_t csa2_index_score_topk_noalloc(
 CSA2_API size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t cap, int K,
                             int pool_blocks);
 
+/* Number of kernels one csa2_sparse_attn_decode call launches for B queries with K selected
+ * entries and W window rows on the current device: 1 with no rows, 2 (row staging +
+ * attention) when a query's rows are not split or when its splits merge inside the
+ * attention kernel (a thread-block cluster per query, when the device can hold all of them
+ * at once), 3 when a separate merge kernel combines the splits. For launch accounting and
+ * graph planning; -1 on invalid arguments. */
+CSA2_API int csa2_sparse_attn_decode_launches(int B, int K, int W);
+
 /* Static text for a status code. Never NULL. */
 CSA2_API const char* csa2_status_string(csa2_status_t status);
 
