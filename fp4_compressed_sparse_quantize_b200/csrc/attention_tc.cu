@@ -932,12 +932,53 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
             ginv[tid] = L > 0.f ? 1.f / L : 0.f;
         }
         __syncthreads();
+        // items of this thread: (box k + ns i / 2, half i mod 2 of its 512 16-byte chunks)
+        const int nitems = 2 * (int)((16 - k + ns - 1) / ns);
+        auto item_off = [&](int i) {
+            const int bx = (int)k + (int)ns * (i >> 1);
+            const int u = (i & 1) * 256 + tid, hh = u >> 3, ch = u & 7;
+            return bx * (kHeads * 32) + hh * 32 + ((ch ^ (hh & 7)) << 2);
+        };
+        if (ns <= 4) {
+            // four items at a time, every split's chunk of all four loads in flight at once
 #pragma unroll 1
-        for (uint32_t bx = k; bx < 16; bx += ns) {
+            for (int i0 = 0; i0 < nitems; i0 += 4) {
+                float4 v[4][4];
 #pragma unroll
-            for (int u0 = 0; u0 < 512; u0 += 256) {
-                const int u = u0 + tid, hh = u >> 3, ch = u & 7;
-                const int off = (int)bx * (kHeads * 32) + hh * 32 + ((ch ^ (hh & 7)) << 2);
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (uint32_t sp = 0; sp < 4; ++sp)
+                        if (i0 + j < nitems && sp < ns) {
+                            const int off = item_off(i0 + j);
+                            v[j][sp] = sp == k ? *reinterpret_cast<const float4*>(osm + off)
+                                               : ld_peer_f4(peer_addr(osm + off, sp));
+                        }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (i0 + j < nitems) {
+                        const int off = item_off(i0 + j);
+                        const int hh = ((((i0 + j) & 1) * 256 + tid) >> 3);
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (uint32_t sp = 0; sp < 4; ++sp)
+                            if (sp < ns) {
+                                const float wv = wgt[sp * kHeads + hh];
+                                acc.x += wv * v[j][sp].x;
+                                acc.y += wv * v[j][sp].y;
+                                acc.z += wv * v[j][sp].z;
+                                acc.w += wv * v[j][sp].w;
+                            }
+                        const float iv = ginv[hh];
+                        *reinterpret_cast<float4*>(osm + off) =
+                            make_float4(acc.x * iv, acc.y * iv, acc.z * iv, acc.w * iv);
+                    }
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int i = 0; i < nitems; ++i) {
+                const int off = item_off(i);
+                const int hh = (((i & 1) * 256 + tid) >> 3);
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (uint32_t sp = 0; sp < 8; ++sp) {
