@@ -409,6 +409,30 @@ def _main_rows(w, seed, b, dev):
 
 # ---- CPU baseline / reference arm (the oracle as it stands) --------------------------------------
 
+def decode_config(w, world, eager):
+    return {"workload": w.name, "batch_per_gpu": w.B, "context_tokens": w.ctx,
+            "launch": "eager" if eager else "cuda graph replay per step",
+            "ratio": w.ratio, "compressed_entries": w.N, "topk": w.K,
+            "indexer_heads": w.H_I, "indexer_dtype": w.idx_dtype, "query_heads": w.H,
+            "window": synth.WINDOW, "layers": list(w.layers),
+            "parallelism": f"dp{world} (independent batches)",
+            "l2": "flushed between steps (256 MiB write + read, outside the timed events)"}
+
+
+class RefInputs:
+    """The seeded inputs of a decode workload without any library work (reference arm)."""
+
+    def __init__(self, w, seed, dev):
+        self.w, self.seed, self.dev = w, seed, dev
+        self.tau = 1.0 / math.sqrt(synth.D_MAIN)
+        self.layers = [synth.layer_inputs(w, li, seed, dev) for li in range(len(w.layers))]
+        dirs = None
+        if w.planted:
+            dirs = synth.planted_direction([L["q_I"] for L, m in zip(self.layers, w.layers)
+                                            if m in ("full", "reindex")])
+        self.k_I, _ = synth.indexer_keys(w, seed, dev, planted_dirs=dirs)
+
+
 def oracle_queries(state, budget_s):
     """Run the oracle over whole decode queries of this workload until ~budget_s of CPU work;
     returns (queries done, seconds, cores)."""
@@ -593,13 +617,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": per_step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3/fp4/fp16 (fp32 accumulate)", "data": "synthetic",
-            "config": {"workload": args.workload, "batch_per_gpu": w.B, "context_tokens": w.ctx,
-                       "launch": "eager" if args.eager else "cuda graph replay per step",
-                       "ratio": w.ratio, "compressed_entries": w.N, "topk": w.K,
-                       "indexer_heads": w.H_I, "indexer_dtype": w.idx_dtype, "query_heads": w.H,
-                       "window": synth.WINDOW, "layers": list(w.layers),
-                       "parallelism": f"dp{world} (independent batches)",
-                       "l2": "flushed between steps (256 MiB write + read, outside the timed events)"},
+            "config": decode_config(w, world, args.eager),
             "hbm_gbs_step": alg_bytes / (per_step_ms / 1e3) / 1e9,
             "roofline": {"kernel": "csa2 indexer scan (tcgen05, FP8 keys)", "bound": "hbm",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -629,7 +647,7 @@ def reference_arm(args, rank, world, local):
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     if dev.type == "cuda":
         torch.cuda.set_device(local)
-    state = Decode(w, args.seed, dev)
+    state = RefInputs(w, args.seed, dev)
     # each step is a bounded sample: whole queries until ~budget/steps seconds
     per = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -645,7 +663,7 @@ def reference_arm(args, rank, world, local):
             "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * s_tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "batch_per_gpu": w.B},
+            "data": "synthetic", "config": decode_config(w, world, args.eager),
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores,
                              "kind": "oracle",
                              "sample": f"{n_tot} whole decode queries over {args.steps} steps"},
