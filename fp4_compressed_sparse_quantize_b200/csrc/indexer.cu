@@ -19,6 +19,8 @@
 //               row group.
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128 keys,
 //               N = G queries x H_I heads, K = 128 channels) into a TMEM accumulator ring.
+//   warp 2      does warp 1's mbarrier waits one tile ahead and hands each tile over at a
+//               named barrier (a wait behind in-flight MMA commits is slow).
 //   then EPI    epilogue groups of 4 warps: tcgen05.ld of one key row per thread,
 //               ReLU-weighted head sum in fp32, coalesced score stores, shared-memory
 //               histogram of the top 12 key bits per query row (first radix-select digit),
@@ -83,6 +85,9 @@ struct ScanSmem {
 __device__ __forceinline__ void epi_bar_sync(int group) {
     asm volatile("bar.sync %0, 128;" ::"r"(group + 1) : "memory");
 }
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 // Last row group g with prefix[g] <= t.
 __device__ __forceinline__ int find_group(const int64_t* prefix, int ngroups, int64_t t) {
@@ -138,11 +143,10 @@ __device__ __forceinline__ void fence_proxy_async() {
 // ESZ    = 1 (E4M3, kind::f8f6f4) or 2 (bf16, kind::f16)
 // GATHER = Reindex: tile rows come from a pool list instead of a contiguous range
 // TM     = 128-key halves per tile (one TMA box, TM MMA groups into adjacent TMEM columns)
-// One thread issues every tcgen05.mma of the CTA. (Issuing from two warps on alternate
-// tiles was faster but intermittently never completed an MMA commit on the 256K-context
-// workload, so the MMA issue stays with a single thread.)
-constexpr int kIssuers = 1;                       // MMA-issuing warps
-constexpr int kEpiWarp0 = 1 + kIssuers;           // first epilogue warp
+// One thread issues every tcgen05.mma of the CTA (warp 1); warp 2 does its barrier waits.
+// (Issuing from two warps on alternate tiles intermittently never completed an MMA commit
+// on the 256K-context workload.)
+constexpr int kEpiWarp0 = 3;                      // first epilogue warp
 
 template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM>
 __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
@@ -195,13 +199,13 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qfull[s], 1);
-            mbar_init(&qempty[s], kIssuers);   // every issuer releases the query slot
+            mbar_init(&qempty[s], 1);
         }
         for (int s = 0; s < ACC; ++s) {
             mbar_init(&accfull[s], 1);
             mbar_init(&accempty[s], 4);
         }
-        mbar_init(done_bar, kIssuers);
+        mbar_init(done_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -308,54 +312,78 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                 mbar_wait(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), p.status);
             if (qcount > 0) mbar_wait(&qfull[(qcount - 1) & 1], ((qcount - 1) >> 1) & 1, p.status);
         }
-    } else if (warp <= kIssuers) {
-        // ------------------------------------------------------------ MMA issuers
-        // issuer m issues the tiles it == m (mod kIssuers) but follows every row-group
-        // change, so that each issuer releases every query slot
-        const int m = warp - 1;
-        if (lane == 0) {
-            GroupCursor cur;
-            cur.init(p.prefix, ngroups, t0);
-            int qg = -1, qcount = 0, qs = 0;
-            int64_t it = 0;
-            const uint64_t a_desc0 = sw128_desc(smem_u32(stage_base), 16, 1024);
-            const uint64_t b_desc0 = sw128_desc(smem_u32(q_base), 16, 1024);
-            for (int64_t t = t0; t < t1; ++t, ++it) {
-                if (*abort_flag) break;
-                cur.advance(p.prefix, t);
-                if (cur.g != qg) {
-                    if (qg >= 0) mma_commit(&qempty[qs]);
-                    qs = qcount & 1;
-                    if (!mbar_wait(&qfull[qs], (qcount >> 1) & 1, p.status)) { *abort_flag = 1; break; }
-                    qg = cur.g;
-                    ++qcount;
+    } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------------ MMA issue (warp 1)
+        // and its barrier waits (warp 2). An mbarrier wait by the thread whose MMAs and
+        // commits are still in flight costs a few hundred cycles even on a completed phase,
+        // so the issuing thread never waits on an mbarrier: warp 2 waits for tile t+1's key
+        // tile, accumulator and query slot while warp 1 issues tile t, and the two meet at a
+        // named barrier once per tile. The waiter's verdict (go / abort) crosses with it, so
+        // both warps always take the same number of hand-overs.
+        volatile int* go_flag = abort_flag + 1;
+        const bool waiter = warp == 2;
+        GroupCursor cur;
+        cur.init(p.prefix, ngroups, t0);
+        int qg = -1, qcount = 0, qs = 0;
+        int64_t it = 0;
+        const uint64_t a_desc0 = sw128_desc(smem_u32(stage_base), 16, 1024);
+        const uint64_t b_desc0 = sw128_desc(smem_u32(q_base), 16, 1024);
+        for (int64_t t = t0; t < t1; ++t, ++it) {
+            cur.advance(p.prefix, t);
+            const bool newgroup = cur.g != qg;
+            const int qs_new = newgroup ? (qcount & 1) : qs;
+            const int s = (int)(it % STAGES);
+            const int a = (int)(it % ACC);
+            if (waiter) {
+                bool ok = true;
+                if (lane == 0) {
+                    ok = !*abort_flag;
+                    if (ok && newgroup)
+                        ok = mbar_wait(&qfull[qs_new], (uint32_t)((qcount >> 1) & 1), p.status);
+                    if (ok) ok = mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), p.status);
+                    if (ok) ok = mbar_wait(&accempty[a], (uint32_t)(((it / ACC) & 1) ^ 1), p.status);
+                    if (!ok) *abort_flag = 1;
+                    *go_flag = ok ? 1 : 0;
                 }
-                if ((int)(it % kIssuers) != m) continue;
-                const int s = (int)(it % STAGES);
-                if (!mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), p.status)) { *abort_flag = 1; break; }
-                const int a = (int)(it % ACC);
-                if (!mbar_wait(&accempty[a], (uint32_t)(((it / ACC) & 1) ^ 1), p.status)) { *abort_flag = 1; break; }
-                tc_fence_after();
-                // descriptor start addresses advance in 16-byte units
-                const uint64_t a_s = a_desc0 + ((uint64_t)(s * L::kTileBytes) >> 4);
-                const uint64_t b_s = b_desc0 + ((uint64_t)(qs * L::kQBytes) >> 4);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                named_bar_sync(15, 64);
+                if (!ok) break;
+            } else {
+                // the previous row group's query slot is free once this thread's MMAs are done
+                if (lane == 0 && newgroup && qg >= 0) mma_commit(&qempty[qs]);
+                named_bar_sync(15, 64);
+                if (!*go_flag) break;
+                if (lane == 0) {
+                    tc_fence_after();
+                    // descriptor start addresses advance in 16-byte units
+                    const uint64_t a_s = a_desc0 + ((uint64_t)(s * L::kTileBytes) >> 4);
+                    const uint64_t b_s = b_desc0 + ((uint64_t)(qs_new * L::kQBytes) >> 4);
 #pragma unroll
-                for (int hh = 0; hh < TM; ++hh) {
-                    const uint32_t d = tmem_base + a * kAccCols + hh * NQ;
+                    for (int hh = 0; hh < TM; ++hh) {
+                        const uint32_t d = tmem_base + a * kAccCols + hh * NQ;
 #pragma unroll
-                    for (int kk = 0; kk < kKSteps; ++kk) {
-                        const uint64_t ad = a_s + ((uint64_t)((kk >> 2) * kSlab + hh * 128 * 128 +
-                                                              (kk & 3) * 32) >> 4);
-                        const uint64_t bd = b_s + ((uint64_t)((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
-                        if (ESZ == 1)
-                            mma_f8(d, ad, bd, kIdesc, kk > 0);
-                        else
-                            mma_f16(d, ad, bd, kIdesc, kk > 0);
+                        for (int kk = 0; kk < kKSteps; ++kk) {
+                            const uint64_t ad = a_s + ((uint64_t)((kk >> 2) * kSlab + hh * 128 * 128 +
+                                                                  (kk & 3) * 32) >> 4);
+                            const uint64_t bd = b_s + ((uint64_t)((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
+                            if (ESZ == 1)
+                                mma_f8(d, ad, bd, kIdesc, kk > 0);
+                            else
+                                mma_f16(d, ad, bd, kIdesc, kk > 0);
+                        }
                     }
+                    mma_commit(&empty[s]);
+                    mma_commit(&accfull[a]);
                 }
-                mma_commit(&empty[s]);
-                mma_commit(&accfull[a]);
+                __syncwarp();
             }
+            if (newgroup) {
+                qs = qs_new;
+                qg = cur.g;
+                ++qcount;
+            }
+        }
+        if (!waiter && lane == 0) {
             // all MMAs must complete before TMEM is released
             mma_commit(done_bar);
             mbar_wait(done_bar, 0, p.status);

@@ -550,7 +550,7 @@ struct RowState {
 template <int PER, class IdOf>
 __device__ __forceinline__ void row_classify(const TopkDev& a, const RowState& S, int r,
                                              const uint32_t (&key)[PER], IdOf ID,
-                                             uint32_t valid, bool many, int d0) {
+                                             uint32_t valid, bool many, int d0, int ccap) {
     uint32_t wmask = 0, cmask = 0;
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
@@ -580,7 +580,7 @@ __device__ __forceinline__ void row_classify(const TopkDev& a, const RowState& S
         } else {
             const uint64_t c = ((uint64_t)kk << 32) | (uint64_t)(~id);
             if (pc < (uint32_t)kRowCands) S.cand_s[pc] = c;
-            else if (pc < (uint32_t)a.ccap) gcand[pc] = c;
+            else if (pc < (uint32_t)ccap) gcand[pc] = c;
             ++pc;
         }
         wm &= ~bit;
@@ -623,7 +623,7 @@ __device__ __forceinline__ void row_threshold(const RowState& S, const uint32_t 
 // Refinement, picks and the ordered output of one row, after every element was classified.
 template <bool GATHER>
 __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t n,
-                             uint32_t id_lim, bool many, int d0, uint32_t above) {
+                             uint32_t id_lim, bool many, int d0, uint32_t above, int ccap) {
     const int tid = threadIdx.x;
     const int K = a.K;
     const bool use_bm = a.bitmap_words > 0;
@@ -637,7 +637,7 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
 
     if (many) {
         const uint32_t need = (uint32_t)K - above;
-        const bool from_row = ncand > (uint32_t)max(a.ccap, kRowCands);
+        const bool from_row = ncand > (uint32_t)max(ccap, kRowCands);
         const int64_t nsrc = from_row ? n : (int64_t)ncand;
         // candidate i of the source (false: not a candidate)
         auto cand = [&](int64_t i, uint64_t& c) -> bool {
@@ -763,10 +763,10 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
 // contiguous part of the row into its own lists; CTA 0 then gathers the other CTAs' lists
 // through distributed shared memory and finishes the row alone.
 template <bool GATHER, int CL>
-__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a_in) {
+__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a) {
     static_assert(!GATHER || CL == 1, "gather rows are short: one CTA each");
-    TopkDev a = a_in;
-    if (CL > 1) a.ccap = 0;   // per-CTA candidate lists live in shared memory only
+    // with a cluster, every CTA's candidate list lives in shared memory only
+    const int ccap = CL > 1 ? 0 : a.ccap;
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ uint32_t wsum[40];
     __shared__ int dig_s[4];
@@ -826,13 +826,13 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
                 const int64_t i = base + (int64_t)k * kRowThreads + tid;
                 if (i < n && (int32_t)id[k] >= 0 && id[k] < id_lim) valid |= 1u << k;
             }
-            row_classify<PER>(a, S, r, key, [&](int k) { 
+            row_classify<PER>(a, S, r, key, [&](int k) {
                 uint32_t v = 0;
 #pragma unroll
                 for (int j = 0; j < PER; ++j)
                     if (j == k) v = id[j];
                 return v;
-            }, valid, many, d0);
+            }, valid, many, d0, ccap);
         }
     } else {
         // ---- positions: histogram and elements through bulk copies -------------------------
@@ -906,7 +906,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
             const uint32_t idb = (uint32_t)(h0 + pb + e0 + tid);
             row_classify<kRowPer + 1>(a, S, r, key, [&](int k) {
                 return k < kRowPer ? idb + (uint32_t)k * kRowThreads : (uint32_t)xi;
-            }, valid, many, d0);
+            }, valid, many, d0, ccap);
             // every thread has read buffer (c & 1): refill it with chunk c + 2
             if (tid == 0 && ok && c + 2 < nch) issue(c + 2);
         }
@@ -940,7 +940,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
         cluster_sync_all();   // the other CTAs' lists have been read: they may exit
         if (crank != 0) return;
     }
-    row_finalize<GATHER>(a, S, r, n, id_lim, many, d0, above);
+    row_finalize<GATHER>(a, S, r, n, id_lim, many, d0, above, ccap);
 }
 
 cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
