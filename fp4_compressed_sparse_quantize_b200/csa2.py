@@ -23,7 +23,9 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_sparse_attn_prefill", "csa2_workspace_bytes", "csa2_status_string",
            "csa2_read_device_status", "csa2_reset_device_status", "csa2_version",
            "csa2_debug_bounded_wait", "csa2_set_stage_events",
-           "csa2_index_score_topk_noalloc", "csa2_sparse_attn_decode_launches")
+           "csa2_index_score_topk_noalloc", "csa2_sparse_attn_decode_launches",
+           "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
+           "csa2_cp_pool_expand")
 
 
 class Csa2Error(RuntimeError):
@@ -62,6 +64,10 @@ def lib():
         L.csa2_index_score_topk_noalloc.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P,
                                                     i32, P, i32, P, i32, P, i32, P, P, P, P]
         L.csa2_sparse_attn_decode_launches.argtypes = [i32, i32, i32]
+        L.csa2_cp_topk_candidates.argtypes = [i32, P, i64, P, i32, i64, P, P, P]
+        L.csa2_cp_pool_candidates.argtypes = [i32, P, i64, P, i32, i32, i64, P, P, P]
+        L.csa2_cp_merge.argtypes = [i32, i32, P, P, i32, P, P]
+        L.csa2_cp_pool_expand.argtypes = [i32, P, i32, P, i32, P, P]
         for name in EXPORTS:
             if name not in ("csa2_workspace_bytes", "csa2_status_string"):
                 getattr(L, name).restype = i32
@@ -256,3 +262,58 @@ def sparse_attn_prefill(q, codes, scales, idx, swa, out, ws, W, q_pos0=None, sca
                                         _p(idx), K, _p(swa), int(W), _p(q_pos0), sc, _p(out),
                                         _p(ws), ws.numel(), _stream(stream))
     _check(st, "csa2_sparse_attn_prefill")
+
+
+# ---- context parallelism (one shard of every sequence's entries per GPU) -----------------
+
+def cp_topk_candidates(scores, idx, offset, cand_score, cand_idx, stream=None):
+    """A shard's Top-K as candidates: scores fp32 [rows, ld] (the shard's scores_out),
+    idx int32 [rows, K] (shard-local, -1 padded), offset = global index of the shard's first
+    entry -> cand_score fp32 / cand_idx int32 [rows, K] (global indices, -1 padded)."""
+    for t, dt, nm in ((scores, torch.float32, "scores"), (idx, torch.int32, "idx"),
+                      (cand_score, torch.float32, "cand_score"), (cand_idx, torch.int32, "cand_idx")):
+        _need(t, dt, nm)
+    K = idx.shape[-1]
+    rows = idx.numel() // K
+    ld = scores.shape[-1]
+    _check(lib().csa2_cp_topk_candidates(rows, _p(scores), ld, _p(idx), K, int(offset),
+                                         _p(cand_score), _p(cand_idx), _stream(stream)),
+           "csa2_cp_topk_candidates")
+
+
+def cp_pool_candidates(scores, pool, offset, cand_bmax, cand_block, stream=None):
+    """A shard's candidate pool as (block maximum, global block) pairs: pool int32 [rows, P]
+    (shard-local positions), offset a multiple of 8 -> cand_bmax fp32 / cand_block int32
+    [rows, nb] (nb = the pool's block count, -1 padded)."""
+    for t, dt, nm in ((scores, torch.float32, "scores"), (pool, torch.int32, "pool"),
+                      (cand_bmax, torch.float32, "cand_bmax"), (cand_block, torch.int32, "cand_block")):
+        _need(t, dt, nm)
+    P, nb = pool.shape[-1], cand_block.shape[-1]
+    rows = pool.numel() // P
+    _check(lib().csa2_cp_pool_candidates(rows, _p(scores), scores.shape[-1], _p(pool), P, nb,
+                                         int(offset), _p(cand_bmax), _p(cand_block),
+                                         _stream(stream)), "csa2_cp_pool_candidates")
+
+
+def cp_merge(cand_score, cand_idx, idx_out, stream=None):
+    """The exact Top-K of every row from gathered candidates [rows, n_cand] into idx_out
+    int32 [rows, K]: (score desc, index asc), written in ascending index order."""
+    for t, dt, nm in ((cand_score, torch.float32, "cand_score"), (cand_idx, torch.int32, "cand_idx"),
+                      (idx_out, torch.int32, "idx_out")):
+        _need(t, dt, nm)
+    n, K = cand_idx.shape[-1], idx_out.shape[-1]
+    rows = cand_idx.numel() // n
+    _check(lib().csa2_cp_merge(rows, n, _p(cand_score), _p(cand_idx), K, _p(idx_out),
+                               _stream(stream)), "csa2_cp_merge")
+
+
+def cp_pool_expand(blocks, n_row, pool_out, stream=None):
+    """Merged pool blocks int32 [rows, nb] (ascending, -1 padded) -> entry positions int32
+    [rows, P]; n_row int32 [rows] visible entries per row (None: all)."""
+    for t, dt, nm in ((blocks, torch.int32, "blocks"), (n_row, torch.int32, "n_row"),
+                      (pool_out, torch.int32, "pool_out")):
+        _need(t, dt, nm)
+    nb, P = blocks.shape[-1], pool_out.shape[-1]
+    rows = blocks.numel() // nb
+    _check(lib().csa2_cp_pool_expand(rows, _p(blocks), nb, _p(n_row), P, _p(pool_out),
+                                     _stream(stream)), "csa2_cp_pool_expand")

@@ -287,6 +287,22 @@ __device__ __forceinline__ float key_score(uint32_t k) {
     return __uint_as_float(u);
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: each lane an IEEE fp32 operation) --------
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t x, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi), each rounded once (round to nearest even)
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // ---- small format helpers --------------------------------------------------------------
 
 // Two E4M3 bytes (low byte = first) -> two fp16 values, exactly.

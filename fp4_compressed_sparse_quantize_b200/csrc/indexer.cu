@@ -487,13 +487,19 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                         tmem_ld16(col + c * 16, vc);
                     }
                     tmem_ld_wait();
-                    // four independent accumulation chains; padding columns have weight 0
-                    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                    // four independent accumulation chains (heads h mod 4), two per packed
+                    // f32x2 FMA; padding columns have weight 0
+                    uint64_t c01 = 0ull, c23 = 0ull;
 #pragma unroll
-                    for (int h = 0; h < kCols; ++h) {
-                        const float wh = kWReg ? wr[kWReg ? h : 0] : wv[gg * kCols + h];
-                        s4[h & 3] = fmaf(wh, fmaxf(__uint_as_float(v[h]), 0.f), s4[h & 3]);
+                    for (int h = 0; h < kCols; h += 4) {
+                        auto wgt = [&](int x) { return kWReg ? wr[kWReg ? x : 0] : wv[gg * kCols + x]; };
+                        auto pos = [&](int x) { return fmaxf(__uint_as_float(v[x]), 0.f); };
+                        c01 = ffma2(f2pack(wgt(h), wgt(h + 1)), f2pack(pos(h), pos(h + 1)), c01);
+                        c23 = ffma2(f2pack(wgt(h + 2), wgt(h + 3)), f2pack(pos(h + 2), pos(h + 3)), c23);
                     }
+                    float s4[4];
+                    f2unpack(c01, s4[0], s4[1]);
+                    f2unpack(c23, s4[2], s4[3]);
                     sc[hh][gg] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + 0.0f;
                 }
             }

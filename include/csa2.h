@@ -168,7 +168,7 @@ CSA2_API csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int
  *
  *   mode      recorded and validated only: Full, Reindex and Reuse layers run the same
  *             kernel (a Reuse layer passes the earlier layer's idx).
- *   q         bf16 [B][H][512], H in 1..128.
+ *   q         bf16 [B][H][512], H in 1..64 (more heads: CSA2_ERR_UNSUPPORTED).
  *   codes, scales  main-KV cache as written by csa2_quantize_kv, capacity cap.
  *   idx       int32 [B][K]; -1 entries are skipped; other entries outside [0, cap) are
  *             skipped and set CSA2_DEV_BAD_INDEX.
@@ -238,6 +238,60 @@ CSA2_API size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t 
  * at once), 3 when a separate merge kernel combines the splits. For launch accounting and
  * graph planning; -1 on invalid arguments. */
 CSA2_API int csa2_sparse_attn_decode_launches(int B, int K, int W);
+
+/*
+ * Context parallelism: G GPUs each own a contiguous shard [lo, hi) of every sequence's
+ * compressed entries (lo a multiple of 8), run csa2_index_score_topk(FULL) on it with
+ * scores_out (and pool_out), turn the selections into candidate lists with the calls below,
+ * all-gather the lists (e.g. NCCL) and merge them. The merged Top-K and pool equal the
+  * single-GPU ones exactly. [TDG Compressed Sparse Attention 2 (CSA2)]: the Full layer keeps the 512
+ * highest-scoring entries and the 2,048 blocks of 8 with the highest block maxima; both
+ * selections decompose over shards because the order (score descending, index ascending) is
+ * total and a score depends only on its own entry. (The pages describe one GPU; sharding is
+ * this library's extension for million-entry contexts.) All pointers are device pointers,
+ * all calls asynchronous on `stream`; CSA2_ERR_ARG on bad sizes or null pointers.
+ *
+ * csa2_cp_topk_candidates — a shard's Top-K as (score, global index) pairs.
+ *   scores     fp32 [rows][ld_scores]: the shard's scores_out.
+ *   idx        int32 [rows][K]: the shard's idx_out (shard-local, -1 padded).
+ *   offset     global index of the shard's first entry (offset + ld_scores < 2^31).
+ *   cand_score fp32 [rows][K], cand_idx int32 [rows][K]: (score, offset + idx), or (0, -1).
+ */
+CSA2_API csa2_status_t csa2_cp_topk_candidates(int rows, const float* scores, int64_t ld_scores,
+                                               const int32_t* idx, int K, int64_t offset,
+                                               float* cand_score, int32_t* cand_idx,
+                                               void* stream);
+
+/*
+ * csa2_cp_pool_candidates — a shard's candidate pool as (block maximum, global block) pairs.
+ *   pool       int32 [rows][P]: the shard's pool_out (ascending shard-local positions).
+ *   max_blocks pairs per row written to cand_bmax fp32 / cand_block int32 [rows][max_blocks],
+ *              block = (offset + position) / 8, padded with (0, -1). offset % 8 == 0.
+ */
+CSA2_API csa2_status_t csa2_cp_pool_candidates(int rows, const float* scores, int64_t ld_scores,
+                                               const int32_t* pool, int P, int max_blocks,
+                                               int64_t offset, float* cand_bmax,
+                                               int32_t* cand_block, void* stream);
+
+/*
+ * csa2_cp_merge — the K best of every row's n_cand candidates by (score descending, index
+ * ascending), written to idx_out int32 [rows][K] in ascending index order, -1 padded.
+ * Candidates with index -1 are ignored; indices must be distinct. n_cand <= 8192
+ * (CSA2_ERR_UNSUPPORTED above), K <= n_cand. Used for entries (scores) and for pool blocks
+ * (block maxima) alike.
+ */
+CSA2_API csa2_status_t csa2_cp_merge(int rows, int n_cand, const float* cand_score,
+                                     const int32_t* cand_idx, int K, int32_t* idx_out,
+                                     void* stream);
+
+/*
+ * csa2_cp_pool_expand — merged pool blocks int32 [rows][nb] (ascending, -1 padded) to the
+ * pool's entry positions int32 [rows][P] (ascending, -1 padded): block b contributes the
+ * positions 8b .. 8b+7 below n_row[r] (nullable int32 [rows]: NULL = all).
+ */
+CSA2_API csa2_status_t csa2_cp_pool_expand(int rows, const int32_t* blocks, int nb,
+                                           const int32_t* n_row, int P, int32_t* pool_out,
+                                           void* stream);
 
 /* Static text for a status code. Never NULL. */
 CSA2_API const char* csa2_status_string(csa2_status_t status);

@@ -1,0 +1,227 @@
+"""Context-parallel Full-layer selection (one shard of the entries per rank).
+
+CPU (gloo, world size 2): the decomposition itself. Each rank selects on its shard with the
+oracle, the lists travel through cp.all_gather_last, and the merge by the oracle's own
+(score desc, index asc) selection equals the oracle's selection over the whole context, for
+the Top-K and for the block pool, with planted exact ties at both boundaries.
+
+GPU (one device, shards run one after another): the cp_* kernels. The selection merged from
+G shard scans is bit-identical to the single-scan selection (indices and pool)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from fp4_compressed_sparse_quantize_b200 import cp
+from oracle import oracle as O
+
+
+def test_shards_cover_and_align():
+    for n in (0, 1, 7, 8, 9, 4095, 32768, 32773, 1 << 20):
+        for g in (1, 2, 3, 4, 7, 8):
+            sh = cp.shards(n, g)
+            assert len(sh) == g and sh[0][0] == 0 and sh[-1][1] == n
+            for (a, b), (c, d) in zip(sh, sh[1:]):
+                assert b == c
+            sizes = [b - a for a, b in sh]
+            assert all(a % 8 == 0 for a, _ in sh)
+            assert max(sizes) - min(sizes) <= 8
+
+
+def test_local_counts():
+    n_vis = torch.tensor([0, 5, 100, 260], dtype=torch.int32)
+    assert cp.local_counts(n_vis, 96, 200).tolist() == [0, 0, 4, 104]
+    assert cp.local_counts(n_vis, 0, 64).tolist() == [0, 5, 64, 64]
+
+
+def _scores(seed, n):
+    g = torch.Generator().manual_seed(seed)
+    s = torch.randn(n, generator=g, dtype=torch.float64).abs().numpy()
+    s[100:104] = s[7]                    # exact ties with a low-index entry
+    s[n // 2 + 3] = s[7]                 # ... and one in the second shard
+    s[np.argsort(-s)[60:70]] = s[np.argsort(-s)[60]]   # a tie run across the K boundary
+    return s
+
+
+def _local(s, lo, hi, K, nblk):
+    """One shard's selections as exchange lists (global ids, -1 padded)."""
+    loc = s[lo:hi]
+    ti = O.topk(loc, K)
+    v = ti >= 0
+    cand_s = np.where(v, loc[np.maximum(ti, 0)], 0.0)
+    cand_i = np.where(v, ti + lo, -1).astype(np.int32)
+    pos = O.pool(loc, nblk)
+    pos = pos[pos >= 0]
+    blocks = np.unique(pos // 8)
+    bmax = np.array([loc[b * 8:min(b * 8 + 8, hi - lo)].max() for b in blocks])
+    cb = np.zeros(nblk)
+    ci = np.full(nblk, -1, np.int32)
+    cb[:len(blocks)] = bmax
+    ci[:len(blocks)] = blocks + lo // 8
+    return cand_s, cand_i, cb, ci
+
+
+def _merge(cand_s, cand_i, K):
+    v = cand_i >= 0
+    return O.topk(cand_s[v], K, ids=cand_i[v])
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = []
+        for n, K, nblk in ((5000, 64, 32), (4093, 64, 600), (130, 64, 8)):
+            s = _scores(n, n)
+            lo, hi = cp.shards(n, world)[rank]
+            cs, ci, cb, cblk = _local(s, lo, hi, K, nblk)
+            t = [torch.from_numpy(x) for x in (cs, ci, cb, cblk)]
+            g = [cp.all_gather_last(x) for x in t]
+            idx = _merge(g[0].numpy(), g[1].numpy(), K)
+            blocks = _merge(g[2].numpy(), g[3].numpy(), nblk)
+            blocks = blocks[blocks >= 0]
+            pool = np.concatenate([np.arange(b * 8, min(b * 8 + 8, n)) for b in blocks]) \
+                if len(blocks) else np.zeros(0, np.int64)
+            ref_pool = O.pool(s, nblk)
+            res.append((np.array_equal(idx, O.topk(s, K)),
+                        np.array_equal(pool, ref_pool[ref_pool >= 0])))
+        q.put((rank, res))
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    p = sk.getsockname()[1]
+    sk.close()
+    return p
+
+
+def test_two_rank_merge_equals_whole_context():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=180) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, res in out:
+        for k, (topk_ok, pool_ok) in enumerate(res):
+            assert topk_ok, f"rank {rank} case {k}: merged Top-K differs"
+            assert pool_ok, f"rank {rank} case {k}: merged pool differs"
+
+
+def test_planted_decomposition_fails_without_shard_offsets():
+    """The check above is sensitive: dropping the shard offset of rank 1's ids breaks it."""
+    s = _scores(5000, 5000)
+    (lo0, hi0), (lo1, hi1) = cp.shards(5000, 2)
+    a = _local(s, lo0, hi0, 64, 32)
+    b = _local(s, lo1, hi1, 64, 32)
+    bad_i = np.where(b[1] >= 0, b[1] - lo1, -1).astype(np.int32)
+    good = _merge(np.concatenate([a[0], b[0]]), np.concatenate([a[1], b[1]]), 64)
+    bad = _merge(np.concatenate([a[0], b[0]]), np.concatenate([a[1], bad_i]), 64)
+    assert np.array_equal(good, O.topk(s, 64))
+    assert not np.array_equal(bad, O.topk(s, 64))
+
+
+# ---- GPU: the cp_* kernels ---------------------------------------------------------------
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("G,n_list,K,nblk", [(2, [32768, 20001, 9], 512, 2048),
+                                              (3, [40000, 32773, 4000], 512, 2048),
+                                              (4, [262144, 131075], 512, 2048)])
+def test_gpu_sharded_selection_equals_single(G, n_list, K, nblk):
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from fp4_compressed_sparse_quantize_b200 import csa2
+    dev = "cuda"
+    g = torch.Generator().manual_seed(G * 1000 + K)
+    B, H_I, cap = len(n_list), 64, max(n_list)
+    k_I = torch.randn((B, cap, 128), generator=g).to(torch.float8_e4m3fn).to(dev)
+    k_I[:, 200] = k_I[:, 100]            # exact score ties inside and across shards
+    k_I[:, cap // 2 + 5] = k_I[:, 100]
+    q_I = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn).to(dev)
+    w = torch.rand((B, 1, H_I), generator=g).to(dev)
+    n_vis = torch.tensor(n_list, dtype=torch.int32, device=dev)
+
+    ref_idx = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+    ref_pool = torch.empty((B, 1, nblk * 8), dtype=torch.int32, device=dev)
+    ws = csa2.new_workspace(csa2.workspace_bytes(0, B, 1, H_I, cap, K, nblk))
+    csa2.index_score_topk("full", q_I, w, k_I, K, ref_idx, ws, n_vis0=n_vis, pool_out=ref_pool,
+                          pool_blocks=nblk)
+
+    cs, ci, cb, cblk = [], [], [], []
+    for lo, hi in cp.shards(cap, G):
+        shard = k_I[:, lo:hi].contiguous()
+        idx = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+        pool = torch.empty((B, 1, nblk * 8), dtype=torch.int32, device=dev)
+        scores = torch.zeros((B, 1, hi - lo), dtype=torch.float32, device=dev)
+        wss = csa2.new_workspace(csa2.workspace_bytes(0, B, 1, H_I, hi - lo, K, nblk))
+        csa2.index_score_topk("full", q_I, w, shard, K, idx, wss,
+                              n_vis0=cp.local_counts(n_vis, lo, hi), pool_out=pool,
+                              pool_blocks=nblk, scores_out=scores)
+        for lst, shape, dt in ((cs, K, torch.float32), (ci, K, torch.int32),
+                               (cb, nblk, torch.float32), (cblk, nblk, torch.int32)):
+            lst.append(torch.empty((B, 1, shape), dtype=dt, device=dev))
+        csa2.cp_topk_candidates(scores, idx, lo, cs[-1], ci[-1])
+        csa2.cp_pool_candidates(scores, pool, lo, cb[-1], cblk[-1])
+        assert csa2.read_device_status(wss) == 0
+    idx = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+    csa2.cp_merge(torch.cat(cs, -1), torch.cat(ci, -1), idx)
+    blocks = torch.empty((B, 1, nblk), dtype=torch.int32, device=dev)
+    csa2.cp_merge(torch.cat(cb, -1), torch.cat(cblk, -1), blocks)
+    pool = torch.empty((B, 1, nblk * 8), dtype=torch.int32, device=dev)
+    csa2.cp_pool_expand(blocks, n_vis, pool)
+    torch.cuda.synchronize()
+    assert csa2.read_device_status(ws) == 0
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(pool, ref_pool)
+
+
+def _select_worker(port, q):
+    """cp.select over a one-rank NCCL group equals the plain Full-layer call."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        from fp4_compressed_sparse_quantize_b200 import csa2
+        dev = "cuda"
+        g = torch.Generator().manual_seed(77)
+        n_list, K, nblk, H_I = [32768, 5003], 512, 2048, 64
+        B, cap = len(n_list), max(n_list)
+        k_I = torch.randn((B, cap, 128), generator=g).to(torch.float8_e4m3fn).to(dev)
+        q_I = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn).to(dev)
+        w = torch.rand((B, 1, H_I), generator=g).to(dev)
+        n_vis = torch.tensor(n_list, dtype=torch.int32, device=dev)
+        ws = csa2.new_workspace(csa2.workspace_bytes(0, B, 1, H_I, cap, K, nblk))
+        ref_idx = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+        ref_pool = torch.empty((B, 1, nblk * 8), dtype=torch.int32, device=dev)
+        csa2.index_score_topk("full", q_I, w, k_I, K, ref_idx, ws, n_vis0=n_vis,
+                              pool_out=ref_pool, pool_blocks=nblk)
+        idx, pool = cp.select(q_I, w, k_I, n_vis, 0, K, ws, pool_blocks=nblk)
+        torch.cuda.synchronize()
+        q.put((bool(torch.equal(idx, ref_idx)), bool(torch.equal(pool, ref_pool)),
+               csa2.read_device_status(ws)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_gpu_select_one_rank_nccl():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_select_worker, args=(_free_port(), q))
+    p.start()
+    res = q.get(timeout=300)
+    p.join(timeout=60)
+    assert p.exitcode == 0
+    assert res == (True, True, 0)
