@@ -244,12 +244,13 @@ CSA2_API int csa2_sparse_attn_decode_launches(int B, int K, int W);
  * compressed entries (lo a multiple of 8), run csa2_index_score_topk(FULL) on it with
  * scores_out (and pool_out), turn the selections into candidate lists with the calls below,
  * all-gather the lists (e.g. NCCL) and merge them. The merged Top-K and pool equal the
-  * single-GPU ones exactly. [TDG Compressed Sparse Attention 2 (CSA2)]: the Full layer keeps the 512
- * highest-scoring entries and the 2,048 blocks of 8 with the highest block maxima; both
- * selections decompose over shards because the order (score descending, index ascending) is
- * total and a score depends only on its own entry. (The pages describe one GPU; sharding is
- * this library's extension for million-entry contexts.) All pointers are device pointers,
- * all calls asynchronous on `stream`; CSA2_ERR_ARG on bad sizes or null pointers.
+ * single-GPU ones exactly. [TDG Compressed Sparse Attention 2 (CSA2)]: the Full layer
+ * keeps the 512 highest-scoring entries and the 2,048 blocks of 8 with the highest block
+ * maxima; both selections decompose over shards because the order (score descending, index
+ * ascending) is total and a score depends only on its own entry. (The pages describe one
+ * GPU; sharding is this library's extension for million-entry contexts.) All pointers are
+ * device pointers, all calls asynchronous on `stream`; CSA2_ERR_ARG on bad sizes or null
+ * pointers.
  *
  * csa2_cp_topk_candidates — a shard's Top-K as (score, global index) pairs.
  *   scores     fp32 [rows][ld_scores]: the shard's scores_out.
