@@ -208,6 +208,14 @@ class Decode:
     def step_outputs(self):
         return self.out
 
+    def set_io(self, ins, outs):
+        """Point the step at another set of per-step inputs and outputs (the order of
+        step_inputs / step_outputs)."""
+        self.kv_new = ins[0]
+        for li, L in enumerate(self.layers):
+            L["q_I"], L["w"], L["q"], L["swa"] = ins[1 + 4 * li:5 + 4 * li]
+        self.out = list(outs)
+
     def algorithmic_bytes(self):
         w = self.w
         B, N, K, H, W = w.B, w.N, w.K, w.H, synth.WINDOW
@@ -559,37 +567,72 @@ def main():
     scan_ms = [a.elapsed_time(b) for a, b in sev]
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
 
-    # end-to-end: host inputs -> device -> step -> host output, through the public API
-    ins = state.step_inputs()
-    outs = state.step_outputs()
-    h_in = [x.detach().cpu().pin_memory() for x in ins]
-    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    # end-to-end: host inputs -> device -> step -> host output, through the public API.
+    # Steps are pipelined as a serving loop would run them: two sets of device inputs and
+    # outputs, so that the host->device copy of step k+1 and the device->host copy of step
+    # k-1 (copy streams) overlap step k (compute stream). Every step copies all of its
+    # inputs in and its outputs back. L2 is not flushed inside this continuous region: each
+    # step streams the 134 MB indexer-key cache (evict-first), more than the 126 MB L2.
+    ins0 = state.step_inputs()
+    outs0 = state.step_outputs()
+    h_in = [x.detach().cpu().pin_memory() for x in ins0]
+    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs0]
     bi = sum(x.numel() * x.element_size() for x in h_in)
     bo = sum(x.numel() * x.element_size() for x in h_out)
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    g_plain = None
-    if graphs:
-        g_plain = torch.cuda.CUDAGraph()
+    io = [(ins0, outs0), ([torch.empty_like(x) for x in ins0], [torch.empty_like(o) for o in outs0])]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    g_io = []
+    if not args.eager:
         side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        with torch.cuda.graph(g_plain, stream=side):
-            state.step(stream=side)
+        for ins, outs in io:
+            state.set_io(ins, outs)
+            side.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                state.step(stream=side)
+            g_io.append(g)
         torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush_l2(flush, k)
-        e2e_ev[k][0].record(stream)
-        for d, h in zip(ins, h_in):
-            d.copy_(h, non_blocking=True)
-        if g_plain:
-            g_plain.replay()
-        else:
-            state.step()
-        for h, o in zip(h_out, outs):
-            h.copy_(o, non_blocking=True)
-        e2e_ev[k][1].record(stream)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    loaded, consumed, drained = [[ev(), ev()] for _ in range(3)]
+
+    def pipelined(n):
+        for k in range(n):
+            s_ = k & 1
+            ins, outs = io[s_]
+            with torch.cuda.stream(h2d):
+                if k >= 2:
+                    h2d.wait_event(consumed[s_])      # step k-2 no longer reads set s_
+                for d, h in zip(ins, h_in):
+                    d.copy_(h, non_blocking=True)
+                loaded[s_].record(h2d)
+            stream.wait_event(loaded[s_])
+            if k >= 2:
+                stream.wait_event(drained[s_])        # step k-2's outputs are on the host
+            if g_io:
+                with torch.cuda.stream(stream):
+                    g_io[s_].replay()
+            else:
+                state.set_io(ins, outs)
+                state.step(stream=stream)
+            consumed[s_].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(consumed[s_])
+                for h, o in zip(h_out, outs):
+                    h.copy_(o, non_blocking=True)
+                drained[s_].record(d2h)
+
+    pipelined(2)                                      # warm the copy streams
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), pg, dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(h2d)
+    pipelined(args.steps)
+    d2h.wait_stream(h2d)
+    d2h.wait_stream(stream)
+    e1.record(d2h)
+    torch.cuda.synchronize()
+    state.set_io(ins0, outs0)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     st_i = csa2.read_device_status(state.ws_idx)
     st_a = csa2.read_device_status(state.ws_attn)
 
@@ -627,7 +670,9 @@ def main():
                          "traffic": traffic},
             "step_roofline_frac": (alg_bytes / (per_step_ms / 1e3) / 1e9) / peak,
             "e2e": {"value": queries / (e2e_ms / 1e3), "unit": "queries/s",
-                    "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+                    "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                    "schedule": "pipelined: step k+1's inputs in and step k-1's outputs out "
+                                "on copy streams while step k runs (two device buffer sets)"},
             "gpu_launches": state.launches_per_step() * args.steps,
             "clocks": clk,
             "device_status": [st_i, st_a],

@@ -25,7 +25,8 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_debug_bounded_wait", "csa2_set_stage_events",
            "csa2_index_score_topk_noalloc", "csa2_sparse_attn_decode_launches",
            "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
-           "csa2_cp_pool_expand")
+           "csa2_cp_pool_expand", "csa2_cache_record_bytes", "csa2_cache_export",
+           "csa2_cache_import")
 
 
 class Csa2Error(RuntimeError):
@@ -68,8 +69,13 @@ def lib():
         L.csa2_cp_pool_candidates.argtypes = [i32, P, i64, P, i32, i32, i64, P, P, P]
         L.csa2_cp_merge.argtypes = [i32, i32, P, P, i32, P, P]
         L.csa2_cp_pool_expand.argtypes = [i32, P, i32, P, i32, P, P]
+        L.csa2_cache_record_bytes.argtypes = [i64, i32]
+        L.csa2_cache_record_bytes.restype = sz
+        L.csa2_cache_export.argtypes = [P, P, P, i32, i64, i32, i64, i64, P, sz, P]
+        L.csa2_cache_import.argtypes = [P, sz, P, P, P, i64, i32, P]
         for name in EXPORTS:
-            if name not in ("csa2_workspace_bytes", "csa2_status_string"):
+            if name not in ("csa2_workspace_bytes", "csa2_status_string",
+                            "csa2_cache_record_bytes"):
                 getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -317,3 +323,41 @@ def cp_pool_expand(blocks, n_row, pool_out, stream=None):
     rows = blocks.numel() // nb
     _check(lib().csa2_cp_pool_expand(rows, _p(blocks), nb, _p(n_row), P, _p(pool_out),
                                      _stream(stream)), "csa2_cp_pool_expand")
+
+
+# ---- persistent-cache records --------------------------------------------------------------
+
+def _key_bytes(k_I):
+    return 0 if k_I is None else k_I.shape[-1] * k_I.element_size()
+
+
+def cache_record_bytes(n, key_bytes=0):
+    """Bytes of a record of n entries (key_bytes 0, 128 for E4M3 keys or 256 for bf16)."""
+    return int(lib().csa2_cache_record_bytes(int(n), int(key_bytes)))
+
+
+def cache_export(codes, scales, b, lo, n, host, k_I=None, stream=None):
+    """Entries [lo, lo + n) of sequence b (codes [B, cap, 256], scales [B, cap, 32], optional
+    k_I [B, cap, 128]) into `host`, a CPU uint8 tensor of at least cache_record_bytes bytes
+    (pinned for an asynchronous copy)."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    if host.dtype != torch.uint8 or host.is_cuda or not host.is_contiguous():
+        raise Csa2Error(ERR_ARG, "host must be a contiguous CPU uint8 tensor")
+    if k_I is not None and (not k_I.is_cuda or not k_I.is_contiguous()):
+        raise Csa2Error(ERR_ARG, "k_I must be a contiguous CUDA tensor")
+    _check(lib().csa2_cache_export(_p(codes), _p(scales), _p(k_I), _key_bytes(k_I),
+                                   codes.shape[1], int(b), int(lo), int(n), _p(host),
+                                   host.numel(), _stream(stream)), "csa2_cache_export")
+
+
+def cache_import(host, codes, scales, b, k_I=None, stream=None):
+    """A complete record in `host` back into sequence b of the caches, at its own lo."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    if host.dtype != torch.uint8 or host.is_cuda or not host.is_contiguous():
+        raise Csa2Error(ERR_ARG, "host must be a contiguous CPU uint8 tensor")
+    if k_I is not None and (not k_I.is_cuda or not k_I.is_contiguous()):
+        raise Csa2Error(ERR_ARG, "k_I must be a contiguous CUDA tensor")
+    _check(lib().csa2_cache_import(_p(host), host.numel(), _p(codes), _p(scales), _p(k_I),
+                                   codes.shape[1], int(b), _stream(stream)), "csa2_cache_import")

@@ -294,6 +294,35 @@ CSA2_API csa2_status_t csa2_cp_pool_expand(int rows, const int32_t* blocks, int 
                                            const int32_t* n_row, int P, int32_t* pool_out,
                                            void* stream);
 
+/*
+ * Persistent-cache records: one sequence's entries [lo, lo + n) copied between the device
+ * caches and a host buffer in a fixed byte format. [AIS Main Findings]: the global KV cache
+ * is held in HBM and a persistent KV cache exists besides it; [TDG The KV Cache Revolution]:
+ * the cache is accounted in bytes per token. The byte format and the copies only (no storage
+ * tier). Record: a 64-byte header (magic "CSA2", version 1, D = 512, D_I = 128, lo, n,
+ * key_bytes, bytes per entry) | codes [n][256] | scales [n][32] | indexer keys [n][key_bytes]
+ * (key_bytes 0 = none, 128 = E4M3 keys, 256 = bf16 keys). Host buffers may be pageable or
+ * pinned (pinned: the copies are asynchronous on `stream`).
+ *
+ * csa2_cache_record_bytes — bytes of a record of n entries (0 on bad arguments).
+ * csa2_cache_export — writes the header at once and enqueues one device-to-host copy per
+ *   array; the record is complete when `stream` reaches that point. codes/scales/k_I are the
+ *   caches ([B][cap][256], [B][cap][32], [B][cap][key_bytes]); k_I NULL iff key_bytes = 0.
+ *   CSA2_ERR_ARG when lo + n > cap, host_bytes is too small, or arguments are inconsistent.
+ * csa2_cache_import — validates the (complete) record's header on the host and enqueues
+ *   host-to-device copies to the header's lo of sequence b. CSA2_ERR_ARG on a bad magic,
+ *   version, size or range, or when the record's keys and k_I disagree;
+ *   CSA2_ERR_UNSUPPORTED for other channel counts.
+ */
+CSA2_API size_t csa2_cache_record_bytes(int64_t n, int key_bytes);
+CSA2_API csa2_status_t csa2_cache_export(const uint8_t* codes, const uint8_t* scales,
+                                         const void* k_I, int key_bytes, int64_t cap, int b,
+                                         int64_t lo, int64_t n, void* host, size_t host_bytes,
+                                         void* stream);
+CSA2_API csa2_status_t csa2_cache_import(const void* host, size_t host_bytes, uint8_t* codes,
+                                         uint8_t* scales, void* k_I, int64_t cap, int b,
+                                         void* stream);
+
 /* Static text for a status code. Never NULL. */
 CSA2_API const char* csa2_status_string(csa2_status_t status);
 
