@@ -1,4 +1,4 @@
-"""Context parallelism of a Full layer's selection over G GPUs.
+"""Context parallelism of a Full layer (selection and attention) over G GPUs.
 
 Each GPU (rank) holds one contiguous shard of every sequence's compressed entries (its own
 indexer-K and main-KV cache for those positions), scans it with the ordinary Full-mode
@@ -9,8 +9,14 @@ context ("DeepSeek-V4.1-Flash: A New Era in Efficient Large-Scale LLM Serving", 
 Sparse Attention 2 (CSA2): the Full layer keeps the 512 best entries and a candidate pool of
 the 2,048 best blocks of 8 positions).
 
-All selection work runs in libcsa2's kernels (csa2.cp_*); this module plans the shards and
-moves the lists with torch.distributed (NCCL between GPUs, gloo on the host).
+The attention follows the same split: each rank attends over the selected entries it holds
+(and one rank over the window rows), leaves a partial result (maximum, sum, unnormalised
+output), the ranks all-gather the partials and every rank merges them by the exact
+log-sum-exp identity.
+
+All selection and attention work runs in libcsa2's kernels (csa2.cp_*, csa2.*_partial*); this
+module plans the shards and moves the lists with torch.distributed (NCCL between GPUs, gloo
+on the host).
 """
 import torch
 import torch.distributed as dist
@@ -79,3 +85,28 @@ def select(q_I, w, k_I_shard, n_vis, lo, K, ws, pool_blocks=0, group=None):
     pool_out = torch.empty_like(pool)
     csa2.cp_pool_expand(blocks, n_vis.to(i32).contiguous(), pool_out)
     return out, pool_out
+
+
+def all_gather_stack(t, group=None):
+    """Every rank's t stacked along a new leading dimension, in rank order."""
+    parts = [torch.empty_like(t) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, t.contiguous(), group=group)
+    return torch.stack(parts).contiguous()
+
+
+def attend(mode, q, codes_shard, scales_shard, idx, lo, swa, out, ws, swa_valid=None,
+           scale=None, group=None):
+    """Decode attention over the merged selection `idx` int32 [B, K] (global indices), with
+    this rank holding main-KV entries [lo, lo + cap_shard) in codes_shard / scales_shard.
+    Pass swa (and swa_valid) on exactly one rank, None elsewhere. Writes out fp32
+    [B, H, 512] on every rank."""
+    B, H, _ = q.shape
+    cap = codes_shard.shape[1]
+    dev = q.device
+    local = torch.empty_like(idx)
+    csa2.cp_local_idx(idx, lo, lo + cap, local)
+    o = torch.empty((B, H, csa2.D_MAIN), dtype=torch.float32, device=dev)
+    ml = torch.empty((B, 2, H), dtype=torch.float32, device=dev)
+    csa2.sparse_attn_decode_partial(mode, q, codes_shard, scales_shard, local, swa, o, ml, ws,
+                                    scale=scale, swa_valid=swa_valid)
+    csa2.attn_merge_partials(all_gather_stack(o, group), all_gather_stack(ml, group), out)

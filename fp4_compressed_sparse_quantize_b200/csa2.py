@@ -26,7 +26,8 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_index_score_topk_noalloc", "csa2_sparse_attn_decode_launches",
            "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
            "csa2_cp_pool_expand", "csa2_cache_record_bytes", "csa2_cache_export",
-           "csa2_cache_import")
+           "csa2_cache_import", "csa2_cp_local_idx", "csa2_sparse_attn_decode_partial",
+           "csa2_attn_merge_partials")
 
 
 class Csa2Error(RuntimeError):
@@ -69,6 +70,10 @@ def lib():
         L.csa2_cp_pool_candidates.argtypes = [i32, P, i64, P, i32, i32, i64, P, P, P]
         L.csa2_cp_merge.argtypes = [i32, i32, P, P, i32, P, P]
         L.csa2_cp_pool_expand.argtypes = [i32, P, i32, P, i32, P, P]
+        L.csa2_cp_local_idx.argtypes = [i64, P, i64, i64, P, P]
+        L.csa2_sparse_attn_decode_partial.argtypes = [i32, i32, i32, P, P, P, i64, P, i32, P,
+                                                      i32, P, f32, P, P, P, sz, P]
+        L.csa2_attn_merge_partials.argtypes = [i32, i32, i32, P, P, P, P]
         L.csa2_cache_record_bytes.argtypes = [i64, i32]
         L.csa2_cache_record_bytes.restype = sz
         L.csa2_cache_export.argtypes = [P, P, P, i32, i64, i32, i64, i64, P, sz, P]
@@ -250,6 +255,40 @@ def sparse_attn_decode(mode, q, codes, scales, idx, swa, out, ws, scale=None, sw
     _check(st, "csa2_sparse_attn_decode")
 
 
+def sparse_attn_decode_partial(mode, q, codes, scales, idx, swa, o_part, ml_part, ws, scale=None,
+                               swa_valid=None, stream=None):
+    """sparse_attn_decode over the caller's rows, left as a partial: o_part fp32 [B, H, 512],
+    ml_part fp32 [B, 2, H] (base-2 maximum and sum). swa may be None (no window rows)."""
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    _need(q, torch.bfloat16, "q")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    _need(idx, torch.int32, "idx")
+    _need(swa, torch.float8_e4m3fn, "swa")
+    _need(o_part, torch.float32, "o_part")
+    _need(ml_part, torch.float32, "ml_part")
+    _need(swa_valid, torch.int32, "swa_valid")
+    B, H, D = q.shape
+    K = idx.shape[-1] if idx is not None else 0
+    W = swa.shape[1] if swa is not None else 0
+    sc = float(scale) if scale is not None else D_MAIN ** -0.5
+    st = lib().csa2_sparse_attn_decode_partial(m, B, H, _p(q), _p(codes), _p(scales),
+                                               codes.shape[1], _p(idx), K, _p(swa), W,
+                                               _p(swa_valid), sc, _p(o_part), _p(ml_part),
+                                               _p(ws), ws.numel(), _stream(stream))
+    _check(st, "csa2_sparse_attn_decode_partial")
+
+
+def attn_merge_partials(o_parts, ml_parts, out, stream=None):
+    """o_parts fp32 [G, B, H, 512], ml_parts fp32 [G, B, 2, H] -> out fp32 [B, H, 512]."""
+    _need(o_parts, torch.float32, "o_parts")
+    _need(ml_parts, torch.float32, "ml_parts")
+    _need(out, torch.float32, "out")
+    G, B, H, _ = o_parts.shape
+    _check(lib().csa2_attn_merge_partials(B, H, G, _p(o_parts), _p(ml_parts), _p(out),
+                                          _stream(stream)), "csa2_attn_merge_partials")
+
+
 def sparse_attn_prefill(q, codes, scales, idx, swa, out, ws, W, q_pos0=None, scale=None,
                         stream=None):
     """q bf16 [B, T, H, 512]; idx int32 [B, T, K]; swa E4M3 [B, W-1+T, 512];
@@ -361,3 +400,11 @@ def cache_import(host, codes, scales, b, k_I=None, stream=None):
         raise Csa2Error(ERR_ARG, "k_I must be a contiguous CUDA tensor")
     _check(lib().csa2_cache_import(_p(host), host.numel(), _p(codes), _p(scales), _p(k_I),
                                    codes.shape[1], int(b), _stream(stream)), "csa2_cache_import")
+
+
+def cp_local_idx(idx, lo, hi, idx_local, stream=None):
+    """Global selected indices -> indices local to the shard [lo, hi), -1 elsewhere."""
+    _need(idx, torch.int32, "idx")
+    _need(idx_local, torch.int32, "idx_local")
+    _check(lib().csa2_cp_local_idx(idx.numel(), _p(idx), int(lo), int(hi), _p(idx_local),
+                                   _stream(stream)), "csa2_cp_local_idx")

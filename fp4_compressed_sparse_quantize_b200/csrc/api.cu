@@ -88,14 +88,14 @@ static TopkPlan plan_topk(int B, int T, int H_I, int esz, int64_t row_len, int K
     return p;
 }
 
-// Attention workspace: status word, split partials (decode with nsplit > 1), and for decode
-// the staging area of the dequantised rows (`rows` = K + W per query).
-static size_t attn_partial_bytes(int Q, int H, int nsplit) {
-    return nsplit > 1 ? align_up(sizeof(float) * (size_t)Q * nsplit * H * (CSA2_D_MAIN + 2), 256)
-                      : 0;
+// Attention workspace: status word, split partials, and for decode the staging area of the
+// dequantised rows (`rows` = K + W per query). Partials (np splits; 0 = none) are needed when
+// a decode query's rows are split or the call leaves a partial result.
+static size_t attn_partial_bytes(int Q, int H, int np) {
+    return np > 0 ? align_up(sizeof(float) * (size_t)Q * np * H * (CSA2_D_MAIN + 2), 256) : 0;
 }
-static size_t attn_ws_bytes(int Q, int H, int nsplit, int stage_rows) {
-    size_t b = kStatusBytes + attn_partial_bytes(Q, H, nsplit);
+static size_t attn_ws_bytes(int Q, int H, int np, int stage_rows) {
+    size_t b = kStatusBytes + attn_partial_bytes(Q, H, np);
     if (stage_rows > 0) b += attention_stage_bytes(Q, stage_rows);
     return b;
 }
@@ -212,7 +212,7 @@ size_t csa2_workspace_bytes(csa2_op_t op, int B, int T, int H, int64_t cap, int 
             // sized for windows of up to 1024 rows
             return attn_ws_bytes(B, H, attn_split_bound(B, K), K + 1024);
         case CSA2_OP_SPARSE_ATTN_PREFILL:
-            return attn_ws_bytes(B * T, H, 1, 0);
+            return attn_ws_bytes(B * T, H, 0, 0);
     }
     return 0;
 }
@@ -378,10 +378,16 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
                                  const uint8_t* codes, const uint8_t* scales, int64_t cap,
                                  const int32_t* idx, int K, const uint8_t* swa, int W,
                                  const int32_t* swa_valid, const int32_t* q_pos0, float scale,
-                                 float* out, void* ws, size_t ws_bytes, void* stream) {
+                                 float* out, void* ws, size_t ws_bytes, void* stream,
+                                 float* o_part = nullptr, float* ml_part = nullptr) {
     if (B < 1 || T < 1 || cap < 1 || K < 0 || W < 0) return CSA2_ERR_ARG;
     if (H < 1) return CSA2_ERR_ARG;
     if (H > 64 || W > 1024 || K > 65536) return CSA2_ERR_UNSUPPORTED;
+    const bool part = o_part != nullptr;
+    if (part) {
+        if (!ml_part || !aligned16(o_part) || prefill || K + W < 1) return CSA2_ERR_ARG;
+        out = o_part;   // only checked for alignment below; the result goes to o_part/ml_part
+    }
     if (!q || !out || !ws) return !ws ? CSA2_ERR_WORKSPACE : CSA2_ERR_ARG;
     if (K > 0 && (!codes || !scales || !idx)) return CSA2_ERR_ARG;
     if (W > 0 && !swa) return CSA2_ERR_ARG;
@@ -393,7 +399,8 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
     if (Q > 2147483647) return CSA2_ERR_UNSUPPORTED;
     const int nsplit = attention_splits((int)Q, K, W, prefill);
     const int stage_rows = prefill ? 0 : K + W;
-    if (ws_bytes < attn_ws_bytes((int)Q, H, nsplit, stage_rows)) return CSA2_ERR_WORKSPACE;
+    const int np = (nsplit > 1 || part) ? nsplit : 0;   // partial splits in the workspace
+    if (ws_bytes < attn_ws_bytes((int)Q, H, np, stage_rows)) return CSA2_ERR_WORKSPACE;
     AttnLaunch l;
     memset(&l, 0, sizeof l);
     l.Q = (int)Q;
@@ -411,11 +418,13 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
     l.q_pos0 = q_pos0;
     l.prefill = prefill;
     l.scale = scale;
-    l.out = out;
+    l.out = part ? nullptr : out;
+    l.o_part = part ? o_part : nullptr;
+    l.ml_part = part ? ml_part : nullptr;
     l.nsplit = nsplit;
     l.partial = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kStatusBytes);
     l.stage = stage_rows > 0 ? reinterpret_cast<uint8_t*>(ws) + kStatusBytes +
-                                   attn_partial_bytes((int)Q, H, nsplit)
+                                   attn_partial_bytes((int)Q, H, np)
                              : nullptr;
     l.status = reinterpret_cast<int32_t*>(ws);
     return cuda_status(launch_attention(l, reinterpret_cast<cudaStream_t>(stream)));
@@ -441,6 +450,39 @@ csa2_status_t csa2_sparse_attn_prefill(int B, int T, int H, const void* q,
                                        void* stream) {
     return attn_common(true, B, T, H, q, codes, scales, cap, idx, K, swa, W, nullptr, q_pos0,
                        scale, out, ws, ws_bytes, stream);
+}
+
+csa2_status_t csa2_sparse_attn_decode_partial(csa2_mode_t mode, int B, int H, const void* q,
+                                              const uint8_t* codes, const uint8_t* scales,
+                                              int64_t cap, const int32_t* idx, int K,
+                                              const uint8_t* swa, int W,
+                                              const int32_t* swa_valid, float scale,
+                                              float* o_part, float* ml_part, void* ws,
+                                              size_t ws_bytes, void* stream) {
+    if (mode != CSA2_MODE_FULL && mode != CSA2_MODE_REINDEX && mode != CSA2_MODE_REUSE)
+        return CSA2_ERR_ARG;
+    if (!o_part || !ml_part) return CSA2_ERR_ARG;
+    return attn_common(false, B, 1, H, q, codes, scales, cap, idx, K, swa, W, swa_valid,
+                       nullptr, scale, nullptr, ws, ws_bytes, stream, o_part, ml_part);
+}
+
+csa2_status_t csa2_attn_merge_partials(int B, int H, int G, const float* o_parts,
+                                       const float* ml_parts, float* out, void* stream) {
+    if (B < 1 || H < 1 || H > 64 || G < 1 || !o_parts || !ml_parts || !out) return CSA2_ERR_ARG;
+    if (!aligned16(o_parts) || !aligned16(out)) return CSA2_ERR_ARG;
+    CombineArgs c;
+    c.o = o_parts;
+    c.ml = ml_parts;
+    c.o_q = (int64_t)H * CSA2_D_MAIN;
+    c.o_s = (int64_t)B * c.o_q;
+    c.ml_q = 2 * (int64_t)H;
+    c.ml_s = (int64_t)B * c.ml_q;
+    c.nsplit = G;
+    c.H = H;
+    c.out = out;
+    c.o_part = nullptr;
+    c.ml_part = nullptr;
+    return cuda_status(launch_combine(c, B, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

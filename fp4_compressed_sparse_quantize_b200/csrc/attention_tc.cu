@@ -69,6 +69,7 @@ struct TcAttnDev {
     float* partial;          // O [Q * nsplit][H][512]
     float* partial_ml;       // (m, l) [Q * nsplit][2][H]
     int nsplit, nchunks, chunks_per_split;
+    bool part;               // decode: write (m, l, unnormalised O) partials even for one split
     int32_t* status;
     // staged decode: rows / query already dequantised by attn_stage_kernel
     const int32_t* st_valid;   // [Q][K + W] row kinds (0 = empty)
@@ -869,7 +870,7 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     const int oblk = a.nsplit == 1 ? qrow : qrow * a.nsplit + split;
     const uint32_t tq = (uint32_t)(32 * quad) << 16;
     const int cbase = 256 * wh;                // channels of this warp
-    const float oscale = a.nsplit == 1 ? inv_s[h] : 1.f;
+    const float oscale = (a.nsplit == 1 && !a.part) ? inv_s[h] : 1.f;
     if (ok) {
 #pragma unroll 1
         for (int cc = 0; cc < 256; cc += 64) {
@@ -1009,7 +1010,7 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
         }
         cluster_sync_all();   // the other splits have finished reading this CTA's tiles
     } else {
-        if (ok && a.nsplit > 1 && warp == 0) {
+        if (ok && (a.nsplit > 1 || a.part) && warp == 0) {
             float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
             for (int x = lane; x < a.H; x += 32) {
                 ml[x] = m_s[x];
@@ -1154,7 +1155,9 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merg
     a.scale = l.scale;
     a.out = l.out;
     a.partial = l.partial;
-    a.partial_ml = l.nsplit > 1 ? l.partial + (int64_t)l.Q * l.nsplit * l.H * kD : nullptr;
+    a.part = l.o_part != nullptr;
+    a.partial_ml = (l.nsplit > 1 || a.part) ? l.partial + (int64_t)l.Q * l.nsplit * l.H * kD
+                                            : nullptr;
     a.nsplit = l.nsplit;
     a.nchunks = (l.K + l.W + kRows - 1) / kRows;
     if (a.nchunks < 1) a.nchunks = 1;
@@ -1195,7 +1198,7 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merg
         const int dsmem = DecSmem(rps).bytes() + 1024;
         CUtensorMap mos;
         memset(&mos, 0, sizeof mos);
-        if (l.nsplit > 1 && cluster_merge_fits(l.Q, l.nsplit, dsmem)) {
+        if (l.nsplit > 1 && !a.part && cluster_merge_fits(l.Q, l.nsplit, dsmem)) {
             // the splits of a query form one cluster and write the final output themselves
             if (!out_map_sw(&mos, l.out, l.H, l.Q)) return cudaErrorInvalidValue;
             e = cudaFuncSetAttribute(attn_decode_kernel<true>,
@@ -1220,8 +1223,8 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merg
             if (e == cudaSuccess) *merged = true;
             return e;
         }
-        if (l.nsplit > 1 ? !out_map_sw(&mos, l.partial, l.H, (int64_t)l.Q * l.nsplit)
-                         : !out_map_sw(&mos, l.out, l.H, l.Q))
+        if ((l.nsplit > 1 || a.part) ? !out_map_sw(&mos, l.partial, l.H, (int64_t)l.Q * l.nsplit)
+                                     : !out_map_sw(&mos, l.out, l.H, l.Q))
             return cudaErrorInvalidValue;
         e = cudaFuncSetAttribute(attn_decode_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, dsmem);

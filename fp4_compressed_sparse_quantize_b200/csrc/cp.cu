@@ -202,6 +202,20 @@ __global__ void __launch_bounds__(kCpThreads) cp_pool_expand_kernel(
     for (int i = base + (int)threadIdx.x; i < P; i += kCpThreads) pool_out[r * P + i] = -1;
 }
 
+// Global selected indices -> this shard's local indices (-1 outside [lo, hi)), for the
+// shard's partial attention over the rows it holds.
+__global__ void __launch_bounds__(256) cp_local_idx_kernel(const int32_t* __restrict__ idx,
+                                                           int64_t n, int64_t lo, int64_t hi,
+                                                           int32_t* __restrict__ out) {
+    grid_dep_launch();
+    grid_dep_wait();
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t v = idx[i];
+        out[i] = (v >= lo && v < hi) ? (int32_t)(v - lo) : -1;
+    }
+}
+
 static int pow2_at_least(int n) {
     int p = 1;
     while (p < n) p <<= 1;
@@ -266,6 +280,18 @@ CSA2_API csa2_status_t csa2_cp_pool_expand(int rows, const int32_t* blocks, int 
     const cudaError_t e = launch_pdl(cp_pool_expand_kernel, dim3((unsigned)rows),
                                      dim3(kCpThreads), 0, reinterpret_cast<cudaStream_t>(stream),
                                      blocks, nb, n_row, P, pool_out);
+    return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+CSA2_API csa2_status_t csa2_cp_local_idx(int64_t n, const int32_t* idx, int64_t lo, int64_t hi,
+                                         int32_t* idx_local, void* stream) {
+    if (n < 0 || lo < 0 || hi < lo || !idx || !idx_local) return CSA2_ERR_ARG;
+    if (n == 0) return CSA2_OK;
+    const int64_t blocks = (n + 255) / 256;
+    const cudaError_t e = launch_pdl(cp_local_idx_kernel,
+                                     dim3((unsigned)(blocks < 4096 ? blocks : 4096)), dim3(256), 0,
+                                     reinterpret_cast<cudaStream_t>(stream), idx, n, lo, hi,
+                                     idx_local);
     return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
 }
 

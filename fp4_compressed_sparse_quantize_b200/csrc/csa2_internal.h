@@ -113,12 +113,26 @@ struct AttnLaunch {
     float scale;
     float* out;              // [Q][H][512]
     float* partial;          // workspace for split rows
+    float* o_part;           // non-null: leave the result as a partial (unnormalised O [Q][H][512]
+    float* ml_part;          //   and (M, L) [Q][2][H], base-2 logits) instead of writing out
     int nsplit;
     void* stage;             // decode staging area (attention_stage_bytes), or null
     int32_t* status;
 };
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st);
+// Merge of partial attention results: split s of row q at o + s*o_s + q*o_q ([H][512]) and
+// (m, l) at ml + s*ml_s + q*ml_q ([2][H]); into out [Q][H][512], or (o_part, ml_part) when set.
+struct CombineArgs {
+    const float* o;
+    const float* ml;
+    int64_t o_s, o_q, ml_s, ml_q;
+    int nsplit, H;
+    float* out;
+    float* o_part;
+    float* ml_part;
+};
+cudaError_t launch_combine(const CombineArgs& a, int Q, cudaStream_t st);
 size_t attention_stage_bytes(int Q, int rows);
 // Decode splits the K + W rows of a query into equal runs of at most kAttnDecodeRows rows
 // (a multiple of 32), as many as fill one wave of CTAs; prefill never splits.

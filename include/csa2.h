@@ -295,6 +295,38 @@ CSA2_API csa2_status_t csa2_cp_pool_expand(int rows, const int32_t* blocks, int 
                                            void* stream);
 
 /*
+ * csa2_cp_local_idx — this shard's view of the merged selection: idx_local[i] = idx[i] - lo
+ * for lo <= idx[i] < hi, else -1 (n elements, any row layout).
+ */
+CSA2_API csa2_status_t csa2_cp_local_idx(int64_t n, const int32_t* idx, int64_t lo, int64_t hi,
+                                         int32_t* idx_local, void* stream);
+
+/*
+ * csa2_sparse_attn_decode_partial — csa2_sparse_attn_decode over the rows this caller holds
+ * (its shard's selected entries, and the window rows on one shard only), left as a partial
+ * result for csa2_attn_merge_partials: o_part fp32 [B][H][512] = sum_i 2^(l_i - m) x_i and
+ * ml_part fp32 [B][2][H] = (m, sum_i 2^(l_i - m)), with l_i the logits in base-2 units
+ * (scale * log2(e) * <q_h, x_i>); a head with no rows gives (-inf, 0) and a zero o_part.
+ * Same arguments and checks as csa2_sparse_attn_decode, K + W >= 1, the same workspace.
+ * [TDG Compressed Sparse Attention 2 (CSA2)]: one softmax over the selected entries and the
+ * window rows; splitting the rows and merging partials is the exact log-sum-exp identity.
+ *
+ * csa2_attn_merge_partials — out fp32 [B][H][512] = sum_g 2^(m_g - M) o_g / sum_g 2^(m_g - M)
+ * l_g over G partials laid out rank-major (o_parts [G][B][H][512], ml_parts [G][B][2][H], as
+ * an all-gather along a new leading dimension leaves them). H <= 64.
+ */
+CSA2_API csa2_status_t csa2_sparse_attn_decode_partial(csa2_mode_t mode, int B, int H,
+                                                       const void* q, const uint8_t* codes,
+                                                       const uint8_t* scales, int64_t cap,
+                                                       const int32_t* idx, int K,
+                                                       const uint8_t* swa, int W,
+                                                       const int32_t* swa_valid, float scale,
+                                                       float* o_part, float* ml_part, void* ws,
+                                                       size_t ws_bytes, void* stream);
+CSA2_API csa2_status_t csa2_attn_merge_partials(int B, int H, int G, const float* o_parts,
+                                                const float* ml_parts, float* out, void* stream);
+
+/*
  * Persistent-cache records: one sequence's entries [lo, lo + n) copied between the device
  * caches and a host buffer in a fixed byte format. [AIS Main Findings]: the global KV cache
  * is held in HBM and a persistent KV cache exists besides it; [TDG The KV Cache Revolution]:

@@ -225,3 +225,105 @@ def test_gpu_select_one_rank_nccl():
     p.join(timeout=60)
     assert p.exitcode == 0
     assert res == (True, True, 0)
+
+
+# ---- attention over shards: partial results merged by the log-sum-exp identity -------------
+
+def _partial(q, rows, tau):
+    """(m, l, o) of one rank's rows, natural-log units, fp64 (a plain restatement)."""
+    H = q.shape[0]
+    if rows.shape[0] == 0:
+        return np.full(H, -np.inf), np.zeros(H), np.zeros((H, q.shape[1]))
+    lg = tau * (q @ rows.T)
+    m = lg.max(axis=1)
+    p = np.exp(lg - m[:, None])
+    return m, p.sum(axis=1), p @ rows
+
+
+def _attn_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(11)
+        n, K, W, H, tau = 3000, 512, 128, 8, 1 / np.sqrt(512)
+        main = rng.standard_normal((n, 512)) * np.exp(rng.standard_normal(512))
+        swa = rng.standard_normal((W, 512))
+        qh = rng.standard_normal((H, 512))
+        idx = np.sort(rng.choice(n, K, replace=False))
+        lo, hi = cp.shards(n, world)[rank]
+        mine = idx[(idx >= lo) & (idx < hi)]
+        rows = main[mine]
+        if rank == 0:
+            rows = np.concatenate([rows, swa])
+        m, l, o = _partial(qh, rows, tau)
+        gm, gl, go = (cp.all_gather_stack(torch.from_numpy(x)).numpy() for x in (m, l, o))
+        M = gm.max(axis=0)
+        wgt = np.exp(gm - M)
+        out = (wgt[:, :, None] * go).sum(axis=0) / (wgt * gl).sum(axis=0)[:, None]
+        ref = O.attention(qh, np.concatenate([main[idx], swa]), tau)
+        q.put((rank, float(np.max(np.abs(out - ref)) / np.sqrt(np.mean(ref * ref)))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_attention_partials_merge_to_whole():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_attn_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=180) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, rel in out:
+        assert rel < 1e-12, f"rank {rank}: merged partials differ from the whole ({rel:.3g})"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("G,B,H,n,K,W", [(2, 3, 64, 20000, 512, 128), (3, 2, 40, 4001, 512, 37),
+                                          (4, 32, 64, 32768, 512, 128)])
+def test_gpu_sharded_attention_matches_oracle(G, B, H, n, K, W):
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import math
+    from fp4_compressed_sparse_quantize_b200 import csa2
+    from tests.helpers import bits16, bits8, check_attention, oracle_main_rows
+    dev = "cuda"
+    g = torch.Generator().manual_seed(G * 7 + n)
+    kv = (torch.randn((B, n, 512), generator=g) *
+          torch.exp(torch.randn((B, 1, 512), generator=g))).to(torch.bfloat16)
+    codes = torch.zeros((B, n, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, n, 32), dtype=torch.uint8, device=dev)
+    csa2.quantize_kv(kv.to(dev), torch.zeros(B, dtype=torch.int32, device=dev), codes, scales)
+    rng = np.random.default_rng(n)
+    idx = np.stack([np.sort(rng.choice(n, K, replace=False)) for _ in range(B)]).astype(np.int32)
+    # query 0 selects only entries of the first shard: the other shards hold no row of it
+    idx[0] = np.sort(rng.choice(n // G, K, replace=False))
+    q = torch.randn((B, H, 512), generator=g).to(torch.bfloat16)
+    swa = torch.randn((B, W, 512), generator=g).to(torch.float8_e4m3fn)
+    tau = 1 / math.sqrt(512)
+    tI = torch.from_numpy(idx).to(dev)
+    o_parts, ml_parts = [], []
+    for r, (lo, hi) in enumerate(cp.shards(n, G)):
+        cs, ss = codes[:, lo:hi].contiguous(), scales[:, lo:hi].contiguous()
+        local = torch.empty_like(tI)
+        csa2.cp_local_idx(tI, lo, hi, local)
+        o = torch.empty((B, H, 512), dtype=torch.float32, device=dev)
+        ml = torch.empty((B, 2, H), dtype=torch.float32, device=dev)
+        ws = csa2.new_workspace(csa2.workspace_bytes(1, B, 1, H, hi - lo, K))
+        csa2.sparse_attn_decode_partial("full", q.to(dev), cs, ss, local,
+                                        swa.to(dev) if r == 0 else None, o, ml, ws, scale=tau)
+        assert csa2.read_device_status(ws) == 0
+        o_parts.append(o)
+        ml_parts.append(ml)
+    out = torch.empty((B, H, 512), dtype=torch.float32, device=dev)
+    csa2.attn_merge_partials(torch.stack(o_parts), torch.stack(ml_parts), out)
+    torch.cuda.synchronize()
+    for b in range(min(B, 4)):
+        sel = [i for i in idx[b] if i >= 0]
+        rows = np.concatenate([oracle_main_rows(bits16(kv[b, sel])),
+                               O.e4m3_array_to_f64(bits8(swa[b])).reshape(W, 512)])
+        ref = O.attention(O.bf16_array_to_f64(bits16(q[b])).reshape(H, 512), rows, tau)
+        check_attention(out[b].cpu().numpy(), ref, f"G={G} b={b}")
