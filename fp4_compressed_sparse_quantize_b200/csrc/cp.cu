@@ -21,7 +21,7 @@
 namespace csa2 {
 
 constexpr int kCpThreads = 1024;
-constexpr int kCpMaxCand = 8192;   // candidates per row the merge accepts
+constexpr int kCpMaxCand = 16384;  // candidates per row the merge accepts (8 x 2,048 pool blocks)
 
 // exclusive prefix sum of v over the CTA (blockDim.x == kCpThreads); *total gets the sum
 __device__ __forceinline__ int cp_excl_scan(int v, int* warp_sums, int* total) {

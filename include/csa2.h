@@ -277,9 +277,9 @@ CSA2_API csa2_status_t csa2_cp_pool_candidates(int rows, const float* scores, in
 /*
  * csa2_cp_merge — the K best of every row's n_cand candidates by (score descending, index
  * ascending), written to idx_out int32 [rows][K] in ascending index order, -1 padded.
- * Candidates with index -1 are ignored; indices must be distinct. n_cand <= 8192
- * (CSA2_ERR_UNSUPPORTED above), K <= n_cand. Used for entries (scores) and for pool blocks
- * (block maxima) alike.
+ * Candidates with index -1 are ignored; indices must be distinct. n_cand <= 16384
+ * (CSA2_ERR_UNSUPPORTED above: 8 shards of 2,048 pool blocks, or 32 shards of K = 512),
+ * K <= n_cand. Used for entries (scores) and for pool blocks (block maxima) alike.
  */
 CSA2_API csa2_status_t csa2_cp_merge(int rows, int n_cand, const float* cand_score,
                                      const int32_t* cand_idx, int K, int32_t* idx_out,

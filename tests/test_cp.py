@@ -132,12 +132,30 @@ def test_planted_decomposition_fails_without_shard_offsets():
     assert not np.array_equal(bad, O.topk(s, 64))
 
 
+def test_cp_calls_reject_bad_arguments():
+    """Argument checks that run before any launch (no GPU needed)."""
+    import ctypes as C
+    from fp4_compressed_sparse_quantize_b200 import csa2
+    L, f = csa2.lib(), C.c_void_p(256)
+    assert L.csa2_cp_merge(1, 16385, f, f, 512, f, None) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_cp_merge(1, 100, f, f, 101, f, None) == csa2.ERR_ARG
+    assert L.csa2_cp_merge(1, 100, None, f, 10, f, None) == csa2.ERR_ARG
+    assert L.csa2_cp_pool_candidates(1, f, 64, f, 64, 8, 12, f, f, None) == csa2.ERR_ARG
+    assert L.csa2_cp_topk_candidates(1, f, 64, f, 8, -1, f, f, None) == csa2.ERR_ARG
+    assert L.csa2_cp_topk_candidates(1, f, 1 << 30, f, 8, 1 << 30, f, f, None) == csa2.ERR_UNSUPPORTED
+    assert L.csa2_cp_local_idx(10, f, 5, 4, f, None) == csa2.ERR_ARG
+    assert L.csa2_attn_merge_partials(1, 65, 2, f, f, f, None) == csa2.ERR_ARG
+    with pytest.raises(csa2.Csa2Error):
+        cp.select(torch.zeros((1, 2, 1, 128)), None, None, None, 0, 1, None)
+
+
 # ---- GPU: the cp_* kernels ---------------------------------------------------------------
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("G,n_list,K,nblk", [(2, [32768, 20001, 9], 512, 2048),
                                               (3, [40000, 32773, 4000], 512, 2048),
-                                              (4, [262144, 131075], 512, 2048)])
+                                              (4, [262144, 131075], 512, 2048),
+                                              (8, [262144, 100003], 512, 2048)])
 def test_gpu_sharded_selection_equals_single(G, n_list, K, nblk):
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
