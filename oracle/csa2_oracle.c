@@ -27,7 +27,10 @@
  *  - Top-K / pool: against Python's sorted() on tiny inputs with planted ties and
  *    against the Top-K-inside-pool invariant;
  *  - attention: K = all entries against torch's scaled_dot_product_attention in fp64,
- *    one-key and q = 0 closed forms.
+ *    one-key and q = 0 closed forms;
+ *  - prefill visibility and window rows: a token-by-token simulation of the compressor
+ *    and of the window buffer, for ratios 1-3 and windows clipped at position 0; the
+ *    composed prefill query with every visible entry selected against dense attention.
  *  The index-score FORMULA itself (sum over heads of w_h * ReLU(q_h . k)) is not
  *  printed on the pages: parity with the pages' own scorer is unpinned; the reading is
  *  stated where it is used.
@@ -352,6 +355,42 @@ ORC_EXPORT void orc_attention(int H, int D, const double* q, const double* rows,
         }
         free(logit);
     }
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Prefill visibility and the causal window                                        */
+/* [TDG Causal Encoder-Decoder]: every layer attends over a 128-token sliding       */
+/* window; [TDG CSA2] and [AIS Methodology]: the Full layer scores the causally     */
+/* visible compressed entries; [TDG CSA2]: the encoder compresses at ratio 2, the   */
+/* decoder at ratio 1. Reading (the pages do not spell the rule out): a compressed  */
+/* entry at ratio r summarises r consecutive tokens, entry j covering positions     */
+/* r*j .. r*j + r - 1, and a token at position p may read entry j only once every   */
+/* token the entry covers is at or before p. The window of the token at position p  */
+/* is the positions p-W+1 .. p that exist (>= 0).                                  */
+/* ------------------------------------------------------------------------------ */
+
+/* Number of compressed entries visible to the token at position p (they are the
+ * prefix 0 .. n-1): count the entries whose last covered position is <= p. */
+ORC_EXPORT int64_t orc_prefill_visible(int64_t p, int ratio) {
+    int64_t n = 0;
+    while ((int64_t)ratio * n + ratio - 1 <= p) ++n;
+    return n;
+}
+
+/* Window rows of query token t of a prefill chunk whose first token sits at position
+ * q_pos0. The chunk's window buffer holds W-1+T rows, row i holding position
+ * q_pos0 - (W-1) + i (the W-1 positions before the chunk, then the chunk's own). Writes
+ * the buffer rows of the positions p-W+1 .. p (p = q_pos0 + t) that are >= 0, ascending,
+ * and returns their number. */
+ORC_EXPORT int orc_prefill_window_rows(int64_t q_pos0, int W, int64_t t, int32_t* rows_out) {
+    const int64_t p = q_pos0 + t;
+    const int64_t first_buffer_pos = q_pos0 - (W - 1);
+    int n = 0;
+    for (int64_t pos = p - W + 1; pos <= p; ++pos) {
+        if (pos < 0) continue;
+        rows_out[n++] = (int32_t)(pos - first_buffer_pos);
+    }
+    return n;
 }
 
 /* ------------------------------------------------------------------------------ */

@@ -62,6 +62,10 @@ def lib():
         L.orc_main_entry_bytes.argtypes = [C.c_int]
         L.orc_kv_bytes_per_token.restype = d
         L.orc_kv_bytes_per_token.argtypes = [C.c_int, d, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.orc_prefill_visible.restype = i64
+        L.orc_prefill_visible.argtypes = [i64, C.c_int]
+        L.orc_prefill_window_rows.restype = C.c_int
+        L.orc_prefill_window_rows.argtypes = [i64, C.c_int, i64, P]
         _lib = L
     return _lib
 
@@ -224,6 +228,46 @@ def attention_decode_query(q_bits, codes, scales, idx, swa_codes, tau, swa_valid
     swa = e4m3_array_to_f64(swa_codes[W - v:]).reshape(-1, D)
     rows = np.concatenate([sel, swa], axis=0)
     return attention(q, rows, tau)
+
+
+# ---- prefill: causal visibility, window rows, one whole query ------------------------------
+
+def prefill_visible(p, ratio):
+    """Compressed entries visible to the token at position p (the prefix 0 .. n-1)."""
+    return int(lib().orc_prefill_visible(int(p), int(ratio)))
+
+
+def prefill_window_rows(q_pos0, W, t):
+    """Rows of a prefill chunk's [W-1+T] window buffer that token t attends to (ascending)."""
+    out = np.zeros(max(int(W), 1), np.int32)
+    n = lib().orc_prefill_window_rows(int(q_pos0), int(W), int(t), _p(out))
+    return out[:n].copy()
+
+
+def prefill_query(qi_raw, w, k_raw, dtype, kv_bits, q_bits, swa_buf, q_pos0, t, ratio, K, W,
+                  tau, D=512, idx_override=None):
+    """One prefill query token t of a chunk starting at position q_pos0, step by step:
+    indexer scores over the entries visible at p = q_pos0 + t, Top-K, then attention over
+    the selected entries (quantised by the oracle from their bf16 source rows kv_bits
+    [n, D]) plus the token's causal window rows of swa_buf (E4M3 [W-1+T, D]).
+    idx_override: attend over these indices instead of the oracle's own Top-K (for picks
+    that differ inside the near-tie exemption). Returns (idx [K], out float64 [H, D])."""
+    if idx_override is None:
+        n = prefill_visible(q_pos0 + t, ratio)
+        s = index_scores(qi_raw, w, k_raw[:n], dtype)
+        idx = topk(s, K)
+    else:
+        idx = np.asarray(idx_override, np.int32)
+    sel = [int(i) for i in idx if i >= 0]
+    kvb = _c(kv_bits, np.uint16).reshape(-1, D)
+    if sel:
+        c, sc = quantize_entries(kvb[sel], D)
+        main = dequant_entries(c, sc, D)
+    else:
+        main = np.zeros((0, D), np.float64)
+    win = e4m3_array_to_f64(_c(swa_buf, np.uint8).reshape(-1, D)[prefill_window_rows(q_pos0, W, t)])
+    q = bf16_array_to_f64(q_bits).reshape(-1, D)
+    return idx, attention(q, np.concatenate([main, win.reshape(-1, D)], axis=0), tau)
 
 
 def bytes_per_token(D=512, indexer_entry_bytes=68.0, enc_full=3, enc_ratio=2, dec_full=1,

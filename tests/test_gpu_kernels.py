@@ -349,7 +349,7 @@ def test_prefill_indexer_and_attention_small():
     idx_np = idx.cpu().numpy()
     for b in range(B):
         for t in range(T):
-            n = (q_pos0[b] + t + 1) // r
+            n = O.prefill_visible(q_pos0[b] + t, r)
             s = O.index_scores(raw_qk(q_I[b, t]), w[b, t].numpy(), raw_qk(k_I[b, :n]), O.E4M3)
             check_topk(idx_np[b, t], s, np.arange(n), K, f"b={b} t={t}")
     # attention with the oracle's indices
@@ -357,14 +357,16 @@ def test_prefill_indexer_and_attention_small():
     codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
     scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
     C().quantize_kv(kv.to(dev), torch.zeros(B, dtype=torch.int32, device=dev), codes, scales)
-    oidx = np.zeros((B, T, K), np.int32)
-    for b in range(B):
-        for t in range(T):
-            n = (q_pos0[b] + t + 1) // r
-            s = O.index_scores(raw_qk(q_I[b, t]), w[b, t].numpy(), raw_qk(k_I[b, :n]), O.E4M3)
-            oidx[b, t] = O.topk(s, K)
     q = torch.randn((B, T, H, 512), generator=g).to(torch.bfloat16)
     swa = torch.randn((B, W - 1 + T, 512), generator=g).to(torch.float8_e4m3fn)
+    # the oracle's whole prefill query: visibility, scores, Top-K, window rows, attention
+    oidx = np.zeros((B, T, K), np.int32)
+    refs = {}
+    for b in range(B):
+        for t in range(T):
+            oidx[b, t], refs[b, t] = O.prefill_query(
+                raw_qk(q_I[b, t]), w[b, t].numpy(), raw_qk(k_I[b]), O.E4M3, bits16(kv[b]),
+                bits16(q[b, t]), bits8(swa[b]), q_pos0[b], t, r, K, W, 512 ** -0.5)
     out = torch.empty((B, T, H, 512), dtype=torch.float32, device=dev)
     wsa = C().new_workspace(C().workspace_bytes(2, B, T, H, cap, K))
     C().sparse_attn_prefill(q.to(dev), codes, scales, torch.from_numpy(oidx).to(dev), swa.to(dev),
@@ -373,13 +375,7 @@ def test_prefill_indexer_and_attention_small():
     assert C().read_device_status(wsa) == 0
     for b in range(B):
         for t in range(T):
-            sel = [i for i in oidx[b, t] if i >= 0]
-            rows = [oracle_main_rows(bits16(kv[b, sel]))]
-            lo = max(t, (W - 1) - q_pos0[b])       # first buffer row with position >= 0
-            rows.append(O.e4m3_array_to_f64(bits8(swa[b, lo:t + W])).reshape(-1, 512))
-            ref = O.attention(O.bf16_array_to_f64(bits16(q[b, t])).reshape(H, 512),
-                              np.concatenate(rows), 512 ** -0.5)
-            check_attention(out[b, t].cpu().numpy(), ref, f"b={b} t={t}")
+            check_attention(out[b, t].cpu().numpy(), refs[b, t], f"b={b} t={t}")
 
 
 # ---- bounded waits -------------------------------------------------------------------------

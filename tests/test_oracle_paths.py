@@ -204,3 +204,77 @@ def test_bytes_per_token_accounting():
     assert round(v4 / g["global_kv_bytes_per_token"]["value"]) == 4
     assert round(v1 / g["global_kv_bytes_per_token"]["value"]) == g["v1_bytes_per_token"]["ratio_claim"]
     assert g["pool_blocks"]["value"] * g["pool_block_size"]["value"] == g["pool_positions"]["value"]
+
+
+# ---- prefill visibility and the causal window ------------------------------------------
+
+def _simulated_visible_counts(ratio, last_pos):
+    """Feed tokens one by one to a compressor that emits an entry whenever `ratio` tokens
+    have arrived; the count after token p is what that token can read."""
+    counts, pending, emitted = [], 0, 0
+    for _p in range(last_pos + 1):
+        pending += 1
+        if pending == ratio:
+            emitted += 1
+            pending = 0
+        counts.append(emitted)
+    return counts
+
+
+@pytest.mark.parametrize("ratio", [1, 2, 3])
+def test_prefill_visible_matches_token_by_token_compressor(ratio):
+    counts = _simulated_visible_counts(ratio, 200)
+    assert [O.prefill_visible(p, ratio) for p in range(201)] == counts
+    # positions whose p + 1 is not a multiple of the ratio see the previous whole entry only
+    if ratio > 1:
+        assert O.prefill_visible(ratio - 2, ratio) == 0
+        assert O.prefill_visible(2 * ratio - 2, ratio) == 1
+
+
+def test_prefill_visible_at_workload_ends():
+    # 4,096 new tokens on 131,072 cached at ratio 2: the first new token sees the 65,536
+    # cached entries, the last one all 67,584
+    assert O.prefill_visible(131072, 2) == 65536
+    assert O.prefill_visible(131072 + 4095, 2) == 67584
+    assert O.prefill_visible(0, 1) == 1 and O.prefill_visible(0, 2) == 0
+
+
+@pytest.mark.parametrize("q_pos0,W,T", [(0, 4, 9), (3, 4, 6), (0, 128, 200), (127, 128, 3),
+                                        (300, 128, 5), (5, 1, 4), (14, 16, 8)])
+def test_prefill_window_rows_match_buffer_scan(q_pos0, W, T):
+    """Scan the window buffer row by row (row i holds position q_pos0 - (W-1) + i) and keep
+    the rows whose position exists and lies in the token's last W positions."""
+    buf_pos = [q_pos0 - (W - 1) + i for i in range(W - 1 + T)]
+    for t in range(T):
+        p = q_pos0 + t
+        expect = [i for i, pos in enumerate(buf_pos) if pos >= 0 and p - W < pos <= p]
+        got = O.prefill_window_rows(q_pos0, W, t).tolist()
+        assert got == expect, (q_pos0, W, t)
+        assert len(got) == min(W, p + 1)
+        assert got[-1] == t + W - 1          # the token's own row is the last one
+
+
+def test_prefill_query_with_every_entry_selected_is_dense_attention():
+    """K >= visible entries: the prefill query attends over all visible entries and the
+    token's window rows, i.e. plain dense attention over those rows."""
+    rng = np.random.default_rng(21)
+    ratio, q_pos0, T, W, H, D, K = 2, 5, 4, 4, 3, 512, 16
+    cap = (q_pos0 + T) // ratio
+    kv = _bf16_bits(rng.standard_normal((cap, D)))
+    k_I = _e4m3_bits(rng.standard_normal((cap, 128)))
+    swa = _e4m3_bits(rng.standard_normal((W - 1 + T, D)))
+    tau = 1 / math.sqrt(D)
+    for t in range(T):
+        qi = _e4m3_bits(rng.standard_normal((2, 128)))
+        w = rng.random(2).astype(np.float32)
+        q = _bf16_bits(rng.standard_normal((H, D)))
+        idx, out = O.prefill_query(qi, w, k_I, O.E4M3, kv, q, swa, q_pos0, t, ratio, K, W, tau)
+        n = sum(1 for j in range(cap) if ratio * j + ratio - 1 <= q_pos0 + t)
+        assert idx.tolist() == list(range(n)) + [-1] * (K - n)
+        c, s = O.quantize_entries(kv[:n])
+        rows = np.concatenate([O.dequant_entries(c, s),
+                               O.e4m3_array_to_f64(swa[max(t, W - 1 - q_pos0):t + W]).reshape(-1, D)])
+        tq = torch.from_numpy(O.bf16_array_to_f64(q).reshape(H, D))[None, :, None, :]
+        tk = torch.from_numpy(rows)[None, None].expand(1, H, rows.shape[0], D)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tk, scale=tau)
+        np.testing.assert_allclose(out, ref[0, :, 0, :].numpy(), rtol=1e-12, atol=1e-13)
