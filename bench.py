@@ -11,8 +11,9 @@ heads of 512 channels, 128-row FP8 window.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
 
-For N > 1 launch under torchrun: every rank runs its own batch (weak scaling, no collective
-on the data path); the time is the max over ranks.
+For N > 1 bench.py starts N ranks itself (torch.distributed.run on 127.0.0.1) unless it
+already runs under a launcher: every rank runs its own batch (weak scaling, no collective on
+the data path); the time is the max over ranks.
 """
 import argparse
 import hashlib
@@ -485,8 +486,28 @@ def oracle_queries(state, budget_s):
         t_total += time.perf_counter() - t0
         done += 1
         b += 1
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return done, t_total, cores
+    return done, t_total, O.num_threads()
+
+
+# ---- launcher ---------------------------------------------------------------------------------
+
+def _free_port():
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def spawn_ranks(n, argv, timeout_s=3600):
+    """Re-run this script with the same arguments as n ranks of one node
+    (torch.distributed.run on 127.0.0.1); returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1",
+           f"--master-port={_free_port()}", os.path.abspath(__file__)] + list(argv)
+    try:
+        return subprocess.run(cmd, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        return 124
 
 
 # ---- main -------------------------------------------------------------------------------------
@@ -505,9 +526,14 @@ def main():
                     help="launch every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args()
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not under a launcher: start one rank per GPU on this node and wait for them
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         return reference_arm(args, rank, world, local)
     torch.cuda.set_device(local)
@@ -688,6 +714,11 @@ def reference_arm(args, rank, world, local):
     """The oracle, as it stands, timed on the host cores: rank 0 only."""
     if rank != 0:
         return
+    # a launcher's one-thread-per-rank default must not starve the only working rank: the
+    # oracle's parallel loops take every host core
+    if world > 1:
+        from oracle import oracle as O
+        O.set_num_threads(os.cpu_count() or 1)
     w = synth.WORKLOADS[args.workload]
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     if dev.type == "cuda":

@@ -697,6 +697,7 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar[10];   // 0-7: slab j of X and Q landed; 8: S done; 9: P X done
     __shared__ uint32_t tmem_holder;
+    __shared__ int mma_stuck;      // a wait for the last MMA commit gave up: keep TMEM
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const DecSmem L(rps);
@@ -720,6 +721,7 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     if (tid == 0) {
 #pragma unroll
         for (int j = 0; j < 10; ++j) mbar_init(&bar[j], 1);
+        mma_stuck = 0;
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(&tmem_holder, 512);
@@ -859,7 +861,10 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
             }
         mma_commit(&bar[9]);
     }
-    if (!mbar_wait(&bar[9], 0, a.status)) ok = false;
+    if (!mbar_wait(&bar[9], 0, a.status)) {
+        ok = false;
+        mma_stuck = 1;   // MMAs may still write TMEM: it is not released below
+    }
     tc_fence_after();
     __syncthreads();
 
@@ -1031,7 +1036,7 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     if (tid == 0 && !loads_ok)   // a load that timed out may still be in flight: bounded
         for (int j = 0; j < 8; ++j) mbar_wait(&bar[j], 0, a.status);
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0 && !mma_stuck) tmem_dealloc(tmem, 512);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

@@ -11,6 +11,7 @@
 // Record = header (64 B) | codes [n][256] | scales [n][32] | (optional) indexer keys
 // [n][key_bytes] (128 for E4M3 keys, 256 for bf16).
 // The copies are plain cudaMemcpyAsync calls on the caller's stream, one per array.
+#include <cstdint>
 #include <cstring>
 
 #include "csa2.h"
@@ -36,12 +37,25 @@ size_t entry_bytes(int kb) {
     return (size_t)CSA2_ENTRY_CODE_BYTES + CSA2_ENTRY_SCALE_BYTES + (size_t)kb;
 }
 
+// [lo, lo + n) inside [0, cap), tested without forming lo + n (a record's header is
+// untrusted input and may hold values whose sum overflows)
+bool range_ok(int64_t lo, int64_t n, int64_t cap) {
+    return cap >= 1 && lo >= 0 && n >= 0 && n <= cap && lo <= cap - n;
+}
+
+// the byte offsets of sequence b's entries, (b * cap + cap) * (288 + key bytes), fit int64
+bool offsets_ok(int b, int64_t cap, int kb) {
+    const int64_t per = (int64_t)entry_bytes(kb);
+    return b >= 0 && cap >= 1 && cap <= INT64_MAX / per / ((int64_t)b + 1);
+}
+
 }  // namespace
 
 extern "C" {
 
 CSA2_API size_t csa2_cache_record_bytes(int64_t n, int key_bytes) {
     if (n < 0 || !key_bytes_ok(key_bytes)) return 0;
+    if ((uint64_t)n > (SIZE_MAX - sizeof(Header)) / entry_bytes(key_bytes)) return 0;
     return sizeof(Header) + (size_t)n * entry_bytes(key_bytes);
 }
 
@@ -49,10 +63,11 @@ CSA2_API csa2_status_t csa2_cache_export(const uint8_t* codes, const uint8_t* sc
                                          const void* k_I, int key_bytes, int64_t cap, int b,
                                          int64_t lo, int64_t n, void* host, size_t host_bytes,
                                          void* stream) {
-    if (!codes || !scales || !host || cap < 1 || b < 0 || lo < 0 || n < 0 || lo + n > cap)
-        return CSA2_ERR_ARG;
+    if (!codes || !scales || !host || !range_ok(lo, n, cap)) return CSA2_ERR_ARG;
     if (!key_bytes_ok(key_bytes) || (key_bytes > 0) != (k_I != nullptr)) return CSA2_ERR_ARG;
-    if (host_bytes < csa2_cache_record_bytes(n, key_bytes)) return CSA2_ERR_ARG;
+    if (!offsets_ok(b, cap, key_bytes)) return CSA2_ERR_ARG;
+    const size_t need = csa2_cache_record_bytes(n, key_bytes);
+    if (need == 0 || host_bytes < need) return CSA2_ERR_ARG;
     Header h;
     memset(&h, 0, sizeof h);
     h.magic = kMagic;
@@ -91,11 +106,14 @@ CSA2_API csa2_status_t csa2_cache_import(const void* host, size_t host_bytes, ui
     memcpy(&h, host, sizeof h);
     if (h.magic != kMagic || h.version != kVersion) return CSA2_ERR_ARG;
     if (h.d_main != CSA2_D_MAIN || h.d_index != CSA2_D_INDEX) return CSA2_ERR_UNSUPPORTED;
+    // every header field is validated before any arithmetic on it
+    if (h.key_bytes > 2u * CSA2_D_INDEX) return CSA2_ERR_ARG;
     const int kb = (int)h.key_bytes;
-    if (!key_bytes_ok(kb) || h.lo < 0 || h.n < 0 || h.lo + h.n > cap ||
-        h.entry_bytes != entry_bytes(kb))
+    if (!key_bytes_ok(kb) || !range_ok(h.lo, h.n, cap) || h.entry_bytes != entry_bytes(kb))
         return CSA2_ERR_ARG;
-    if (host_bytes < csa2_cache_record_bytes(h.n, kb)) return CSA2_ERR_ARG;
+    if (!offsets_ok(b, cap, kb)) return CSA2_ERR_ARG;
+    const size_t need = csa2_cache_record_bytes(h.n, kb);
+    if (need == 0 || host_bytes < need) return CSA2_ERR_ARG;
     if ((kb > 0) != (k_I != nullptr)) return CSA2_ERR_ARG;   // keys in the record <=> a key cache
     if (h.n == 0) return CSA2_OK;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

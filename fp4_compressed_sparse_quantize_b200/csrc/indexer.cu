@@ -186,6 +186,9 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     uint64_t* done_bar = accempty + ACC;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+    // set when the wait for this CTA's last MMA commit gave up: MMAs may still be in flight,
+    // so neither TMEM nor the shared-memory operands may be released or reused
+    volatile int* mma_stuck = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -207,6 +210,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
+        *mma_stuck = 0;
         fence_mbar_init();
     }
     if (warp >= kEpiWarp0) {
@@ -384,9 +388,13 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             }
         }
         if (!waiter && lane == 0) {
-            // all MMAs must complete before TMEM is released
+            // all MMAs must complete before TMEM is released. If this wait gives up, the
+            // commit never arrived and MMAs may still be reading the stage ring and writing
+            // TMEM: the CTA then leaves its TMEM allocated (the status word carries TIMEOUT,
+            // after which the caller must discard the context) rather than free columns that
+            // the tensor core may still write.
             mma_commit(done_bar);
-            mbar_wait(done_bar, 0, p.status);
+            if (!mbar_wait(done_bar, 0, p.status)) *mma_stuck = 1;
         }
         __syncwarp();
     } else {
@@ -553,7 +561,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+    if (warp == 1 && !*mma_stuck) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 // ---- per-row visible counts and tile prefix ---------------------------------------------
@@ -662,16 +670,9 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int esz, in
     return r == CUDA_SUCCESS;
 }
 
-static int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
+// SM count of the current device (looked up per call: one process may drive GPUs of
+// different sizes)
+static int num_sms() { return device_sm_count(); }
 
 // Largest stage count (<= 8) whose shared-memory plan fits in one SM.
 template <int NQ, int ESZ, int ACC, int G, int EPI, bool POOL, int TM>

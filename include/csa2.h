@@ -30,9 +30,13 @@
  *     csa2_read_device_status(). The status word is sticky until
  *     csa2_reset_device_status() clears it. A workspace must be zero-filled (or reset)
  *     once before first use.
- *   - The library keeps no global mutable state; calls on different streams with
- *     different workspaces may run concurrently. Calls that share a workspace must be
- *     ordered (same stream).
+ *   - Calls on different streams with different workspaces may run concurrently; calls
+ *     that share a workspace must be ordered (same stream). The library's only global
+ *     state is: lookups of immutable facts, made once and shared by all threads under a
+ *     lock or as a benign race of identical values (the driver's tensor-map encoder entry
+ *     point; per decode-attention shape, whether its split clusters fit one wave of the
+ *     current device); the per-host-thread benchmark events of csa2_set_stage_events();
+ *     and the fixed device array of csa2_index_score_topk_noalloc() (see there).
  *   - Fixed geometry: main-KV latent D = 512 channels, indexer dimension 128, candidate
  *     pool blocks of 8 positions. Other sizes return CSA2_ERR_UNSUPPORTED.
  */

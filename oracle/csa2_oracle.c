@@ -42,6 +42,28 @@
 
 #define ORC_EXPORT __attribute__((visibility("default")))
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads for the oracle's parallel loops from now on (n >= 1). */
+ORC_EXPORT void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* Threads the oracle's parallel loops use (for reporting a CPU baseline's core count). */
+ORC_EXPORT int orc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
 /* ------------------------------------------------------------------------------ */
 /* Number formats                                                                  */
 /* ------------------------------------------------------------------------------ */

@@ -62,6 +62,10 @@ def lib():
         L.orc_main_entry_bytes.argtypes = [C.c_int]
         L.orc_kv_bytes_per_token.restype = d
         L.orc_kv_bytes_per_token.argtypes = [C.c_int, d, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.orc_num_threads.restype = C.c_int
+        L.orc_num_threads.argtypes = []
+        L.orc_set_num_threads.restype = None
+        L.orc_set_num_threads.argtypes = [C.c_int]
         L.orc_prefill_visible.restype = i64
         L.orc_prefill_visible.argtypes = [i64, C.c_int]
         L.orc_prefill_window_rows.restype = C.c_int
@@ -76,6 +80,16 @@ def _p(a):
 
 def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_num_threads(n):
+    """Threads for the oracle's parallel loops from now on."""
+    lib().orc_set_num_threads(int(n))
+
+
+def num_threads():
+    """Threads the oracle's parallel loops use."""
+    return int(lib().orc_num_threads())
 
 
 # ---- formats -------------------------------------------------------------------------

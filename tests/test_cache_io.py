@@ -42,7 +42,13 @@ def _header(magic=0x32415343, version=1, d=512, di=128, lo=0, n=4, kb=0, eb=288)
                                         (dict(eb=300), csa2.ERR_ARG),
                                         (dict(kb=100, eb=388), csa2.ERR_ARG),
                                         (dict(lo=998), csa2.ERR_ARG),
-                                        (dict(n=1000), csa2.ERR_ARG)])
+                                        (dict(n=1000), csa2.ERR_ARG),
+                                        # forged ranges whose sums or byte sizes overflow
+                                        (dict(lo=2**62, n=2**62), csa2.ERR_ARG),
+                                        (dict(lo=2**63 - 1, n=1), csa2.ERR_ARG),
+                                        (dict(lo=-1, n=2), csa2.ERR_ARG),
+                                        (dict(lo=0, n=2**60), csa2.ERR_ARG),
+                                        (dict(kb=2**31 + 128, eb=416), csa2.ERR_ARG)])
 def test_import_rejects_bad_records_before_copying(bad, status):
     rec = np.zeros(64 + 4 * 288, np.uint8)
     rec[:64] = _header(**bad)
@@ -50,6 +56,11 @@ def test_import_rejects_bad_records_before_copying(bad, status):
     st = csa2.lib().csa2_cache_import(rec.ctypes.data_as(C.c_void_p), rec.nbytes, fake, fake,
                                       None, 1000, 0, None)
     assert st == status
+
+
+def test_record_bytes_overflow_is_rejected():
+    assert csa2.cache_record_bytes(2**62) == 0
+    assert csa2.cache_record_bytes(2**62, 256) == 0
 
 
 def test_export_rejects_bad_arguments():
@@ -61,6 +72,9 @@ def test_export_rejects_bad_arguments():
     assert L.csa2_cache_export(fake, fake, None, 0, 100, 0, 96, 8, hp, host.nbytes, None) == csa2.ERR_ARG
     assert L.csa2_cache_export(fake, fake, None, 128, 100, 0, 0, 8, hp, host.nbytes, None) == csa2.ERR_ARG
     assert L.csa2_cache_export(fake, fake, fake, 128, 100, 0, 0, 8, hp, 64 + 8 * 300, None) == csa2.ERR_ARG
+    # ranges whose end overflows int64, and a sequence offset past int64
+    assert L.csa2_cache_export(fake, fake, None, 0, 100, 0, 2**63 - 1, 8, hp, host.nbytes, None) == csa2.ERR_ARG
+    assert L.csa2_cache_export(fake, fake, None, 0, 2**62, 2**30, 0, 8, hp, host.nbytes, None) == csa2.ERR_ARG
 
 
 @pytest.mark.gpu

@@ -60,9 +60,12 @@ def test_noalloc_matches_workspace_entry_point_twice():
     csa2.index_score_topk("reindex", q_I, w, k_I, K, idx2_ref, ws2, n_vis0=n_vis,
                           pool_in=pool_ref)
     idx2 = torch.empty_like(idx2_ref)
+    status2 = torch.zeros(1, dtype=torch.int32, device=dev)
     csa2.index_score_topk_noalloc("reindex", q_I, w, k_I, K, idx2, n_vis0=n_vis,
-                                  pool_in=pool_ref)
+                                  pool_in=pool_ref, status=status2)
     torch.cuda.synchronize()
+    assert csa2.read_device_status(ws2) == 0
+    assert int(status2.item()) == 0, "device status of the Reindex call"
     assert torch.equal(idx2, idx2_ref)
 
 
