@@ -35,6 +35,9 @@ sys.path.insert(0, ROOT)
 from fp4_compressed_sparse_quantize_b200 import csa2, synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "decode_full_b32_ctx64k_r2"
+# reported beside the default line: the rest of the 64K-1M decode range and the prefill chunk
+EXTRA_DECODE = ("decode_group4_b64_ctx256k", "decode_pool_reindex_b4_ctx1m")
+EXTRA_PREFILL = "prefill_b2_t4k_ctx128k_r2"
 L2_FLUSH_BYTES = 256 << 20
 SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csrc", "indexer.cu")
 
@@ -160,7 +163,10 @@ class Decode:
         self.ws_attn = csa2.new_workspace(csa2.workspace_bytes(1, B, 1, w.H, cap, w.K))
         torch.cuda.synchronize()
 
-    def step(self, scan_events=None, stream=None):
+    def step(self, scan_events=None, attn_events=None, stream=None):
+        """One decode step. scan_events: (start, stop) around the first Full layer's indexer
+        scan; attn_events: one (start, stop) pair per layer around its attention call (both
+        become external event nodes when the step is captured into a graph)."""
         w = self.w
         csa2.quantize_kv(self.kv_new, self.dst, self.codes, self.scales,
                          status=self.ws_idx[:4].view(torch.int32), stream=stream)
@@ -184,9 +190,13 @@ class Decode:
             else:
                 csa2.index_score_topk("reuse", L["q_I"], L["w"], self.k_I, w.K, cur,
                                       self.ws_idx, n_vis0=self.n_vis, stream=stream)
+            if attn_events is not None:
+                csa2.record_event(attn_events[li][0], stream)
             csa2.sparse_attn_decode(mode, L["q"], self.codes, self.scales, cur.view(w.B, w.K),
                                     L["swa"], self.out[li], self.ws_attn, scale=self.tau,
                                     stream=stream)
+            if attn_events is not None:
+                csa2.record_event(attn_events[li][1], stream)
 
     def launches_per_step(self):
         """Kernels of this library per step (memsets excluded)."""
@@ -237,6 +247,14 @@ class Decode:
             tot += B * (K * 4 + K * 288 + W * 512 + H * 512 * 2 + H * 512 * 4)
         return tot, scan
 
+    def attention_bytes(self):
+        """Algorithmic bytes of every layer's decode attention in one step: per query the
+        K indices, the K gathered FP4 entries (288 B), the W window rows (512 B E4M3), the bf16
+        query and the fp32 output."""
+        w = self.w
+        per_q = w.K * 4 + w.K * 288 + synth.WINDOW * 512 + w.H * 512 * 2 + w.H * 512 * 4
+        return len(w.layers) * w.B * per_q
+
 
 def flush_l2(buf, k):
     """Evict L2 between timed steps: write a buffer twice the size of L2, then read it back
@@ -245,9 +263,9 @@ def flush_l2(buf, k):
     torch.sum(buf.view(torch.int64))
 
 
-def capture_steps(state, events, stream):
-    """One CUDA graph per timed step: the step's library calls, with that step's pair of
-    scan events recorded inside (as external event nodes)."""
+def capture_steps(state, events, attn_events, stream):
+    """One CUDA graph per timed step: the step's library calls, with that step's scan events
+    and per-layer attention events recorded inside (as external event nodes)."""
     graphs = []
     side = torch.cuda.Stream()
     side.wait_stream(stream)
@@ -255,13 +273,104 @@ def capture_steps(state, events, stream):
         state.step()                      # warm the side stream
     stream.wait_stream(side)
     torch.cuda.synchronize()
-    for ev in events:
+    for ev, aev in zip(events, attn_events):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
-            state.step(scan_events=ev, stream=side)
+            state.step(scan_events=ev, attn_events=aev, stream=side)
         graphs.append(g)
     torch.cuda.synchronize()
     return graphs
+
+
+def _event_pair():
+    pair = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    return pair
+
+
+def timed_decode(state, steps, warmup, stream, local, eager=False, pg=None):
+    """Warm up, then time `steps` decode steps (one graph replay each, L2 flushed between
+    them outside the events) with the scan and attention events inside. Returns a dict of
+    the device-timed figures (milliseconds) and the clocks seen."""
+    w = state.w
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=stream.device)
+    for _ in range(max(3, warmup)):
+        state.step()
+    torch.cuda.synchronize()
+    assert csa2.read_device_status(state.ws_idx) == 0, "device status set during warm-up"
+    assert csa2.read_device_status(state.ws_attn) == 0
+    ev = [_event_pair() for _ in range(steps)]
+    sev = [_event_pair() for _ in range(steps)]
+    aev = [[_event_pair() for _ in w.layers] for _ in range(steps)]
+    for pair in sev + [p for step in aev for p in step]:   # events exist once recorded
+        pair[0].record(stream)
+        pair[1].record(stream)
+    # Each timed step is one CUDA-graph replay of the whole step (captured once per step so
+    # that every replay records its own events): launches reach the GPU back to back.
+    graphs = capture_steps(state, sev, aev, stream) if not eager else None
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(local)
+    clocks.start()
+    for k in range(steps):
+        flush_l2(flush, k)                      # evict L2 between steps (outside the events)
+        ev[k][0].record(stream)
+        if graphs:
+            graphs[k].replay()
+        else:
+            state.step(scan_events=sev[k], attn_events=aev[k])
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if pg:
+        pg.barrier()
+    del graphs, flush
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    has_scan = any(m == "full" for m in w.layers)
+    scan_ms = [a.elapsed_time(b) for a, b in sev] if has_scan else [0.0]
+    attn_ms = [sum(a.elapsed_time(b) for a, b in step) for step in aev]
+    return {"step_ms": step_ms, "scan_ms": scan_ms, "attn_ms": attn_ms, "clocks": clk}
+
+
+def decode_summary(state, tm, peak):
+    """Per-workload figures of a timed_decode run: queries/s, the step's HBM rate and the
+    rooflines of the indexer scan (the dominant kernel) and of the decode attention (row
+    staging + attention kernels, every layer), each as algorithmic bytes over device time."""
+    w = state.w
+    steps = len(tm["step_ms"])
+    per_step = sum(tm["step_ms"]) / steps
+    alg, scan_bytes = state.algorithmic_bytes()
+    scan_avg = sum(tm["scan_ms"]) / len(tm["scan_ms"])
+    attn_avg = sum(tm["attn_ms"]) / steps
+    ab = state.attention_bytes()
+    out = {"queries_per_s": w.B / (per_step / 1e3), "ms_per_step": per_step,
+           "hbm_gbs_step": alg / (per_step / 1e3) / 1e9,
+           "step_roofline_frac": alg / (per_step / 1e3) / 1e9 / peak,
+           "attention": {"bound": "hbm", "bytes_per_step": ab, "avg_ms_per_step": attn_avg,
+                         "achieved": ab / (attn_avg / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": ab / (attn_avg / 1e3) / 1e9 / peak}}
+    if scan_bytes:
+        out["scan"] = {"bound": "hbm", "bytes_per_launch": scan_bytes, "avg_launch_ms": scan_avg,
+                       "achieved": scan_bytes / (scan_avg / 1e3) / 1e9, "peak": peak,
+                       "unit": "GB/s", "frac": scan_bytes / (scan_avg / 1e3) / 1e9 / peak}
+    return out
+
+
+def extra_decode(name, args, dev, local):
+    """A shorter timed run of another decode workload (its own state, freed afterwards)."""
+    w = synth.WORKLOADS[name]
+    state = Decode(w, args.seed, dev)
+    tm = timed_decode(state, args.extra_steps, 3, torch.cuda.current_stream(dev), local)
+    peak, _ = peaks()
+    out = decode_summary(state, tm, peak)
+    out.update({"steps": args.extra_steps, "batch": w.B, "context_tokens": w.ctx,
+                "compressed_entries": w.N, "layers": list(w.layers), "clocks": tm["clocks"],
+                "device_status": [csa2.read_device_status(state.ws_idx),
+                                  csa2.read_device_status(state.ws_attn)]})
+    del state
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
 
 
 def max_over_ranks(ms, pg, dev):
@@ -336,57 +445,72 @@ class Prefill:
         return scan, attn
 
 
-def prefill_main(args, w, dev, rank, world):
-    state = Prefill(w, rank_seed(args.seed, rank), dev)
+def measure_prefill(w, seed, steps, warmup, dev):
+    """Time `steps` chunked-prefill steps with the scan and attention events inside; returns
+    the tokens/s and the tensor-roofline figures of the indexer scan and the attention."""
+    state = Prefill(w, seed, dev)
     stream = torch.cuda.current_stream(dev)
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         state.step()
     torch.cuda.synchronize()
     assert csa2.read_device_status(state.ws) == 0 and csa2.read_device_status(state.wsa) == 0
     mk = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-    ev = [mk() for _ in range(args.steps)]
-    sev = [mk() for _ in range(args.steps)]
-    aev = [mk() for _ in range(args.steps)]
+    ev = [mk() for _ in range(steps)]
+    sev = [mk() for _ in range(steps)]
+    aev = [mk() for _ in range(steps)]
     for pair in sev + aev:
         pair[0].record(stream)
         pair[1].record(stream)
     torch.cuda.synchronize()
     clocks = Clocks(local_rank())
     clocks.start()
-    for k in range(args.steps):
+    for k in range(steps):
         ev[k][0].record(stream)
         state.step(scan_events=sev[k], attn_events=aev[k])
         ev[k][1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
+    st = [csa2.read_device_status(state.ws), csa2.read_device_status(state.wsa)]
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    scan_ms = sum(a.elapsed_time(b) for a, b in sev) / args.steps
-    attn_ms = sum(a.elapsed_time(b) for a, b in aev) / args.steps
+    scan_ms = sum(a.elapsed_time(b) for a, b in sev) / steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in aev) / steps
     scan_f, attn_f = state.flops()
     bf16 = measured_bf16_tflops()
-    tokens = w.B * w.T * args.steps
+    tokens = w.B * w.T * steps
+    del state
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": tokens / (total_ms / 1e3), "ms_per_step": total_ms / steps,
+            "scan": {"kernel": "csa2 indexer scan (tcgen05 kind::f8f6f4)", "bound": "tensor",
+                     "achieved": scan_f / (scan_ms / 1e3) / 1e12, "peak": 2 * bf16,
+                     "unit": "TFLOP/s", "frac": scan_f / (scan_ms / 1e3) / 1e12 / (2 * bf16),
+                     "peak_source": "measured bf16 x 2 (FP8/bf16 nominal ratio)",
+                     "flops_per_launch": scan_f, "avg_launch_ms": scan_ms},
+            "attention": {"kernel": "csa2 prefill attention (tcgen05 kind::f16)",
+                          "bound": "tensor", "achieved": attn_f / (attn_ms / 1e3) / 1e12,
+                          "peak": bf16, "unit": "TFLOP/s",
+                          "frac": attn_f / (attn_ms / 1e3) / 1e12 / bf16,
+                          "flops_per_call": attn_f, "avg_call_ms": attn_ms},
+            "clocks": clk, "device_status": st, "steps": steps}
+
+
+def prefill_main(args, w, dev, rank, world):
+    m = measure_prefill(w, rank_seed(args.seed, rank), args.steps, args.warmup, dev)
     line = {
         "metric": "CSA2 chunked prefill tokens/s (FP8 indexer + sparse attention), 1 B200",
-        "value": tokens / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "value": m["tokens_per_s"] * world, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup),
-        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3 indexer / fp16 attention (fp32 accumulate)",
         "data": "synthetic",
         "config": {"workload": w.name, "batch": w.B, "new_tokens": w.T, "cached_tokens": w.ctx,
                    "ratio": w.ratio, "topk": w.K, "indexer_heads": w.H_I, "query_heads": w.H,
                    "window": synth.WINDOW, "l2": "inputs larger than L2"},
-        "roofline": {"kernel": "csa2 indexer scan (tcgen05 kind::f8f6f4)", "bound": "tensor",
-                     "achieved": scan_f / (scan_ms / 1e3) / 1e12,
-                     "peak": 2 * bf16, "unit": "TFLOP/s",
-                     "frac": scan_f / (scan_ms / 1e3) / 1e12 / (2 * bf16),
-                     "peak_source": "measured bf16 x 2 (FP8/bf16 nominal ratio)",
-                     "flops_per_launch": scan_f, "avg_launch_ms": scan_ms, "traffic": None},
-        "attention": {"bound": "tensor", "achieved": attn_f / (attn_ms / 1e3) / 1e12,
-                      "peak": bf16, "unit": "TFLOP/s",
-                      "frac": attn_f / (attn_ms / 1e3) / 1e12 / bf16,
-                      "flops_per_call": attn_f, "avg_call_ms": attn_ms},
+        "roofline": m["scan"],
+        "attention": m["attention"],
         "gpu_launches": 5 * args.steps,   # quantize, prep, scan, Top-K, attention
-        "clocks": clk,
+        "clocks": m["clocks"],
+        "device_status": m["device_status"],
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -522,6 +646,9 @@ def main():
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the shorter runs of the other workloads (256K, 1M, prefill)")
+    ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--eager", action="store_true",
                     help="launch every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args()
@@ -553,44 +680,9 @@ def main():
             pg.destroy_process_group()
         return
     state = Decode(w, rank_seed(args.seed, rank), dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-
-    for _ in range(max(3, args.warmup)):
-        state.step()
-    torch.cuda.synchronize()
-    assert csa2.read_device_status(state.ws_idx) == 0, "device status set during warm-up"
-    assert csa2.read_device_status(state.ws_attn) == 0
-
-    clocks = Clocks(local)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for a, b in sev:           # torch creates the CUDA event on first record
-        a.record(stream)
-        b.record(stream)
-    # Each timed step is one CUDA-graph replay of the whole step (captured once per step so
-    # that every replay records its own scan events): launches reach the GPU back to back.
-    graphs = capture_steps(state, sev, stream) if not args.eager else None
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    for k in range(args.steps):
-        flush_l2(flush, k)                      # evict L2 between steps (outside the events)
-        ev[k][0].record(stream)
-        if graphs:
-            graphs[k].replay()
-        else:
-            state.step(scan_events=sev[k])
-        ev[k][1].record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    if pg:
-        pg.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    scan_ms = [a.elapsed_time(b) for a, b in sev]
+    tm = timed_decode(state, args.steps, args.warmup, stream, local, args.eager, pg)
+    step_ms, scan_ms, attn_ms, clk = tm["step_ms"], tm["scan_ms"], tm["attn_ms"], tm["clocks"]
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
 
     # end-to-end: host inputs -> device -> step -> host output, through the public API.
@@ -662,6 +754,17 @@ def main():
     st_i = csa2.read_device_status(state.ws_idx)
     st_a = csa2.read_device_status(state.ws_attn)
 
+    # other workloads of the metric's 64K-1M range (and the prefill chunk): one GPU only
+    extra = {}
+    if world == 1 and not args.no_extra:
+        state_keep = state
+        for name in EXTRA_DECODE:
+            if name != args.workload:
+                extra[name] = extra_decode(name, args, dev, local)
+        pw = synth.WORKLOADS[EXTRA_PREFILL]
+        extra[EXTRA_PREFILL] = measure_prefill(pw, args.seed, args.extra_steps, 3, dev)
+        state = state_keep
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, secs, cores = oracle_queries(state, args.cpu_budget)
@@ -695,6 +798,7 @@ def main():
                          "bytes_per_launch": scan_bytes, "avg_launch_ms": scan_avg,
                          "traffic": traffic},
             "step_roofline_frac": (alg_bytes / (per_step_ms / 1e3) / 1e9) / peak,
+            "attention_roofline": decode_summary(state, tm, peak)["attention"],
             "e2e": {"value": queries / (e2e_ms / 1e3), "unit": "queries/s",
                     "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                     "schedule": "pipelined: step k+1's inputs in and step k-1's outputs out "
@@ -703,6 +807,7 @@ def main():
             "clocks": clk,
             "device_status": [st_i, st_a],
             "cpu_baseline": cpu,
+            "workloads": extra,
         }
         print(json.dumps(line), flush=True)
     if pg:

@@ -27,7 +27,7 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
            "csa2_cp_pool_expand", "csa2_cache_record_bytes", "csa2_cache_export",
            "csa2_cache_import", "csa2_cp_local_idx", "csa2_sparse_attn_decode_partial",
-           "csa2_attn_merge_partials")
+           "csa2_attn_merge_partials", "csa2_record_event")
 
 
 class Csa2Error(RuntimeError):
@@ -63,6 +63,7 @@ def lib():
         L.csa2_reset_device_status.argtypes = [P, P]
         L.csa2_debug_bounded_wait.argtypes = [P, C.c_uint64, P]
         L.csa2_set_stage_events.argtypes = [P, P]
+        L.csa2_record_event.argtypes = [P, P]
         L.csa2_index_score_topk_noalloc.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P,
                                                     i32, P, i32, P, i32, P, i32, P, P, P, P]
         L.csa2_sparse_attn_decode_launches.argtypes = [i32, i32, i32]
@@ -153,6 +154,14 @@ def set_stage_events(ev_start, ev_stop):
     a = C.c_void_p(ev_start.cuda_event) if ev_start is not None else None
     b = C.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
     _check(lib().csa2_set_stage_events(a, b), "csa2_set_stage_events")
+
+
+def record_event(ev, stream=None):
+    """Record torch.cuda.Event `ev` (created already: record it once beforehand) on the stream;
+    inside a stream capture the record becomes an external node of the graph, so replays can
+    be timed between two such events."""
+    _check(lib().csa2_record_event(C.c_void_p(ev.cuda_event), _stream(stream)),
+           "csa2_record_event")
 
 
 def debug_bounded_wait(status_word, timeout_ns, stream=None):

@@ -166,6 +166,16 @@ csa2_status_t csa2_set_stage_events(void* ev_start, void* ev_stop) {
     return CSA2_OK;
 }
 
+csa2_status_t csa2_record_event(void* ev, void* stream) {
+    if (!ev) return CSA2_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus capst = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &capst) != cudaSuccess) return CSA2_ERR_CUDA;
+    const unsigned flags =
+        capst == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    return cuda_status(cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(ev), st, flags));
+}
+
 csa2_status_t csa2_reset_device_status(void* ws, void* stream) {
     if (!ws) return CSA2_ERR_ARG;
     return cuda_status(

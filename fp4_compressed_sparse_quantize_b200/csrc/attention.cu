@@ -35,21 +35,21 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const CombineArgs a) 
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             v[j] = s0 + j < nsplit
-                       ? __ldg(reinterpret_cast<const float4*>(base + (s0 + j) * a.o_s +
+                       ? ld_dep(reinterpret_cast<const float4*>(base + (s0 + j) * a.o_s +
                                                                (int64_t)h * kDm + c))
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     load8(0);
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldg(mls + s * a.ml_s));
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ld_dep(mls + s * a.ml_s));
     const float Mb = (M == -INFINITY) ? 0.f : M;
     for (int s0 = 0; s0 < nsplit; s0 += 8) {
         if (s0 > 0) load8(s0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if (s0 + j < nsplit) {
-                const float wv = exp2f(__ldg(mls + (s0 + j) * a.ml_s) - Mb);
-                L += wv * __ldg(mls + (s0 + j) * a.ml_s + H);
+                const float wv = exp2f(ld_dep(mls + (s0 + j) * a.ml_s) - Mb);
+                L += wv * ld_dep(mls + (s0 + j) * a.ml_s + H);
                 acc.x += wv * v[j].x;
                 acc.y += wv * v[j].y;
                 acc.z += wv * v[j].z;
@@ -95,8 +95,10 @@ int attention_splits(int Q, int K, int W, bool prefill) {
 }
 
 cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merged);
+cudaError_t launch_attention_prefill(const AttnLaunch& l, cudaStream_t st);
 
 cudaError_t launch_attention(const AttnLaunch& l, cudaStream_t st) {
+    if (l.prefill) return launch_attention_prefill(l, st);
     bool merged = false;
     cudaError_t e = launch_attention_tc(l, st, &merged);
     const bool part = l.o_part != nullptr;

@@ -139,7 +139,7 @@ __device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, 
     const uint8_t* src_scales = nullptr;
     const uint8_t* src_swa = nullptr;
     if (g < a.K) {
-        const int32_t e = __ldg(a.idx + (int64_t)qrow * a.K + g);
+        const int32_t e = ld_dep(a.idx + (int64_t)qrow * a.K + g);
         if (e >= 0 && e < a.cap) {
             kind = 1;
             const int64_t ent = (int64_t)b * a.cap + e;
@@ -153,13 +153,13 @@ __device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, 
         int64_t srow;
         bool ok;
         if (!a.prefill) {
-            const int nv = a.swa_valid ? __ldg(a.swa_valid + b) : a.W;
+            const int nv = a.swa_valid ? ld_dep(a.swa_valid + b) : a.W;
             ok = v >= a.W - nv;
             srow = (int64_t)b * a.W + v;
         } else {
             const int64_t rw = t + v;
             const int64_t pos =
-                (a.q_pos0 ? (int64_t)__ldg(a.q_pos0 + b) : (int64_t)(a.W - 1)) - (a.W - 1) + rw;
+                (a.q_pos0 ? (int64_t)ld_dep(a.q_pos0 + b) : (int64_t)(a.W - 1)) - (a.W - 1) + rw;
             ok = pos >= 0;
             srow = (int64_t)b * (a.W - 1 + a.T) + rw;
         }
@@ -174,11 +174,11 @@ __device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, 
     uint4 sc4 = make_uint4(0, 0, 0, 0);
     if (kind == 1) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) raw[k] = __ldg(reinterpret_cast<const uint4*>(src_codes) + k);
-        sc4 = __ldg(reinterpret_cast<const uint4*>(src_scales));
+        for (int k = 0; k < 8; ++k) raw[k] = ld_dep(reinterpret_cast<const uint4*>(src_codes) + k);
+        sc4 = ld_dep(reinterpret_cast<const uint4*>(src_scales));
     } else if (kind == 2) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) raw[k] = __ldg(reinterpret_cast<const uint4*>(src_swa) + k);
+        for (int k = 0; k < 16; ++k) raw[k] = ld_dep(reinterpret_cast<const uint4*>(src_swa) + k);
     }
     const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
     // 16 groups of 16 channels: group gl covers channels 256*part + 16*gl
@@ -268,12 +268,12 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
         int kind = 0;
         uint32_t hv[8];
         if (r < a.K) {
-            const int32_t e = __ldg(a.idx + (int64_t)b * a.K + r);
+            const int32_t e = ld_dep(a.idx + (int64_t)b * a.K + r);
             if (e >= 0 && e < a.cap) {
                 kind = 1;
                 const int64_t ent = (int64_t)b * a.cap + e;
-                const uint2 cb = __ldg(reinterpret_cast<const uint2*>(a.codes + ent * CSA2_ENTRY_CODE_BYTES) + lane);
-                const uint8_t sb = __ldg(a.scales + ent * CSA2_ENTRY_SCALE_BYTES + lane);
+                const uint2 cb = ld_dep(reinterpret_cast<const uint2*>(a.codes + ent * CSA2_ENTRY_CODE_BYTES) + lane);
+                const uint8_t sb = ld_dep(a.scales + ent * CSA2_ENTRY_SCALE_BYTES + lane);
                 const __half2 s2 = __half2half2(__float2half_rn(e4m3_to_float(sb)));
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -286,10 +286,10 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
             }
         } else {
             const int v = r - a.K;   // window row 0..W-1, oldest first
-            const int nv = a.swa_valid ? __ldg(a.swa_valid + b) : a.W;
+            const int nv = a.swa_valid ? ld_dep(a.swa_valid + b) : a.W;
             if (v >= a.W - nv) {
                 kind = 2;
-                const uint4 eb = __ldg(reinterpret_cast<const uint4*>(a.swa + ((int64_t)b * a.W + v) * kD) + lane);
+                const uint4 eb = ld_dep(reinterpret_cast<const uint4*>(a.swa + ((int64_t)b * a.W + v) * kD) + lane);
                 const uint32_t ew[4] = {eb.x, eb.y, eb.z, eb.w};
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
     float amax = 0.f;
     if (h < a.H) {
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((int64_t)b * a.H + h) * kD + lane * 16);
-        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+        const uint4 u0 = ld_dep(src), u1 = ld_dep(src + 1);
         const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -393,8 +393,8 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
     if constexpr (STAGED) {
         const int r0 = c_begin * kRows + tid;
         if (tid < kRows && r0 < a.K + a.W)
-            pre_valid = __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r0);
-        if (tid < kHeads) pre_qf = __ldg(a.st_qf + qrow * kHeads + tid);
+            pre_valid = ld_dep(a.st_valid + (int64_t)qrow * (a.K + a.W) + r0);
+        if (tid < kHeads) pre_qf = ld_dep(a.st_qf + qrow * kHeads + tid);
     }
     bool first_chunk = true;
     if (warp == 0) tmem_alloc(tmem_holder, 512);
@@ -487,9 +487,9 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__
                 if (tid < kRows) {
                     const int r = ch * kRows + tid;
                     rvalid[tid] =
-                        (r < a.K + a.W) ? __ldg(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
+                        (r < a.K + a.W) ? ld_dep(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
                 }
-                if (tid < kHeads) qf[tid] = __ldg(a.st_qf + qrow * kHeads + tid);
+                if (tid < kHeads) qf[tid] = ld_dep(a.st_qf + qrow * kHeads + tid);
             }
             wait_bar(2);
             __syncthreads();
@@ -737,8 +737,8 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     // row kinds and logit factors, held in registers until the Q tile is dead
     int pre_valid = 0;
     float pre_qf = 0.f;
-    if (tid < rps && r0 + tid < rows) pre_valid = __ldg(a.st_valid + (int64_t)qrow * rows + r0 + tid);
-    if (tid < kHeads) pre_qf = __ldg(a.st_qf + qrow * kHeads + tid);
+    if (tid < rps && r0 + tid < rows) pre_valid = ld_dep(a.st_valid + (int64_t)qrow * rows + r0 + tid);
+    if (tid < kHeads) pre_qf = ld_dep(a.st_qf + qrow * kHeads + tid);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

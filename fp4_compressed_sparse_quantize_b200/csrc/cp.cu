@@ -53,7 +53,7 @@ __device__ __forceinline__ int cp_excl_scan(int v, int* warp_sums, int* total) {
 // (score, global index) of every selected entry of a shard's Top-K list; -1 entries give
 // (0, -1).
 __global__ void __launch_bounds__(256) cp_topk_candidates_kernel(
-    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ idx, int K,
+    const float* scores, int64_t ld, const int32_t* idx, int K,
     int64_t offset, float* __restrict__ cand_score, int32_t* __restrict__ cand_idx) {
     grid_dep_launch();
     grid_dep_wait();
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256) cp_topk_candidates_kernel(
 // visible positions of a chosen block present, -1 padded); at most nb blocks per row, the
 // rest of the row is (0, -1).
 __global__ void __launch_bounds__(kCpThreads) cp_pool_candidates_kernel(
-    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ pool, int P,
+    const float* scores, int64_t ld, const int32_t* pool, int P,
     int nb, int64_t offset, float* __restrict__ cand_bmax, int32_t* __restrict__ cand_block) {
     __shared__ int warp_sums[32];
     grid_dep_launch();
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kCpThreads) cp_pool_candidates_kernel(
 // (order-preserving score bits, then the complemented index) by a bitonic network in shared
 // memory; the chosen indices are sorted again, ascending.
 __global__ void __launch_bounds__(kCpThreads) cp_merge_kernel(
-    const float* __restrict__ cand_score, const int32_t* __restrict__ cand_idx, int n_cand,
+    const float* cand_score, const int32_t* cand_idx, int n_cand,
     int n2, int K, int k2, int32_t* __restrict__ idx_out) {
     extern __shared__ __align__(16) uint64_t key[];   // [n2], then uint32 [k2]
     uint32_t* sel = reinterpret_cast<uint32_t*>(key + n2);
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kCpThreads) cp_merge_kernel(
 // Entry positions of merged pool blocks (ascending, -1 padded): block b gives the visible
 // positions among 8b .. 8b+7.
 __global__ void __launch_bounds__(kCpThreads) cp_pool_expand_kernel(
-    const int32_t* __restrict__ blocks, int nb, const int32_t* __restrict__ n_row, int P,
+    const int32_t* blocks, int nb, const int32_t* n_row, int P,
     int32_t* __restrict__ pool_out) {
     __shared__ int warp_sums[32];
     grid_dep_launch();
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kCpThreads) cp_pool_expand_kernel(
 
 // Global selected indices -> this shard's local indices (-1 outside [lo, hi)), for the
 // shard's partial attention over the rows it holds.
-__global__ void __launch_bounds__(256) cp_local_idx_kernel(const int32_t* __restrict__ idx,
+__global__ void __launch_bounds__(256) cp_local_idx_kernel(const int32_t* idx,
                                                            int64_t n, int64_t lo, int64_t hi,
                                                            int32_t* __restrict__ out) {
     grid_dep_launch();

@@ -124,8 +124,21 @@ __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
 __device__ __forceinline__ void grid_dep_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// The wait is followed by a generic-to-async proxy fence on global memory: the previous
+// kernel's plain stores are read here by TMA and bulk copies (the async proxy).
 __device__ __forceinline__ void grid_dep_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Load of global data that an earlier kernel on the stream may have written. A dependent
+// kernel starts while that kernel still runs, so nothing it reads is read-only for its whole
+// lifetime: a read-only-path load (__ldg, ld.global.nc, or a const __restrict__ kernel
+// argument) is treated by the compiler as invariant memory and may be scheduled ahead of
+// griddepcontrol.wait, before the data exists. A plain load stays ordered after the wait's
+// memory clobber.
+template <class T>
+__device__ __forceinline__ T ld_dep(const T* p) {
+    return *p;
 }
 
 // ---- TMA (no multicast anywhere in this library) --------------------------------------

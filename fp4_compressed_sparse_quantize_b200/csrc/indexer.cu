@@ -109,8 +109,8 @@ struct GroupCursor {
     int64_t lo, hi;
     __device__ __forceinline__ void init(const int64_t* prefix, int ngroups, int64_t t) {
         g = find_group(prefix, ngroups, t);
-        lo = __ldg(prefix + g);
-        hi = __ldg(prefix + g + 1);
+        lo = ld_dep(prefix + g);
+        hi = ld_dep(prefix + g + 1);
     }
     // returns true when t starts a new row group
     __device__ __forceinline__ bool advance(const int64_t* prefix, int64_t t) {
@@ -118,7 +118,7 @@ struct GroupCursor {
         while (t >= hi) {
             ++g;
             lo = hi;
-            hi = __ldg(prefix + g + 1);
+            hi = ld_dep(prefix + g + 1);
             moved = true;
         }
         return moved;
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     const uint32_t tmem_base = *tmem_holder;
     // the tile prefix (and everything else in global memory) comes from earlier kernels
     grid_dep_wait();
-    const int64_t total = __ldg(p.prefix + ngroups);
+    const int64_t total = ld_dep(p.prefix + ngroups);
     const int64_t t0 = total * blockIdx.x / gridDim.x;
     const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
 
@@ -286,12 +286,12 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             } else {
                 // pool rows of query row r0 (G == 1 in gather mode)
                 const int32_t* pl = p.pool + (int64_t)r0 * p.P + jt * kRowsT;
-                const int n_vis = __ldg(p.n_row + r0);
+                const int n_vis = ld_dep(p.n_row + r0);
                 const uint32_t dst_u = smem_u32(dst);
                 for (int rr = 0; rr < kRowsT; rr += 4) {
                     const int rl = rr + (lane >> 3);       // 4 rows per pass, 8 lanes per row
                     const int64_t slot = jt * kRowsT + rl;
-                    int pos = (slot < p.P) ? __ldg(pl + rl) : -1;
+                    int pos = (slot < p.P) ? ld_dep(pl + rl) : -1;
                     if (pos >= n_vis) pos = -1;
                     if (pos >= 0) {
                         const uint8_t* src = p.keys + ((int64_t)b * p.cap + pos) * (128 * ESZ);
@@ -453,14 +453,14 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                 since_flush = 0;
                 wslot ^= 1;
                 for (int i = et; i < NQ; i += 128)
-                    w_e[wslot * NQ + i] = (i < G * p.H_I) ? __ldg(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
+                    w_e[wslot * NQ + i] = (i < G * p.H_I) ? ld_dep(p.w + (int64_t)r0 * p.H_I + i) : 0.f;
                 epi_bar_sync(e);
                 if (kWReg) {
 #pragma unroll
                     for (int h = 0; h < (kWReg ? NQ : 1); ++h) wr[h] = w_e[wslot * NQ + h];
                 }
 #pragma unroll
-                for (int gg = 0; gg < G; ++gg) nvis[gg] = __ldg(p.n_row + r0 + gg);
+                for (int gg = 0; gg < G; ++gg) nvis[gg] = ld_dep(p.n_row + r0 + gg);
                 gcur = cur.g;
             }
             if (since_flush == kFlushEvery) {
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                     if (!GATHER) {
                         vis = j < nvis[gg];
                     } else {
-                        int pos = (j < p.P) ? __ldg(p.pool + (int64_t)r * p.P + j) : -1;
+                        int pos = (j < p.P) ? ld_dep(p.pool + (int64_t)r * p.P + j) : -1;
                         vis = pos >= 0 && pos < nvis[gg];
                     }
                     const float scv = sc[hh][gg];
@@ -592,9 +592,9 @@ __global__ void __launch_bounds__(1024) prep_rows_kernel(
             int64_t n;
             if (q_pos0) {
                 const int b = r / T, t = r - b * T;
-                n = ((int64_t)__ldg(q_pos0 + b) + t + 1) / ratio;
+                n = ((int64_t)ld_dep(q_pos0 + b) + t + 1) / ratio;
             } else {
-                n = __ldg(n_vis0 + r);
+                n = ld_dep(n_vis0 + r);
             }
             if (n < 0 || n > cap) {
                 set_status(status, CSA2_DEV_BAD_COUNT);

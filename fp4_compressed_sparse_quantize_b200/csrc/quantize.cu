@@ -22,8 +22,8 @@
 namespace csa2 {
 
 __global__ void __launch_bounds__(256) quantize_kv_kernel(
-    const __nv_bfloat16* __restrict__ kv, int B, int n_new, int64_t ld_kv, int64_t bstride_kv,
-    const int32_t* __restrict__ dst_off, uint8_t* __restrict__ codes,
+    const __nv_bfloat16* kv, int B, int n_new, int64_t ld_kv, int64_t bstride_kv,
+    const int32_t* dst_off, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, int64_t cap, int32_t* status) {
     grid_dep_launch();
     grid_dep_wait();
@@ -32,14 +32,14 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(
     if (entry >= (int64_t)B * n_new) return;
     const int b = (int)(entry / n_new);
     const int i = (int)(entry - (int64_t)b * n_new);
-    const int64_t dst = (int64_t)__ldg(dst_off + b) + i;
+    const int64_t dst = (int64_t)ld_dep(dst_off + b) + i;
     if (dst < 0 || dst >= cap) {
         if (lane == 0) set_status(status, CSA2_DEV_BAD_INDEX);
         return;
     }
     const __nv_bfloat16* row = kv + (int64_t)b * bstride_kv + (int64_t)i * ld_kv + lane * 16;
-    uint4 v0 = __ldg(reinterpret_cast<const uint4*>(row));
-    uint4 v1 = __ldg(reinterpret_cast<const uint4*>(row) + 1);
+    uint4 v0 = ld_dep(reinterpret_cast<const uint4*>(row));
+    uint4 v1 = ld_dep(reinterpret_cast<const uint4*>(row) + 1);
     uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float x[16];
 #pragma unroll

@@ -57,7 +57,7 @@ struct TopkDev {
 
 __device__ __forceinline__ int64_t row_len(const TopkDev& a, int r) {
     if (a.ids) return a.ld;
-    const int64_t n = __ldg(a.n_row + r);
+    const int64_t n = ld_dep(a.n_row + r);
     return (n + a.n_row_div - 1) / a.n_row_div;
 }
 
@@ -65,15 +65,15 @@ __device__ __forceinline__ int64_t row_len(const TopkDev& a, int r) {
 __device__ __forceinline__ bool load_elem(const TopkDev& a, int r, int64_t i, uint64_t& comp) {
     uint32_t id = (uint32_t)i;
     if (a.ids) {
-        const int32_t v = __ldg(a.ids + (int64_t)r * a.ld + i);
-        if (v < 0 || v >= __ldg(a.id_limit + r)) return false;
+        const int32_t v = ld_dep(a.ids + (int64_t)r * a.ld + i);
+        if (v < 0 || v >= ld_dep(a.id_limit + r)) return false;
         id = (uint32_t)v;
     }
     uint32_t key;
     if (a.scores)
-        key = score_key(__ldg(a.scores + (int64_t)r * a.ld + i));
+        key = score_key(ld_dep(a.scores + (int64_t)r * a.ld + i));
     else
-        key = __ldg(a.keys + (int64_t)r * a.ld + i);
+        key = ld_dep(a.keys + (int64_t)r * a.ld + i);
     comp = ((uint64_t)key << 32) | (uint64_t)(~id);
     return true;
 }
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const int64_t i = start + (int64_t)k * kThreads + tid;
-                sv[k] = (i < end) ? __ldg(row + i) : 0.f;
+                sv[k] = (i < end) ? ld_dep(row + i) : 0.f;
             }
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
         __syncthreads();
         picks = sorted;
     }
-    const int32_t lim = a.expand8 ? __ldg(a.expand_limit + r) : 0;
+    const int32_t lim = a.expand8 ? ld_dep(a.expand_limit + r) : 0;
     int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
     auto emit = [&](uint32_t slot, int64_t id) {
         if (slot >= (uint32_t)K) return;
@@ -529,8 +529,8 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 }
 
 __device__ __forceinline__ uint32_t elem_key(const TopkDev& a, int r, int64_t i) {
-    return a.scores ? score_key(__ldg(a.scores + (int64_t)r * a.ld + i))
-                    : __ldg(a.keys + (int64_t)r * a.ld + i);
+    return a.scores ? score_key(ld_dep(a.scores + (int64_t)r * a.ld + i))
+                    : ld_dep(a.keys + (int64_t)r * a.ld + i);
 }
 
 // Shared-memory state of one row's selection.
@@ -645,7 +645,7 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
                 const uint32_t kk = elem_key(a, r, i);
                 uint32_t id = (uint32_t)i;
                 if (GATHER) {
-                    const int32_t v = __ldg(a.ids + (int64_t)r * a.ld + i);
+                    const int32_t v = ld_dep(a.ids + (int64_t)r * a.ld + i);
                     if (v < 0 || (uint32_t)v >= id_lim) return false;
                     id = (uint32_t)v;
                 }
@@ -711,7 +711,7 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
     __syncthreads();
 
     // ---- emit in ascending id order ----------------------------------------------------------
-    const int32_t lim = a.expand8 ? __ldg(a.expand_limit + r) : 0;
+    const int32_t lim = a.expand8 ? ld_dep(a.expand_limit + r) : 0;
     int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
     auto emit = [&](uint32_t slot, int64_t id) {
         if (slot >= (uint32_t)K) return;
@@ -787,7 +787,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
     grid_dep_wait();
     const int64_t n = row_len(a, r);
     const int K = a.K;
-    const uint32_t id_lim = GATHER ? (uint32_t)max(0, __ldg(a.id_limit + r)) : 0xFFFFFFFFu;
+    const uint32_t id_lim = GATHER ? (uint32_t)max(0, ld_dep(a.id_limit + r)) : 0xFFFFFFFFu;
     const bool use_bm = a.bitmap_words > 0 && crank == 0;
     const int nwords = a.bitmap_words;
     if (tid == 0) {
@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
             for (int k = 0; k < PER; ++k) {
                 const int64_t i = base + (int64_t)k * kRowThreads + tid;
                 key[k] = i < n ? elem_key(a, r, i) : 0u;
-                id[k] = i < n ? (uint32_t)__ldg(a.ids + (int64_t)r * a.ld + i) : 0xFFFFFFFFu;
+                id[k] = i < n ? (uint32_t)ld_dep(a.ids + (int64_t)r * a.ld + i) : 0xFFFFFFFFu;
             }
         };
         load(0);

@@ -380,6 +380,12 @@ CSA2_API int csa2_version(void);
  * can be timed with them. */
 CSA2_API csa2_status_t csa2_set_stage_events(void* ev_start, void* ev_stop);
 
+/* Benchmark hook: records `ev` (a cudaEvent_t passed as void*) on `stream`; during a stream
+ * capture the record becomes an external event node of the graph, so replays of the graph
+ * can be timed between two such events (a plain cudaEventRecord inside a capture only adds a
+ * dependency). Outside a capture it is an ordinary record. */
+CSA2_API csa2_status_t csa2_record_event(void* ev, void* stream);
+
 /* Test hook for the bounded waits: launches one block that waits on an mbarrier that is
  * never signalled, gives up after timeout_ns and sets CSA2_DEV_TIMEOUT in `status`
  * (device int32). Never faults or hangs. */
