@@ -85,6 +85,10 @@ WORKLOADS = {
     "prefill_b2_t4k_ctx128k_r2": Workload("prefill_b2_t4k_ctx128k_r2", "prefill", B=2,
                                           ctx=131072, ratio=2, H_I=64, idx_dtype="e4m3",
                                           K=512, H=64, T=4096),
+    # the same chunked prefill at one sequence and 1024 new tokens (profiler captures)
+    "prefill_b1_t1k_ctx128k_r2": Workload("prefill_b1_t1k_ctx128k_r2", "prefill", B=1,
+                                          ctx=131072, ratio=2, H_I=64, idx_dtype="e4m3",
+                                          K=512, H=64, T=1024),
 }
 
 

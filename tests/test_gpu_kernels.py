@@ -378,6 +378,38 @@ def test_prefill_indexer_and_attention_small():
             check_attention(out[b, t].cpu().numpy(), refs[b, t], f"b={b} t={t}")
 
 
+def test_prefill_indexer_back_to_back_calls():
+    """Consecutive prefill index calls in one process, each launched while the previous
+    kernel may still run: one workspace reused with a different tile prefix (other query
+    positions), then a freshly zeroed one. Every call must read the prefix its own prep
+    kernel wrote, not what the workspace held before."""
+    g = _gen(23)
+    B, T, H_I, K, r = 2, 256, 64, 256, 2
+    cap = 6000
+    k_I = _keys(B, cap, torch.float8_e4m3fn, g).to(dev)
+    q_I = torch.randn((B, T, H_I, 128), generator=g).to(torch.float8_e4m3fn)
+    w = torch.rand((B, T, H_I), generator=g)
+    q_Id, wd = q_I.to(dev), w.to(dev)
+    wsb = C().workspace_bytes(0, B, T, H_I, cap, K)
+    ws = C().new_workspace(wsb)
+    pick = [0, 1, 77, T - 1]
+    for q_pos0, fresh in (([4000, 900], False), ([11000, 2300], False), ([7000, 11700], True)):
+        if fresh:
+            ws = C().new_workspace(wsb)
+        idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+        qp = torch.tensor(q_pos0, dtype=torch.int32, device=dev)
+        C().index_score_topk("full", q_Id, wd, k_I, K, idx, ws, q_pos0=qp, ratio=r)
+        torch.cuda.synchronize()
+        assert C().read_device_status(ws) == 0, q_pos0
+        idx_np = idx.cpu().numpy()
+        for b in range(B):
+            for t in pick:
+                n = O.prefill_visible(q_pos0[b] + t, r)
+                s = O.index_scores(raw_qk(q_I[b, t]), w[b, t].numpy(),
+                                   raw_qk(k_I[b, :n].cpu()), O.E4M3)
+                check_topk(idx_np[b, t], s, np.arange(n), K, f"q_pos0={q_pos0} b={b} t={t}")
+
+
 # ---- bounded waits -------------------------------------------------------------------------
 
 def test_bounded_wait_reports_timeout():
