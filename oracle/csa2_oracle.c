@@ -31,6 +31,16 @@
  *  - prefill visibility and window rows: a token-by-token simulation of the compressor
  *    and of the window buffer, for ratios 1-3 and windows clipped at position 0; the
  *    composed prefill query with every visible entry selected against dense attention.
+ *  - bf16 encoder: torch's float32 -> bfloat16 cast on float32 inputs, hand-placed
+ *    midpoints and subnormals;
+ *  - compressor: r = 1 is the identity, equal logits give the mean, a dominant logit
+ *    (chosen per channel) selects its token, shifting a channel's logits or permuting
+ *    the tokens of a group changes nothing, every output lies inside its tokens' range,
+ *    and a hand-worked two-token case;
+ *  - projection: one-hot latents give W's columns, an identity W copies the first Di
+ *    channels, and random inputs match a float64 matrix-vector product.
+ *  The compressor and projection follow a READING (the pages lose the equation):
+ *  parity with the pages' own compressor is unpinned.
  *  The index-score FORMULA itself (sum over heads of w_h * ReLU(q_h . k)) is not
  *  printed on the pages: parity with the pages' own scorer is unpinned; the reading is
  *  stated where it is used.
@@ -413,6 +423,98 @@ ORC_EXPORT int orc_prefill_window_rows(int64_t q_pos0, int W, int64_t t, int32_t
         rows_out[n++] = (int32_t)(pos - first_buffer_pos);
     }
     return n;
+}
+
+/* ------------------------------------------------------------------------------ */
+/* KV compressor and indexer-K projection                                          */
+/* [AIS Methodology in Plain English]: the V4.1 compressor no longer uses           */
+/* overlapping source entries or absolute positional embeddings, and the indexer K  */
+/* is derived by projecting the main KV entries. [TLB "How did DeepSeek V4.1 reduce */
+/* the KV cache?"] names the compressed entries C_l and the compression weights     */
+/* Z_l but its equation is lost. Reading (the plainest one these support):          */
+/*  - entry j pools source tokens r*j .. r*j + r - 1 (no overlap, nothing added for  */
+/*    position): per channel d, a softmax over those r tokens of the logits Z[t][d]  */
+/*    weights their latents C[t][d];                                              */
+/*  - the pooled latent is rounded to bf16 (the input format of quantize-on-write),  */
+/*    quantized to FP4 as above, and projected by a [Di][D] matrix W to the indexer  */
+/*    key k[e] = sum_d W[e][d] * x[d], which is then stored in the indexer format.    */
+/* ------------------------------------------------------------------------------ */
+
+/* bf16 encoder: round to nearest, ties to even, onto the binary format with 8
+ * significant bits (exponent range of binary32; subnormal quantum 2^-133). Written from
+ * that definition: scale the magnitude so that its 8 significant bits are the integer
+ * part, round that to the nearest integer with ties to even, scale back. */
+static double round_half_even(double v) {
+    double f = floor(v);
+    double d = v - f;
+    if (d > 0.5) return f + 1.0;
+    if (d < 0.5) return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+ORC_EXPORT uint16_t orc_bf16_encode(double v) {
+    const int sign = signbit(v) ? 1 : 0;
+    double a = fabs(v);
+    double r;
+    if (a == 0.0) {
+        r = 0.0;
+    } else {
+        int e;
+        frexp(a, &e);                  /* a = f * 2^e, 0.5 <= f < 1 */
+        int q = e - 8;                 /* quantum of an 8-significant-bit number */
+        if (q < -133) q = -133;        /* subnormal range */
+        r = round_half_even(ldexp(a, -q));
+        r = ldexp(r, q);
+    }
+    float f = (float)r;                /* exact: r has at most 8 significant bits */
+    if (sign) f = -f;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+ORC_EXPORT void orc_bf16_encode_many(const double* v, int64_t n, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_encode(v[i]);
+}
+
+/* Pooled latents of n_entries entries of D channels. Source token t of the entry group
+ * has latent row C + t*ld and logit row Z + t*ld (bf16 bit patterns); entry j reads tokens
+ * r*j .. r*j + r - 1. out[j*D + d] = sum_t softmax_t(Z[t][d]) * C[t][d], in double (the
+ * largest logit is subtracted before exp, which leaves the softmax unchanged). */
+ORC_EXPORT void orc_compress_entries(const uint16_t* Cs, const uint16_t* Zs, int64_t n_entries,
+                                     int r, int D, int64_t ld, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n_entries; ++j) {
+        for (int d = 0; d < D; ++d) {
+            double zmax = -INFINITY;
+            for (int t = 0; t < r; ++t) {
+                double z = orc_bf16_value(Zs[(j * r + t) * ld + d]);
+                if (z > zmax) zmax = z;
+            }
+            double den = 0.0, num = 0.0;
+            for (int t = 0; t < r; ++t) {
+                double a = exp(orc_bf16_value(Zs[(j * r + t) * ld + d]) - zmax);
+                den += a;
+                num += a * orc_bf16_value(Cs[(j * r + t) * ld + d]);
+            }
+            out[j * D + d] = num / den;
+        }
+    }
+}
+
+/* Indexer keys of n entries: out[i*Di + e] = sum_d W[e][d] * x[i*D + d], W as bf16 bit
+ * patterns [Di][D] (row e = the weights of key channel e), in double. */
+ORC_EXPORT void orc_project_keys(const double* x, int64_t n, int D, const uint16_t* W, int Di,
+                                 double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        for (int e = 0; e < Di; ++e) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += orc_bf16_value(W[(int64_t)e * D + d]) * x[i * D + d];
+            out[i * Di + e] = acc;
+        }
+    }
 }
 
 /* ------------------------------------------------------------------------------ */

@@ -70,6 +70,14 @@ def lib():
         L.orc_prefill_visible.argtypes = [i64, C.c_int]
         L.orc_prefill_window_rows.restype = C.c_int
         L.orc_prefill_window_rows.argtypes = [i64, C.c_int, i64, P]
+        L.orc_bf16_encode.restype = u16
+        L.orc_bf16_encode.argtypes = [d]
+        L.orc_bf16_encode_many.restype = None
+        L.orc_bf16_encode_many.argtypes = [P, i64, P]
+        L.orc_compress_entries.restype = None
+        L.orc_compress_entries.argtypes = [P, P, i64, C.c_int, C.c_int, i64, P]
+        L.orc_project_keys.restype = None
+        L.orc_project_keys.argtypes = [P, i64, C.c_int, P, C.c_int, P]
         _lib = L
     return _lib
 
@@ -282,6 +290,56 @@ def prefill_query(qi_raw, w, k_raw, dtype, kv_bits, q_bits, swa_buf, q_pos0, t, 
     win = e4m3_array_to_f64(_c(swa_buf, np.uint8).reshape(-1, D)[prefill_window_rows(q_pos0, W, t)])
     q = bf16_array_to_f64(q_bits).reshape(-1, D)
     return idx, attention(q, np.concatenate([main, win.reshape(-1, D)], axis=0), tau)
+
+
+# ---- KV compressor and indexer-K projection ----------------------------------------------
+
+def bf16_encode(v):
+    """bf16 bit pattern of v (round to nearest, ties to even)."""
+    return int(lib().orc_bf16_encode(float(v)))
+
+
+def bf16_encode_many(v):
+    v = _c(v, np.float64)
+    out = np.zeros(v.shape, np.uint16)
+    lib().orc_bf16_encode_many(_p(v), v.size, _p(out))
+    return out
+
+
+def compress_entries(c_bits, z_bits, r):
+    """c_bits, z_bits: uint16 [r * n, D] bf16 patterns of one sequence's source tokens.
+    Returns float64 [n, D]: per channel, the softmax over each entry's r tokens of the
+    logits weighting their latents."""
+    c_bits = _c(c_bits, np.uint16)
+    z_bits = _c(z_bits, np.uint16)
+    assert c_bits.shape == z_bits.shape and c_bits.shape[0] % r == 0
+    n, D = c_bits.shape[0] // r, c_bits.shape[1]
+    out = np.zeros((n, D), np.float64)
+    lib().orc_compress_entries(_p(c_bits), _p(z_bits), n, int(r), D, D, _p(out))
+    return out
+
+
+def project_keys(x, w_bits):
+    """x: float64 [n, D] entry latents; w_bits: uint16 [Di, D] bf16 patterns.
+    Returns float64 [n, Di] = x @ W^T."""
+    x = _c(x, np.float64)
+    w_bits = _c(w_bits, np.uint16)
+    Di, D = w_bits.shape
+    out = np.zeros((x.shape[0], Di), np.float64)
+    lib().orc_project_keys(_p(x), x.shape[0], D, _p(w_bits), Di, _p(out))
+    return out
+
+
+def compress_write(c_bits, z_bits, r, w_bits, key_dtype):
+    """The whole write of one sequence's new entries: pooled latents rounded to bf16,
+    their FP4 codes and scales, and the indexer keys (E4M3 codes or bf16 patterns).
+    Returns (latent_bits uint16 [n, D], codes, scales, key_raw, key_exact float64)."""
+    lat_bits = bf16_encode_many(compress_entries(c_bits, z_bits, r))
+    codes, scales = quantize_entries(lat_bits, D=lat_bits.shape[1])
+    k = project_keys(bf16_array_to_f64(lat_bits), w_bits)
+    key_raw = (e4m3_encode_many(k.ravel()).reshape(k.shape) if key_dtype == E4M3
+               else bf16_encode_many(k))
+    return lat_bits, codes, scales, key_raw, k
 
 
 def bytes_per_token(D=512, indexer_entry_bytes=68.0, enc_full=3, enc_ratio=2, dec_full=1,
