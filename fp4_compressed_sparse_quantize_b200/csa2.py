@@ -27,7 +27,7 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
            "csa2_cp_pool_expand", "csa2_cache_record_bytes", "csa2_cache_export",
            "csa2_cache_import", "csa2_cp_local_idx", "csa2_sparse_attn_decode_partial",
-           "csa2_attn_merge_partials", "csa2_record_event")
+           "csa2_attn_merge_partials", "csa2_record_event", "csa2_compress_kv")
 
 
 class Csa2Error(RuntimeError):
@@ -49,6 +49,8 @@ def lib():
         L = C.CDLL(LIB_PATH)
         P, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
         L.csa2_quantize_kv.argtypes = [P, i32, i32, i64, i64, P, P, P, i64, P, P]
+        L.csa2_compress_kv.argtypes = [i32, i32, i32, P, P, i64, i64, P, i32, P, P, P, P, i64,
+                                       P, P, P]
         L.csa2_index_score_topk.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P, i32, P,
                                             i32, P, i32, P, i32, P, P, P, sz, P]
         L.csa2_sparse_attn_decode.argtypes = [i32, i32, i32, P, P, P, i64, P, i32, P, i32, P,
@@ -185,6 +187,35 @@ def quantize_kv(kv, dst_off, codes, scales, status=None, stream=None):
     st = lib().csa2_quantize_kv(_p(kv), B, n_new, kv.stride(1), kv.stride(0), _p(dst_off),
                                 _p(codes), _p(scales), cap, _p(status), _stream(stream))
     _check(st, "csa2_quantize_kv")
+
+
+def compress_kv(C, Z, ratio, w_proj, dst_off, codes, scales, k_I, latent_out=None, status=None,
+                stream=None):
+    """C, Z bf16 [B, ratio * n_new, 512] (unit channel stride; token and batch strides may
+    be larger): source-token latents and compression logits. w_proj bf16 [128, 512];
+    dst_off int32 [B]; codes uint8 [B, cap, 256]; scales uint8 [B, cap, 32]; k_I
+    [B, cap, 128] E4M3 or bf16; latent_out nullable bf16 [B, n_new, 512]."""
+    for t, nm in ((C, "C"), (Z, "Z")):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1 or not t.is_cuda:
+            raise Csa2Error(ERR_ARG, f"{nm} must be a CUDA bf16 tensor with unit channel stride")
+    if C.shape != Z.shape or C.stride() != Z.stride():
+        raise Csa2Error(ERR_ARG, "C and Z must have the same shape and strides")
+    _need(w_proj, torch.bfloat16, "w_proj")
+    _need(dst_off, torch.int32, "dst_off")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    _need(latent_out, torch.bfloat16, "latent_out")
+    if k_I.dtype not in DTYPE:
+        raise Csa2Error(ERR_ARG, "k_I must be bf16 or float8_e4m3fn")
+    _need(k_I, k_I.dtype, "k_I")
+    B, n_tok, D = C.shape
+    if n_tok % ratio:
+        raise Csa2Error(ERR_ARG, "the token count must be a multiple of the ratio")
+    st = lib().csa2_compress_kv(B, n_tok // ratio, int(ratio), _p(C), _p(Z), C.stride(1),
+                                C.stride(0), _p(w_proj), DTYPE[k_I.dtype], _p(dst_off),
+                                _p(codes), _p(scales), _p(k_I), codes.shape[1], _p(latent_out),
+                                _p(status), _stream(stream))
+    _check(st, "csa2_compress_kv")
 
 
 def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None, ratio=1,

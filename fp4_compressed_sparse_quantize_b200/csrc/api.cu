@@ -10,6 +10,20 @@
 
 namespace csa2 {
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
 int device_sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -201,6 +215,42 @@ csa2_status_t csa2_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
     if ((int64_t)B * n_new > (int64_t)1 << 40) return CSA2_ERR_ARG;
     return cuda_status(launch_quantize_kv(kv, B, n_new, ld_kv, bstride_kv, dst_off, codes, scales,
                                           cap, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, const void* Z, int64_t ld,
+                               int64_t bstride, const void* w_proj, csa2_dtype_t key_dtype,
+                               const int32_t* dst_off, uint8_t* codes, uint8_t* scales,
+                               void* k_I, int64_t cap, void* latent_out, int32_t* status,
+                               void* stream) {
+    if (B < 0 || n_new < 0 || cap < 1 || r < 1 || r > 64) return CSA2_ERR_ARG;
+    if ((int64_t)B * n_new == 0) return CSA2_OK;
+    if (key_dtype != CSA2_DTYPE_E4M3 && key_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_ARG;
+    if (!C || !Z || !w_proj || !dst_off || !codes || !scales || !k_I) return CSA2_ERR_ARG;
+    if (ld < CSA2_D_MAIN || ld % 8 != 0 || bstride % 8 != 0 || bstride < 0) return CSA2_ERR_ARG;
+    if (B > 1 && bstride < ((int64_t)r * n_new - 1) * ld + CSA2_D_MAIN) return CSA2_ERR_ARG;
+    if (!aligned16(C) || !aligned16(Z) || !aligned16(w_proj) || !aligned16(codes) ||
+        !aligned16(scales) || !aligned16(k_I) || !aligned16(latent_out))
+        return CSA2_ERR_ARG;
+    if ((int64_t)B * n_new > (int64_t)1 << 31) return CSA2_ERR_ARG;
+    CompressLaunch l;
+    memset(&l, 0, sizeof l);
+    l.B = B;
+    l.n_new = n_new;
+    l.r = r;
+    l.ld = ld;
+    l.bstride = bstride;
+    l.C = C;
+    l.Z = Z;
+    l.w_proj = w_proj;
+    l.key_bf16 = key_dtype == CSA2_DTYPE_BF16;
+    l.dst_off = dst_off;
+    l.codes = codes;
+    l.scales = scales;
+    l.keys = k_I;
+    l.cap = cap;
+    l.latent = latent_out;
+    l.status = status;
+    return cuda_status(launch_compress_kv(l, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int csa2_sparse_attn_decode_launches(int B, int K, int W) {

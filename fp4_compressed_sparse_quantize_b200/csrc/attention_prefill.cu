@@ -708,26 +708,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpMma && !flags[2]) tmem_dealloc(tmem, 512);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 }  // namespace
 
 // Prefill attention of Q = B * T tokens (l.prefill): one persistent CTA per SM.
 cudaError_t launch_attention_prefill(const AttnLaunch& l, cudaStream_t st) {
     if (l.Q < 1) return cudaSuccess;
-    auto enc = encoder();
+    auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorInvalidValue;
     CUtensorMap mq;
     memset(&mq, 0, sizeof mq);

@@ -1039,23 +1039,9 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     if (warp == 0 && !mma_stuck) tmem_dealloc(tmem, 512);
 }
 
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 // [rows][512] fp16 matrix, box = 64 channels x box_rows, 128-byte swizzle
 static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
-    auto enc = encode_fn();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(kD * 2)};
@@ -1068,7 +1054,7 @@ static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int bo
 
 // [blocks][H][512] fp32 output or partial output, box = 128 channels x H heads x 1 block
 static bool out_map(CUtensorMap* m, void* base, int H, int64_t blocks) {
-    auto enc = encode_fn();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)blocks};
     cuuint64_t strides[2] = {(cuuint64_t)(kD * 4), (cuuint64_t)H * kD * 4};
@@ -1081,7 +1067,7 @@ static bool out_map(CUtensorMap* m, void* base, int H, int64_t blocks) {
 
 // [blocks][H][512] fp32, box = 32 channels x H heads x 1 block, 128-byte swizzle
 static bool out_map_sw(CUtensorMap* m, void* base, int H, int64_t blocks) {
-    auto enc = encode_fn();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)blocks};
     cuuint64_t strides[2] = {(cuuint64_t)(kD * 4), (cuuint64_t)H * kD * 4};

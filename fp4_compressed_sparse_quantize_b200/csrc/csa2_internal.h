@@ -1,6 +1,8 @@
 // Internal launch interfaces between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -8,6 +10,9 @@
 #include <utility>
 
 namespace csa2 {
+
+// The driver's tensor-map encoder, looked up once per process (null if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Launch with programmatic stream serialisation (see grid_dep_wait / grid_dep_launch).
 template <typename... KArgs, typename... Args>
@@ -52,6 +57,25 @@ cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
                                int64_t bstride_kv, const int32_t* dst_off, uint8_t* codes,
                                uint8_t* scales, int64_t cap, int32_t* status,
                                cudaStream_t stream);
+
+// Compressor + indexer-K projection + FP4 write (csa2_compress_kv).
+struct CompressLaunch {
+    int B, n_new, r;
+    int64_t ld, bstride;
+    const void* C;
+    const void* Z;
+    const void* w_proj;
+    int key_bf16;
+    const int32_t* dst_off;
+    uint8_t* codes;
+    uint8_t* scales;
+    void* keys;
+    int64_t cap;
+    void* latent;
+    int32_t* status;
+};
+
+cudaError_t launch_compress_kv(const CompressLaunch& l, cudaStream_t st);
 
 // Up to four workspace buffers that the prep kernel clears (16-byte units).
 struct ZeroList {

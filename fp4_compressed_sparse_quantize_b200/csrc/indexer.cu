@@ -640,23 +640,9 @@ __global__ void __launch_bounds__(1024) prep_rows_kernel(
 
 // ---- host side -------------------------------------------------------------------------------
 
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 // 2-D map over a [rows][row_bytes] byte matrix, box = 128 bytes x box_rows, 128B swizzle.
 static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int esz, int box_rows) {
-    auto enc = get_encode();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     const CUtensorMapDataType dt =
         esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;

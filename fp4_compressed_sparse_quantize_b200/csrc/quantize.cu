@@ -10,14 +10,10 @@
 // coalesced sweep); stores are 8 code bytes and 1 scale byte per lane (256 + 32 B per
 // warp, contiguous). The work is trivially HBM-bound (1 KiB in, 288 B out per entry).
 //
-// Rounding: the scale is E4M3(amax / 6) and each magnitude is E2M1(|x| / s), both with
-// round-to-nearest-even and saturation (cvt.rn.satfinite), where the quotients are IEEE
-// fp32 divisions. Neither quotient can land on a rounding midpoint unless the exact
-// quotient does: the numerator has 8 significant bits and the divisor (6, or an E4M3
-// value with at most 4) leaves a non-dyadic quotient far from every dyadic midpoint, and
-// a dyadic quotient is exact in fp32. A reciprocal-multiply would not have that property.
+// Rounding: fp4_quantize_block16 (fp4_block.cuh).
 #include "csa2_common.cuh"
 #include "csa2_internal.h"
+#include "fp4_block.cuh"
 
 namespace csa2 {
 
@@ -47,40 +43,11 @@ __global__ void __launch_bounds__(256) quantize_kv_kernel(
         x[2 * k] = __uint_as_float(w[k] << 16);
         x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
-
-    // scale code: E4M3(amax / 6), RNE, saturating
-    const float q = __fdiv_rn(amax, 6.0f);
-    uint16_t sc2;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sc2) : "f"(0.0f), "f"(q));
-    const uint8_t sc = (uint8_t)(sc2 & 0xFF);
-    const float s = e4m3_to_float(sc);
-
-    uint32_t packed_lo = 0, packed_hi = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        // channel 2k -> low nibble, 2k+1 -> high nibble
-        const float a = (s > 0.f) ? __fdiv_rn(fabsf(x[2 * k]), s) : 0.f;
-        const float c = (s > 0.f) ? __fdiv_rn(fabsf(x[2 * k + 1]), s) : 0.f;
-        uint16_t byte;
-        asm("{\n\t.reg .b8 t;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-            "cvt.u16.u8 %0, t;\n\t}"
-            : "=h"(byte)
-            : "f"(c), "f"(a));
-        uint32_t bb = byte & 0x77u;  // magnitudes only
-        bb |= (__float_as_uint(x[2 * k]) >> 31) << 3;
-        bb |= (__float_as_uint(x[2 * k + 1]) >> 31) << 7;
-        if (k < 4)
-            packed_lo |= bb << (8 * k);
-        else
-            packed_hi |= bb << (8 * (k - 4));
-    }
+    uint2 packed;
+    uint8_t sc;
+    fp4_quantize_block16(x, packed, sc);
     const int64_t e = (int64_t)b * cap + dst;
-    reinterpret_cast<uint2*>(codes + e * CSA2_ENTRY_CODE_BYTES)[lane] =
-        make_uint2(packed_lo, packed_hi);
+    reinterpret_cast<uint2*>(codes + e * CSA2_ENTRY_CODE_BYTES)[lane] = packed;
     scales[e * CSA2_ENTRY_SCALE_BYTES + lane] = sc;
 }
 

@@ -120,6 +120,43 @@ CSA2_API csa2_status_t csa2_quantize_kv(const void* kv, int B, int n_new, int64_
                                uint8_t* scales, int64_t cap, int32_t* status, void* stream);
 
 /*
+ * csa2_compress_kv — KV compressor and indexer-K projection, fused with FP4
+ * quantize-on-write: n_new new entries per sequence from r*n_new source tokens.
+ * [AIS Methodology in Plain English]: no overlapping source entries and no absolute
+ * positional embedding in the compressor; the indexer K is a projection of the main KV
+ * entries. [TLB How did DeepSeek V4.1 reduce the KV cache?] names the compressed entries
+ * (C_l) and compression weights (Z_l); the equation itself is lost, so this is a reading:
+ *   entry j pools tokens r*j .. r*j+r-1; per channel d
+ *     x[j][d] = bf16_RNE( sum_t softmax_t(Z[t][d]) * C[t][d] )   (fp32 arithmetic)
+ *   codes, scales = csa2_quantize_kv's FP4 encoding of x[j], at entry dst_off[b] + j;
+ *   k_I[j][e] = sum_d w_proj[e][d] * x[j][d]  (tensor cores, fp32 accumulation),
+ *     stored as E4M3 (RNE, saturating at 448) or bf16 (RNE).
+ *
+ *   C, Z     bf16 latents and compression logits of the source tokens: element
+ *            (b, token i, channel c) at C[b*bstride + i*ld + c] (same for Z; token i of
+ *            sequence b is source token r*j + t of entry j). ld >= 512, ld and bstride
+ *            multiples of 8; 16-byte aligned; finite values.
+ *   r        tokens per entry, 1..64.
+ *   w_proj   bf16 [128][512], row e = the weights of key channel e; 16-byte aligned.
+ *   key_dtype  CSA2_DTYPE_E4M3 or CSA2_DTYPE_BF16: the storage type of k_I.
+ *   dst_off  int32 [B]: entry index of sequence b's first new entry.
+ *   codes, scales  the FP4 cache as in csa2_quantize_kv.
+ *   k_I      [B][cap][128] in key_dtype: the indexer-key cache.
+ *   latent_out  nullable bf16 [B][n_new][512]: the pooled bf16 latents x.
+ *   status   nullable int32 device word: CSA2_DEV_BAD_INDEX for an entry outside
+ *            [0, cap) (that entry is skipped), CSA2_DEV_TIMEOUT for a bounded wait that
+ *            gave up.
+ * The caller owns every buffer; nothing is allocated. Host-side validation returns
+ * CSA2_ERR_ARG before anything is launched.
+ */
+CSA2_API csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, const void* Z,
+                                        int64_t ld, int64_t bstride, const void* w_proj,
+                                        csa2_dtype_t key_dtype, const int32_t* dst_off,
+                                        uint8_t* codes, uint8_t* scales, void* k_I,
+                                        int64_t cap, void* latent_out, int32_t* status,
+                                        void* stream);
+
+/*
  * csa2_index_score_topk — indexer scoring + exact Top-K selection, per layer mode.
  * [AIS Methodology]: each layer has its own indexer query; Full layers score, Reindex
  * layers rescore the latest Full layer's keys, Reuse layers skip indexing; the first
