@@ -39,6 +39,11 @@
  *    and a hand-worked two-token case;
  *  - projection: one-hot latents give W's columns, an identity W copies the first Di
  *    channels, and random inputs match a float64 matrix-vector product.
+ *  - compact 68-byte keys: keys whose scale is a power of two round-trip exactly,
+ *    the largest magnitude takes code 6, negation flips only sign bits, midpoints
+ *    round to even, an independent nearest-grid search agrees on random keys, the
+ *    68-byte record gives 890 bytes per token, and scores against compact keys equal
+ *    the bf16-key scores of the same values;
  *  The compressor and projection follow a READING (the pages lose the equation):
  *  parity with the pages' own compressor is unpinned.
  *  The index-score FORMULA itself (sum over heads of w_h * ReLU(q_h . k)) is not
@@ -264,6 +269,85 @@ ORC_EXPORT void orc_index_scores(int H, int Di, int dtype, const void* q /*[H,Di
         int64_t r = rows ? rows[j] : j;
         double kd[1024];
         for (int d = 0; d < Di; ++d) kd[d] = load_elem(k, dtype, r * Di + d);
+        double acc = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double dot = 0.0;
+            for (int d = 0; d < Di; ++d) dot += qd[(int64_t)h * Di + d] * kd[d];
+            double relu = dot > 0.0 ? dot : 0.0;
+            acc += (double)w[h] * relu;
+        }
+        s[j] = acc + 0.0;
+    }
+    free(qd);
+}
+
+/* ------------------------------------------------------------------------------ */
+/* Compact indexer keys: 68 bytes per entry                                        */
+/* [AIS Main Findings] and [TLB "How is DeepSeek V4.1 Flash different"] (Figure 1): */
+/* 890 bytes of global KV per token. With 2.5 stored entry-sets per token (byte     */
+/* accounting below) and 288-byte FP4 main entries, 890 leaves 68 bytes for an      */
+/* indexer key. Reading (the pages give no key format): a 128-channel key as E2M1   */
+/* codes (64 bytes, channel 2k in the low nibble of byte k) times one fp32 scale    */
+/* (4 bytes) per key, scale = amax / 6 so that the largest magnitude maps to 6.      */
+/* The quantizer's decisions are taken in IEEE fp32, the precision of the key       */
+/* format's own scale: s = fl32(amax / 6), code = E2M1_RNE_sat(fl32(|x| / s)), the   */
+/* sign bit copied from x; s == 0 gives zero magnitudes.                            */
+/* ------------------------------------------------------------------------------ */
+
+ORC_EXPORT void orc_quantize_key_fp4(const uint16_t* k /*bf16 [Di]*/, int Di, uint8_t* codes,
+                                     float* scale) {
+    float amax = 0.0f;
+    for (int d = 0; d < Di; ++d) {
+        float a = fabsf((float)orc_bf16_value(k[d]));
+        if (a > amax) amax = a;
+    }
+    volatile float six = 6.0f;
+    float sc = amax / six;                       /* one IEEE fp32 division */
+    for (int d = 0; d < Di; d += 2) {
+        unsigned nib[2];
+        for (int t = 0; t < 2; ++t) {
+            float x = (float)orc_bf16_value(k[d + t]);
+            unsigned sign = signbit(x) ? 8u : 0u;
+            unsigned mag = 0;
+            if (sc > 0.0f) {
+                float qv = fabsf(x) / sc;        /* one IEEE fp32 division */
+                mag = orc_e2m1_encode((double)qv) & 7u;
+            }
+            nib[t] = sign | mag;
+        }
+        codes[d / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+    }
+    *scale = sc;
+}
+
+ORC_EXPORT void orc_quantize_keys_fp4(const uint16_t* k, int64_t n, int Di, uint8_t* codes,
+                                      float* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        orc_quantize_key_fp4(k + i * Di, Di, codes + i * (Di / 2), &scales[i]);
+}
+
+/* Value of channel d of a compact key: E2M1 code value times the key's scale. */
+ORC_EXPORT void orc_dequant_key_fp4(const uint8_t* codes, float scale, int Di, double* x) {
+    for (int d = 0; d < Di; ++d) {
+        uint8_t byte = codes[d / 2];
+        unsigned nib = (d % 2 == 0) ? (byte & 15u) : (byte >> 4);
+        x[d] = orc_e2m1_value(nib) * (double)scale;
+    }
+}
+
+/* Index scores (the formula above) against compact keys, q as E4M3 [H][Di]. */
+ORC_EXPORT void orc_index_scores_fp4key(int H, int Di, const uint8_t* q, const float* w,
+                                        const uint8_t* codes /*[*][Di/2]*/,
+                                        const float* scales /*[*]*/, const int32_t* rows,
+                                        int64_t n, double* s) {
+    double* qd = (double*)malloc(sizeof(double) * (size_t)H * Di);
+    for (int64_t i = 0; i < (int64_t)H * Di; ++i) qd[i] = orc_e4m3_value(q[i]);
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; ++j) {
+        int64_t r = rows ? rows[j] : j;
+        double kd[1024];
+        orc_dequant_key_fp4(codes + r * (Di / 2), scales[r], Di, kd);
         double acc = 0.0;
         for (int h = 0; h < H; ++h) {
             double dot = 0.0;

@@ -78,6 +78,12 @@ def lib():
         L.orc_compress_entries.argtypes = [P, P, i64, C.c_int, C.c_int, i64, P]
         L.orc_project_keys.restype = None
         L.orc_project_keys.argtypes = [P, i64, C.c_int, P, C.c_int, P]
+        L.orc_quantize_keys_fp4.restype = None
+        L.orc_quantize_keys_fp4.argtypes = [P, i64, C.c_int, P, P]
+        L.orc_dequant_key_fp4.restype = None
+        L.orc_dequant_key_fp4.argtypes = [P, C.c_float, C.c_int, P]
+        L.orc_index_scores_fp4key.restype = None
+        L.orc_index_scores_fp4key.argtypes = [C.c_int, C.c_int, P, P, P, P, P, i64, P]
         _lib = L
     return _lib
 
@@ -340,6 +346,47 @@ def compress_write(c_bits, z_bits, r, w_bits, key_dtype):
     key_raw = (e4m3_encode_many(k.ravel()).reshape(k.shape) if key_dtype == E4M3
                else bf16_encode_many(k))
     return lat_bits, codes, scales, key_raw, k
+
+
+# ---- compact 68-byte indexer keys -------------------------------------------------------
+
+def quantize_keys_fp4(k_bits):
+    """k_bits: uint16 [n, Di] bf16 patterns -> (codes uint8 [n, Di/2], scales float32 [n])."""
+    k_bits = _c(k_bits, np.uint16)
+    n, Di = k_bits.shape
+    codes = np.zeros((n, Di // 2), np.uint8)
+    scales = np.zeros(n, np.float32)
+    lib().orc_quantize_keys_fp4(_p(k_bits), n, Di, _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequant_keys_fp4(codes, scales):
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.float32)
+    n, half = codes.shape
+    out = np.zeros((n, 2 * half), np.float64)
+    for i in range(n):
+        row = out[i]
+        lib().orc_dequant_key_fp4(_p(codes[i]), float(scales[i]), 2 * half, _p(row))
+    return out
+
+
+def index_scores_fp4key(q, w, codes, scales, rows=None):
+    """q: uint8 [H, Di] E4M3; w: float32 [H]; codes uint8 [n_all, Di/2]; scales float32
+    [n_all]. Returns float64 scores for rows (or all rows)."""
+    q = _c(q, np.uint8)
+    w = _c(w, np.float32)
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.float32)
+    H, Di = q.shape
+    if rows is None:
+        n, r = codes.shape[0], None
+    else:
+        r = _c(rows, np.int32)
+        n = r.shape[0]
+    s = np.zeros(n, np.float64)
+    lib().orc_index_scores_fp4key(H, Di, _p(q), _p(w), _p(codes), _p(scales), _p(r), n, _p(s))
+    return s
 
 
 def bytes_per_token(D=512, indexer_entry_bytes=68.0, enc_full=3, enc_ratio=2, dec_full=1,
