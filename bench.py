@@ -519,6 +519,52 @@ def measure_prefill(w, seed, steps, warmup, dev):
             "clocks": clk, "device_status": st, "steps": steps}
 
 
+COMPRESS_CASES = (("compress_prefill_b2_n2048_r2", 2, 2048, 2, 67584),
+                  ("compress_decode_b32_n1_r2", 32, 1, 2, 32768))
+
+
+def measure_compress(name, B, n_new, r, cap, seed, steps, dev):
+    """Device time of csa2_compress_kv (compressor + indexer-K projection + FP4 write) on
+    synthetic source tokens, L2 flushed between launches (outside the events). Roofline:
+    HBM bytes = the source latents and logits read + the FP4 entry (288 B) and E4M3 key
+    (128 B) written per entry + the projection matrix (128 KiB) once."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    n_tok = r * n_new
+    Cs = torch.randn((B, n_tok, 512), generator=g).to(torch.bfloat16).to(dev)
+    Zs = (torch.randn((B, n_tok, 512), generator=g) * 2).to(torch.bfloat16).to(dev)
+    W = (torch.randn((128, 512), generator=g) * 0.06).to(torch.bfloat16).to(dev)
+    dst = torch.full((B,), cap - n_new, dtype=torch.int32, device=dev)
+    codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
+    keys = torch.zeros((B, cap, 128), dtype=torch.float8_e4m3fn, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        csa2.compress_kv(Cs, Zs, r, W, dst, codes, scales, keys, status=st)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for k in range(steps):
+        flush_l2(flush, k)
+        ev[k][0].record(stream)
+        csa2.compress_kv(Cs, Zs, r, W, dst, codes, scales, keys, status=st)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    entries = B * n_new
+    nbytes = entries * (2 * r * 512 * 2 + 288 + 128) + 128 * 512 * 2
+    peak, _src = peaks()
+    out = {"kernel": "csa2 compressor + indexer-K projection (tcgen05) + FP4 write",
+           "entries": entries, "ratio": r, "bound": "hbm", "bytes_per_launch": nbytes,
+           "avg_launch_ms": ms, "achieved": nbytes / (ms / 1e3) / 1e9, "peak": peak,
+           "unit": "GB/s", "frac": nbytes / (ms / 1e3) / 1e9 / peak,
+           "device_status": int(st.item())}
+    del Cs, Zs, codes, scales, keys, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def prefill_main(args, w, dev, rank, world):
     m = measure_prefill(w, rank_seed(args.seed, rank), args.steps, args.warmup, dev)
     line = {
@@ -788,6 +834,9 @@ def main():
                 extra[name] = extra_decode(name, args, dev, local)
         pw = synth.WORKLOADS[EXTRA_PREFILL]
         extra[EXTRA_PREFILL] = measure_prefill(pw, args.seed, args.extra_steps, 3, dev)
+        for name, B, n_new, r, cap in COMPRESS_CASES:
+            extra[name] = measure_compress(name, B, n_new, r, cap, args.seed, args.extra_steps,
+                                           dev)
         state = state_keep
 
     cpu = None

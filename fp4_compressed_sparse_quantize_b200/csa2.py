@@ -27,7 +27,8 @@ EXPORTS = ("csa2_quantize_kv", "csa2_index_score_topk", "csa2_sparse_attn_decode
            "csa2_cp_topk_candidates", "csa2_cp_pool_candidates", "csa2_cp_merge",
            "csa2_cp_pool_expand", "csa2_cache_record_bytes", "csa2_cache_export",
            "csa2_cache_import", "csa2_cp_local_idx", "csa2_sparse_attn_decode_partial",
-           "csa2_attn_merge_partials", "csa2_record_event", "csa2_compress_kv")
+           "csa2_attn_merge_partials", "csa2_record_event", "csa2_compress_kv",
+           "csa2_quantize_keys_fp4")
 
 
 class Csa2Error(RuntimeError):
@@ -49,6 +50,7 @@ def lib():
         L = C.CDLL(LIB_PATH)
         P, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
         L.csa2_quantize_kv.argtypes = [P, i32, i32, i64, i64, P, P, P, i64, P, P]
+        L.csa2_quantize_keys_fp4.argtypes = [P, i32, i32, i64, i64, P, P, i64, P, P]
         L.csa2_compress_kv.argtypes = [i32, i32, i32, P, P, i64, i64, P, i32, P, P, P, P, i64,
                                        P, P, P]
         L.csa2_index_score_topk.argtypes = [i32, i32, i32, i32, i32, P, P, P, i64, P, i32, P,
@@ -218,18 +220,57 @@ def compress_kv(C, Z, ratio, w_proj, dst_off, codes, scales, k_I, latent_out=Non
     _check(st, "csa2_compress_kv")
 
 
-def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None, ratio=1,
-                     pool_in=None, pool_out=None, pool_blocks=0, scores_out=None, stream=None):
-    """q_I [B, T, H_I, 128] (bf16 or E4M3), w fp32 [B, T, H_I], k_I [B, cap, 128] of the same
-    dtype, idx_out int32 [B, T, K]. Decode: n_vis0 int32 [B]. Prefill: q_pos0 int32 [B] and
-    ratio. Reindex: pool_in int32 [B, T, P]. Full with a pool: pool_out int32
-    [B, T, pool_blocks * 8]."""
-    m = MODE[mode] if isinstance(mode, str) else int(mode)
-    B, T, H_I, Di = q_I.shape
+DTYPE_E4M3_FP4KEY = 2
+FP4KEY_CODE_BYTES = 64
+
+
+class Fp4Keys:
+    """Compact 68-byte indexer keys of B sequences x cap entries: one device buffer holding
+    the E2M1 code plane [B, cap, 64] and then the fp32 scale plane [B, cap] (the layout of
+    CSA2_DTYPE_E4M3_FP4KEY)."""
+
+    def __init__(self, B, cap, device="cuda"):
+        self.B, self.cap = int(B), int(cap)
+        n = self.B * self.cap
+        self.buf = torch.zeros(n * (FP4KEY_CODE_BYTES + 4), dtype=torch.uint8, device=device)
+        self.codes = self.buf[:n * FP4KEY_CODE_BYTES].view(self.B, self.cap, FP4KEY_CODE_BYTES)
+        self.scales = self.buf[n * FP4KEY_CODE_BYTES:].view(torch.float32).view(self.B, self.cap)
+
+
+def quantize_keys_fp4(k, dst_off, keys, status=None, stream=None):
+    """k bf16 [B, n_new, 128] (unit channel stride); dst_off int32 [B]; keys: Fp4Keys."""
+    _need(dst_off, torch.int32, "dst_off")
+    if k.dtype != torch.bfloat16 or k.stride(-1) != 1 or not k.is_cuda:
+        raise Csa2Error(ERR_ARG, "k must be a CUDA bf16 tensor with unit channel stride")
+    B, n_new, Di = k.shape
+    st = lib().csa2_quantize_keys_fp4(_p(k), B, n_new, k.stride(1), k.stride(0), _p(dst_off),
+                                      _p(keys.buf), keys.cap, _p(status), _stream(stream))
+    _check(st, "csa2_quantize_keys_fp4")
+
+
+def _key_args(q_I, k_I):
+    """(dtype code, key pointer, cap) of index_score_topk's key argument."""
+    if isinstance(k_I, Fp4Keys):
+        if q_I.dtype != torch.float8_e4m3fn:
+            raise Csa2Error(ERR_ARG, "compact keys take an E4M3 query")
+        _need(q_I, q_I.dtype, "q_I")
+        return DTYPE_E4M3_FP4KEY, _p(k_I.buf), k_I.cap
     if q_I.dtype not in DTYPE or k_I.dtype != q_I.dtype:
         raise Csa2Error(ERR_ARG, "q_I and k_I must share a dtype (bf16 or float8_e4m3fn)")
     for t, nm in ((q_I, "q_I"), (k_I, "k_I")):
         _need(t, q_I.dtype, nm)
+    return DTYPE[q_I.dtype], _p(k_I), k_I.shape[1]
+
+
+def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None, ratio=1,
+                     pool_in=None, pool_out=None, pool_blocks=0, scores_out=None, stream=None):
+    """q_I [B, T, H_I, 128] (bf16 or E4M3), w fp32 [B, T, H_I], k_I [B, cap, 128] of the same
+    dtype (or Fp4Keys with an E4M3 query), idx_out int32 [B, T, K]. Decode: n_vis0 int32 [B].
+    Prefill: q_pos0 int32 [B] and ratio. Reindex: pool_in int32 [B, T, P]. Full with a pool:
+    pool_out int32 [B, T, pool_blocks * 8]."""
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    B, T, H_I, Di = q_I.shape
+    dt, kp, cap = _key_args(q_I, k_I)
     _need(w, torch.float32, "w")
     _need(idx_out, torch.int32, "idx_out")
     _need(n_vis0, torch.int32, "n_vis0")
@@ -237,10 +278,9 @@ def index_score_topk(mode, q_I, w, k_I, K, idx_out, ws, n_vis0=None, q_pos0=None
     _need(pool_in, torch.int32, "pool_in")
     _need(pool_out, torch.int32, "pool_out")
     _need(scores_out, torch.float32, "scores_out")
-    cap = k_I.shape[1]
     P_in = pool_in.shape[-1] if pool_in is not None else 0
     st = lib().csa2_index_score_topk(
-        m, B, T, H_I, DTYPE[q_I.dtype], _p(q_I), _p(w), _p(k_I), cap, _p(n_vis0), int(ratio),
+        m, B, T, H_I, dt, _p(q_I), _p(w), kp, cap, _p(n_vis0), int(ratio),
         _p(q_pos0), int(K), _p(pool_in), P_in, _p(pool_out), int(pool_blocks), _p(idx_out),
         _p(scores_out), _p(ws), ws.numel() if ws is not None else 0, _stream(stream))
     _check(st, "csa2_index_score_topk")

@@ -253,6 +253,24 @@ csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, const voi
     return cuda_status(launch_compress_kv(l, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+csa2_status_t csa2_quantize_keys_fp4(const void* k, int B, int n_new, int64_t ld, int64_t bstride,
+                                     const int32_t* dst_off, void* keys, int64_t cap,
+                                     int32_t* status, void* stream) {
+    if (B < 0 || n_new < 0 || cap < 1) return CSA2_ERR_ARG;
+    if ((int64_t)B * n_new == 0) return CSA2_OK;
+    if (!k || !dst_off || !keys) return CSA2_ERR_ARG;
+    if (ld < CSA2_D_INDEX || ld % 8 != 0 || bstride % 8 != 0 || bstride < 0) return CSA2_ERR_ARG;
+    if (B > 1 && bstride < (int64_t)(n_new - 1) * ld + CSA2_D_INDEX) return CSA2_ERR_ARG;
+    if (!aligned16(k) || (reinterpret_cast<uintptr_t>(keys) & 31u) != 0) return CSA2_ERR_ARG;
+    if ((int64_t)B * n_new > (int64_t)1 << 40 || (int64_t)B * cap > ((int64_t)1 << 40))
+        return CSA2_ERR_ARG;
+    uint8_t* codes = reinterpret_cast<uint8_t*>(keys);
+    float* scales = reinterpret_cast<float*>(codes + (size_t)B * cap * CSA2_FP4KEY_CODE_BYTES);
+    return cuda_status(launch_quantize_keys_fp4(k, B, n_new, ld, bstride, dst_off, codes, scales,
+                                                cap, status,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int csa2_sparse_attn_decode_launches(int B, int K, int W) {
     if (B < 1 || K < 0 || W < 0 || W > 1024 || K > 65536) return -1;
     return attention_decode_launches(B, K, W);
@@ -295,7 +313,12 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
         if (pool_in || pool_out) return CSA2_ERR_ARG;
         return CSA2_OK;
     }
-    if (qk_dtype != CSA2_DTYPE_BF16 && qk_dtype != CSA2_DTYPE_E4M3) return CSA2_ERR_ARG;
+    if (qk_dtype != CSA2_DTYPE_BF16 && qk_dtype != CSA2_DTYPE_E4M3 &&
+        qk_dtype != CSA2_DTYPE_E4M3_FP4KEY)
+        return CSA2_ERR_ARG;
+    const bool key_fp4 = qk_dtype == CSA2_DTYPE_E4M3_FP4KEY;
+    if (key_fp4 && (mode != CSA2_MODE_FULL || (reinterpret_cast<uintptr_t>(k_I) & 31u) != 0))
+        return mode != CSA2_MODE_FULL ? CSA2_ERR_UNSUPPORTED : CSA2_ERR_ARG;
     if (H_I < 1 || H_I > 128) return CSA2_ERR_UNSUPPORTED;
     if (!q_I || !w || !k_I) return CSA2_ERR_ARG;
     if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(w)) return CSA2_ERR_ARG;
@@ -373,6 +396,10 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
     sl.pool = pool_in;
     sl.P = P_in;
     sl.status = status;
+    sl.key_fp4 = key_fp4;
+    sl.kscale = key_fp4 ? reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(k_I) +
+                                                         (size_t)B * cap * CSA2_FP4KEY_CODE_BYTES)
+                        : nullptr;
     const cudaEvent_t ev0 = g_stage_ev[0], ev1 = g_stage_ev[1];
     g_stage_ev[0] = g_stage_ev[1] = nullptr;
     // inside a stream capture the events become external record nodes (usable for timing)

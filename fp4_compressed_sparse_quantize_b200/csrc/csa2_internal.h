@@ -51,12 +51,19 @@ struct ScanLaunch {
     const int32_t* pool;
     int P;
     int32_t* status;
+    bool key_fp4;           // compact keys: E2M1 codes (TMA-unpacked) + fp32 scale per key
+    const float* kscale;    // [B][cap] scales of compact keys
 };
 
 cudaError_t launch_quantize_kv(const void* kv, int B, int n_new, int64_t ld_kv,
                                int64_t bstride_kv, const int32_t* dst_off, uint8_t* codes,
                                uint8_t* scales, int64_t cap, int32_t* status,
                                cudaStream_t stream);
+
+cudaError_t launch_quantize_keys_fp4(const void* k, int B, int n_new, int64_t ld,
+                                     int64_t bstride, const int32_t* dst_off, uint8_t* codes,
+                                     float* scales, int64_t cap, int32_t* status,
+                                     cudaStream_t stream);
 
 // Compressor + indexer-K projection + FP4 write (csa2_compress_kv).
 struct CompressLaunch {

@@ -59,6 +59,7 @@ struct ScanParams {
     const int32_t* pool;    // gather mode: [R][P] positions, -1 = empty
     int P;
     const uint8_t* keys;    // gather mode: raw key base (row-major [B*cap][128*esize])
+    const float* kscale;    // compact keys: fp32 scale per key [B*cap]
     int32_t* status;
 };
 
@@ -148,13 +149,15 @@ __device__ __forceinline__ void fence_proxy_async() {
 // on the 256K-context workload.)
 constexpr int kEpiWarp0 = 3;                      // first epilogue warp
 
-template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM>
+template <int NQ, int ESZ, int STAGES, int ACC, int G, bool GATHER, bool POOL, int EPI, int TM,
+          bool KF4>
 __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     scan_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
     static_assert(ACC % EPI == 0, "each epilogue group owns fixed accumulators");
     static_assert(!GATHER || TM == 1, "gathered tiles are 128 keys");
+    static_assert(!KF4 || (ESZ == 1 && !GATHER), "compact keys: E4M3 queries, contiguous tiles");
     constexpr int kRowsT = L::kRowsT;
     constexpr int kKSteps = (128 * ESZ) / 32;         // 32 bytes of K per MMA instruction
     constexpr uint32_t kSlab = kRowsT * 128;          // bytes of one 128-byte-wide K slab
@@ -164,7 +167,10 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                                  : (ACC * kAccCols <= 128) ? 128 : (ACC * kAccCols <= 256) ? 256
                                  : 512;
     static_assert(ACC * kAccCols <= 512, "TMEM budget");
-    constexpr uint32_t kIdesc = make_idesc(128, NQ, ESZ == 2 ? 1u : 0u, ESZ == 2 ? 1u : 0u);
+    // A = keys (compact keys: E2M1, format 5 of kind::f8f6f4; the tensor map unpacks each 16
+    // codes into a 16-byte slot, so a key row is 128 bytes as with E4M3), B = queries
+    constexpr uint32_t kIdesc =
+        make_idesc(128, NQ, KF4 ? 5u : (ESZ == 2 ? 1u : 0u), ESZ == 2 ? 1u : 0u);
     constexpr int kCols = NQ / G;                     // accumulator columns per query row
     constexpr bool kWReg = (G == 1 && NQ <= 64);      // weights kept in registers
 
@@ -273,7 +279,10 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             uint8_t* dst = stage_base + s * L::kTileBytes;
             if (!GATHER) {
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)L::kTileBytes);
+                    // compact keys: the unpacking load counts the packed bytes it reads
+                    // (64 per key), half of what it writes to shared memory
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(KF4 ? L::kTileBytes / 2
+                                                                  : L::kTileBytes));
                     const int64_t row = (int64_t)b * p.cap + jt * kRowsT;
                     // one box of 128 rows per 128-key half (and per 64-channel half for bf16)
 #pragma unroll
@@ -471,6 +480,16 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             }
             ++since_flush;
             const int a = (int)(it % ACC);
+            // compact keys: this tile's key scales, loaded before the accumulator wait
+            float ks[TM];
+#pragma unroll
+            for (int hh = 0; hh < TM; ++hh) {
+                ks[hh] = 1.f;
+                if (KF4) {
+                    const int64_t j = jt * kRowsT + hh * 128 + row;
+                    ks[hh] = (j < p.cap) ? ld_dep(p.kscale + (int64_t)(r0 / p.T) * p.cap + j) : 0.f;
+                }
+            }
             aborted = aborted || *abort_flag;
             if (!aborted) {
                 if (!mbar_wait(&accfull[a], (uint32_t)((it / ACC) & 1), p.status)) {
@@ -508,7 +527,9 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                     float s4[4];
                     f2unpack(c01, s4[0], s4[1]);
                     f2unpack(c23, s4[2], s4[3]);
-                    sc[hh][gg] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + 0.0f;
+                    float sv = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                    if (KF4) sv *= ks[hh];   // the key's scale is >= 0: it leaves the ReLU
+                    sc[hh][gg] = sv + 0.0f;
                 }
             }
             tc_fence_before();
@@ -656,6 +677,22 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int esz, in
     return r == CUDA_SUCCESS;
 }
 
+// 2-D map over compact keys: [rows] x 128 E2M1 codes packed 64 bytes per row; the load
+// unpacks every 16 codes (8 bytes) into a 16-byte slot, giving 128-byte rows in shared
+// memory (the operand layout of an E2M1 kind::f8f6f4 MMA), 128-byte swizzle.
+static bool make_map_fp4(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)CSA2_FP4KEY_CODE_BYTES};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // SM count of the current device (looked up per call: one process may drive GPUs of
 // different sizes)
 static int num_sms() { return device_sm_count(); }
@@ -671,7 +708,7 @@ constexpr int pick_stages() {
          : ScanSmem<NQ, ESZ, 3, ACC, G, EPI, POOL, TM>::kAlloc <= 232448 ? 3 : 2;
 }
 
-template <int NQ, int ESZ, int G, bool GATHER, bool POOL>
+template <int NQ, int ESZ, int G, bool GATHER, bool POOL, bool KF4 = false>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
     // 384-key tiles for one FP8 query row per tile (fewer barrier waits and commits per key
@@ -685,7 +722,7 @@ static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
     constexpr int STAGES = pick_stages<NQ, ESZ, ACC, G, EPI, POOL, TM>();
     using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
-    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL, EPI, TM>;
+    auto kern = scan_kernel<NQ, ESZ, STAGES, ACC, G, GATHER, POOL, EPI, TM, KF4>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::kAlloc);
     if (e != cudaSuccess) return e;
@@ -702,8 +739,11 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     memset(&mk, 0, sizeof mk);
     memset(&mq, 0, sizeof mq);
     if (!make_map(&mq, a.q, (int64_t)a.rows * a.H_I, esz, NQ)) return cudaErrorInvalidValue;
-    if (!a.gather &&
+    if (a.key_fp4 && (a.gather || esz != 1)) return cudaErrorNotSupported;
+    if (!a.gather && !a.key_fp4 &&
         !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, kTileRows))
+        return cudaErrorInvalidValue;
+    if (a.key_fp4 && !make_map_fp4(&mk, a.k, (int64_t)a.B * a.cap, kTileRows))
         return cudaErrorInvalidValue;
     ScanParams p;
     p.rows = a.rows;
@@ -723,6 +763,7 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     p.pool = a.pool;
     p.P = a.P;
     p.keys = reinterpret_cast<const uint8_t*>(a.k);
+    p.kscale = a.kscale;
     p.status = a.status;
 
 #define CSA2_SCAN(NQv, ESZv, Gv, GA, PO) return launch_scan_t<NQv, ESZv, Gv, GA, PO>(mk, mq, p, st)
@@ -734,6 +775,25 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
         CSA2_SCAN(128, ESZv, 1, GA, PO);              \
     } while (0)
 
+    if (a.key_fp4) {
+#define CSA2_SCAN4(NQv, Gv, PO) return launch_scan_t<NQv, 1, Gv, false, PO, true>(mk, mq, p, st)
+        if (a.G == 1) {
+            if (a.pool_build) {
+                if (NQ <= 16) CSA2_SCAN4(16, 1, true);
+                if (NQ <= 32) CSA2_SCAN4(32, 1, true);
+                if (NQ <= 64) CSA2_SCAN4(64, 1, true);
+                CSA2_SCAN4(128, 1, true);
+            }
+            if (NQ <= 16) CSA2_SCAN4(16, 1, false);
+            if (NQ <= 32) CSA2_SCAN4(32, 1, false);
+            if (NQ <= 64) CSA2_SCAN4(64, 1, false);
+            CSA2_SCAN4(128, 1, false);
+        } else if (a.G == 2 && NQ <= 128 && !a.pool_build) {
+            CSA2_SCAN4(128, 2, false);
+        }
+#undef CSA2_SCAN4
+        return cudaErrorNotSupported;
+    }
     if (a.G == 1) {
         if (a.gather) {
             if (esz == 1) CSA2_SCAN_NQ(1, true, false);

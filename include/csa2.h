@@ -75,7 +75,11 @@ typedef enum csa2_mode {
 /* Storage type of the indexer query and key. */
 typedef enum csa2_dtype {
     CSA2_DTYPE_BF16 = 0,
-    CSA2_DTYPE_E4M3 = 1    /* OCP FP8 E4M3 ("fn": no infinities, max 448) */
+    CSA2_DTYPE_E4M3 = 1,   /* OCP FP8 E4M3 ("fn": no infinities, max 448) */
+    /* E4M3 query with compact 68-byte keys (csa2_quantize_keys_fp4): the key buffer holds
+     * two planes, E2M1 codes [B][cap][64] and then fp32 scales [B][cap] starting at byte
+     * B*cap*64; its start must be 32-byte aligned. Full mode only. */
+    CSA2_DTYPE_E4M3_FP4KEY = 2
 } csa2_dtype_t;
 
 /* Operations that need a workspace. */
@@ -96,6 +100,7 @@ typedef enum csa2_op {
 #define CSA2_ENTRY_CODE_BYTES 256 /* packed E2M1 bytes per main-KV entry (512 / 2)      */
 #define CSA2_ENTRY_SCALE_BYTES 32 /* E4M3 scale bytes per main-KV entry (512 / 16)      */
 #define CSA2_POOL_BLOCK 8         /* positions per candidate-pool block                 */
+#define CSA2_FP4KEY_CODE_BYTES 64 /* E2M1 code bytes of a compact indexer key (128 / 2)  */
 
 /*
  * csa2_quantize_kv — FP4 quantize-on-write of new main-KV entries.
@@ -157,6 +162,27 @@ CSA2_API csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, 
                                         void* stream);
 
 /*
+ * csa2_quantize_keys_fp4 — compact 68-byte indexer keys.
+ * [AIS Main Findings], [TLB How is DeepSeek V4.1 Flash different] (Figure 1): 890 bytes of
+ * global KV per token; with 2.5 stored entry-sets per token and 288-byte FP4 main entries
+ * that leaves 68 bytes per indexer key. The pages give no key format; reading: E2M1 codes
+ * of the 128 channels (64 bytes, channel 2k in the low nibble of byte k) times one fp32
+ * scale per key. Decisions in IEEE fp32: s = amax / 6; magnitude = E2M1(|x| / s) rounded
+ * to nearest-even and saturated at 6, sign copied from x; s == 0 gives zero magnitudes.
+ *
+ *   k        bf16 [B][n_new][128]: element (b,i,c) at k[b*bstride + i*ld + c]; ld >= 128,
+ *            ld and bstride multiples of 8; 16-byte aligned; finite values.
+ *   dst_off  int32 [B]: entry index of sequence b's first new key.
+ *   keys     the two-plane compact key buffer of CSA2_DTYPE_E4M3_FP4KEY (codes
+ *            [B][cap][64], then fp32 scales [B][cap] at byte B*cap*64); 32-byte aligned.
+ *   status   nullable int32 device word: CSA2_DEV_BAD_INDEX for a key outside [0, cap).
+ */
+CSA2_API csa2_status_t csa2_quantize_keys_fp4(const void* k, int B, int n_new, int64_t ld,
+                                              int64_t bstride, const int32_t* dst_off,
+                                              void* keys, int64_t cap, int32_t* status,
+                                              void* stream);
+
+/*
  * csa2_index_score_topk — indexer scoring + exact Top-K selection, per layer mode.
  * [AIS Methodology]: each layer has its own indexer query; Full layers score, Reindex
  * layers rescore the latest Full layer's keys, Reuse layers skip indexing; the first
@@ -170,8 +196,11 @@ CSA2_API csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, 
  *   mode      FULL / REINDEX / REUSE. REUSE validates arguments and launches nothing.
  *   B, T      sequences and query tokens per sequence (T = 1 for decode).
  *   H_I       indexer heads, 1..128.
- *   qk_dtype  storage type of q_I and k_I.
- *   q_I       [B][T][H_I][128];  w  fp32 [B][T][H_I];  k_I  [B][cap][128].
+ *   qk_dtype  storage type of q_I and k_I; CSA2_DTYPE_E4M3_FP4KEY: E4M3 q_I and compact
+ *             68-byte keys (FULL only; the score is the same formula over the keys'
+ *             decoded values e2m1(code) * scale).
+ *   q_I       [B][T][H_I][128];  w  fp32 [B][T][H_I];  k_I  [B][cap][128] (compact keys:
+ *             the two-plane buffer described at CSA2_DTYPE_E4M3_FP4KEY).
  *   n_vis0    int32 [B]: visible entries per sequence (decode, q_pos0 == NULL).
  *   ratio, q_pos0
  *             prefill visibility (q_pos0 != NULL): token t of sequence b sits at
