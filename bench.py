@@ -36,7 +36,8 @@ from fp4_compressed_sparse_quantize_b200 import csa2, synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "decode_full_b32_ctx64k_r2"
 # reported beside the default line: the rest of the 64K-1M decode range and the prefill chunk
-EXTRA_DECODE = ("decode_group4_b64_ctx256k", "decode_pool_reindex_b4_ctx1m")
+EXTRA_DECODE = ("decode_group4_b64_ctx256k", "decode_pool_reindex_b4_ctx1m",
+                "decode_full_b32_ctx64k_r2_key68")
 EXTRA_PREFILL = "prefill_b2_t4k_ctx128k_r2"
 L2_FLUSH_BYTES = 256 << 20
 SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csrc", "indexer.cu")
@@ -132,6 +133,12 @@ class Decode:
             dirs = synth.planted_direction([L["q_I"] for L, m in zip(self.layers, w.layers)
                                             if m in ("full", "reindex")])
         self.k_I, self.planted = synth.indexer_keys(w, seed, dev, planted_dirs=dirs)
+        if w.key_format == "fp4":
+            # compact 68-byte keys, written by the library's key quantiser
+            kb = self.k_I
+            self.k_I = csa2.Fp4Keys(B, cap, device=dev)
+            csa2.quantize_keys_fp4(kb, torch.zeros(B, dtype=torch.int32, device=dev), self.k_I)
+            del kb
         # FP4 cache built once by the library's own quantize-on-write
         self.codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
         self.scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
@@ -231,14 +238,15 @@ class Decode:
         w = self.w
         B, N, K, H, W = w.B, w.N, w.K, w.H, synth.WINDOW
         ek = 2 if w.idx_dtype == "bf16" else 1
+        kb = 68 if w.key_format == "fp4" else 128 * ek      # indexer-key bytes per entry
         tot = B * (512 * 2 + 288)                         # quantize-on-write
         scan = 0
         for m in w.layers:
             if m in ("full", "reindex"):
                 rows = N if m == "full" else synth.POOL_BLOCKS * synth.POOL_BLOCK
-                b = B * (rows * 128 * ek + w.H_I * 128 * ek + w.H_I * 4 + K * 4)
+                b = B * (rows * kb + w.H_I * 128 * ek + w.H_I * 4 + K * 4)
                 if m == "full":
-                    scan = B * (N * 128 * ek + w.H_I * 128 * ek + w.H_I * 4)
+                    scan = B * (N * kb + w.H_I * 128 * ek + w.H_I * 4)
                 if m == "reindex":
                     b += B * rows * 4
                 if m == "full" and w.pool:
@@ -648,9 +656,14 @@ def oracle_queries(state, budget_s):
     b = 0
     while t_total < budget_s and b < w.B:
         # inputs of sequence b (copied out of device memory before the clock starts)
-        k_raw = state.k_I[b, :w.N].contiguous().cpu().view(torch.uint8 if ek == O.E4M3 else torch.int16).numpy()
-        if ek == O.BF16:
-            k_raw = k_raw.view(np.uint16)
+        fp4 = w.key_format == "fp4"
+        if fp4:
+            k_codes = state.k_I.codes[b, :w.N].cpu().numpy()
+            k_scales = state.k_I.scales[b, :w.N].cpu().numpy()
+        else:
+            k_raw = state.k_I[b, :w.N].contiguous().cpu().view(torch.uint8 if ek == O.E4M3 else torch.int16).numpy()
+            if ek == O.BF16:
+                k_raw = k_raw.view(np.uint16)
         src = _main_rows(w, state.seed, b, state.dev)[: w.N].cpu().view(torch.int16).numpy().view(np.uint16)
         lay = []
         for L in state.layers:
@@ -665,7 +678,8 @@ def oracle_queries(state, budget_s):
         pool = None
         for (qi, wt, qb, swa), mode in zip(lay, w.layers):
             if mode == "full":
-                s = O.index_scores(qi, wt, k_raw, ek)
+                s = (O.index_scores_fp4key(qi, wt, k_codes, k_scales) if fp4
+                     else O.index_scores(qi, wt, k_raw, ek))
                 cur = O.topk(s, w.K)
                 if w.pool:
                     pool = O.pool(s, synth.POOL_BLOCKS)

@@ -42,6 +42,8 @@ class Workload:
     lognormal_channels: bool = False
     planted: int = 0          # planted high-score keys per sequence (recall check)
     pool: bool = False        # Full layer also builds the candidate pool
+    key_format: str = "dense"  # "dense" (keys in idx_dtype) or "fp4" (compact 68-byte keys,
+                               # quantised by the library from bf16 keys; E4M3 queries)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -85,6 +87,11 @@ WORKLOADS = {
     "prefill_b2_t4k_ctx128k_r2": Workload("prefill_b2_t4k_ctx128k_r2", "prefill", B=2,
                                           ctx=131072, ratio=2, H_I=64, idx_dtype="e4m3",
                                           K=512, H=64, T=4096),
+    # decode_full_b32_ctx64k_r2 with compact 68-byte indexer keys (890 bytes per token)
+    "decode_full_b32_ctx64k_r2_key68": Workload("decode_full_b32_ctx64k_r2_key68", "decode",
+                                                B=32, ctx=65536, ratio=2, H_I=64,
+                                                idx_dtype="e4m3", K=512, H=64,
+                                                lognormal_channels=True, key_format="fp4"),
     # the same chunked prefill at one sequence and 1024 new tokens (profiler captures)
     "prefill_b1_t1k_ctx128k_r2": Workload("prefill_b1_t1k_ctx128k_r2", "prefill", B=1,
                                           ctx=131072, ratio=2, H_I=64, idx_dtype="e4m3",
@@ -172,11 +179,12 @@ def indexer_keys(w: Workload, seed0: int, device, planted_dirs=None):
     """Indexer keys [B, cap, 128]; with planted keys, `planted` positions per sequence
     (each in its own 8-entry block) are overwritten by alpha * the given unit direction
     of that sequence (planted_dirs: float32 [B, 128]). Returns (keys, planted positions
-    int64 [B, planted] or None)."""
-    tdt = torch.bfloat16 if w.idx_dtype == "bf16" else torch.float8_e4m3fn
+    int64 [B, planted] or None). With compact keys (key_format "fp4") the keys are returned
+    as bf16, for the library's key quantiser."""
+    kdt = "bf16" if w.key_format == "fp4" else w.idx_dtype
+    tdt = torch.bfloat16 if kdt == "bf16" else torch.float8_e4m3fn
     k = torch.empty((w.B, w.cap, D_IDX), dtype=tdt, device=device)
-    _fill_per_seq(k, w.B, lambda b: _cast(_randn((w.cap, D_IDX), seed0, 3, b, device),
-                                          w.idx_dtype))
+    _fill_per_seq(k, w.B, lambda b: _cast(_randn((w.cap, D_IDX), seed0, 3, b, device), kdt))
     pos = None
     if w.planted:
         alpha = float(w.extra.get("planted_alpha", 24.0))
@@ -189,7 +197,7 @@ def indexer_keys(w: Workload, seed0: int, device, planted_dirs=None):
             p = torch.sort(blocks * POOL_BLOCK + off).values
             pos[b] = p
             vec = (alpha * planted_dirs[b].float()).to(device)
-            k[b, p.to(device)] = _cast(vec.expand(w.planted, D_IDX).contiguous(), w.idx_dtype)
+            k[b, p.to(device)] = _cast(vec.expand(w.planted, D_IDX).contiguous(), kdt)
     return k, pos
 
 

@@ -4,6 +4,7 @@ sampled outputs the oracle computes one by one:
 
   decode_full_b1_ctx4k          every output
   decode_full_b32_ctx64k_r2     every query's Top-512; attention and FP4 codes on samples
+  decode_full_b32_ctx64k_r2_key68  the same with compact 68-byte indexer keys
   decode_group4_b64_ctx256k     Full + 3 Reuse: 16 sampled queries, every layer
   decode_pool_reindex_b4_ctx1m  Full + pool + Reindex on every query; planted-key recall
   prefill_b2_t4k_ctx128k_r2     ~90 sampled query tokens per sequence (first, last, every
@@ -44,6 +45,10 @@ def _bench():
 def _oracle_scores(state, li, b, rows=None):
     L = state.layers[li]
     w = state.w
+    if w.key_format == "fp4":
+        return O.index_scores_fp4key(bits8(L["q_I"][b, 0]), L["w"][b, 0].cpu().numpy(),
+                                     state.k_I.codes[b, :w.N].cpu().numpy(),
+                                     state.k_I.scales[b, :w.N].cpu().numpy(), rows=rows)
     return O.index_scores(raw_qk(L["q_I"][b, 0]), L["w"][b, 0].cpu().numpy(),
                           raw_qk(state.k_I[b, :w.N]), odt(L["q_I"]), rows=rows)
 
@@ -143,6 +148,24 @@ def test_decode_full_b1_ctx4k():
 def test_decode_full_b32_ctx64k_r2():
     state = _run_decode("decode_full_b32_ctx64k_r2", None)
     kinds = _check_decode(state, list(range(32)), check_codes_b=[0, 31])
+    assert kinds.count("exact") >= 24, kinds
+
+
+def test_decode_full_b32_ctx64k_r2_key68():
+    """The same decode step with compact 68-byte indexer keys: every query's Top-512 against
+    the oracle's scores over the keys' decoded values, attention on samples; the compact key
+    cache against the oracle's quantiser on two sequences."""
+    from fp4_compressed_sparse_quantize_b200 import synth
+    state = _run_decode("decode_full_b32_ctx64k_r2_key68", None)
+    w = state.w
+    kb, _ = synth.indexer_keys(w, SEED, torch.device(dev))
+    for b in (0, 31):
+        oc, os_ = O.quantize_keys_fp4(bits16(kb[b]))
+        np.testing.assert_array_equal(state.k_I.codes[b].cpu().numpy(), oc)
+        np.testing.assert_array_equal(state.k_I.scales[b].cpu().numpy().view(np.uint32),
+                                      os_.view(np.uint32))
+    del kb
+    kinds = _check_decode(state, list(range(32)), check_codes_b=[0])
     assert kinds.count("exact") >= 24, kinds
 
 
