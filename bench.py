@@ -595,6 +595,101 @@ def prefill_main(args, w, dev, rank, world):
         print(json.dumps(line), flush=True)
 
 
+CP_WORKLOAD = "decode_pool_reindex_b4_ctx1m"
+
+
+def cp_main(args, dev, rank, world, local):
+    """Context-parallel Full layer of the 1M-context workload (--cp): every rank holds one
+    contiguous shard of every sequence's entries (indexer keys and FP4 main KV); the layer's
+    selection (scan, candidate pool, Top-512) and its attention run through cp.select and
+    cp.attend, whose exchanges are NCCL all-gathers of the shard selections and of the
+    attention partials. Strong scaling: the same B queries whatever the rank count."""
+    import socket
+    import torch.distributed as dist
+    from fp4_compressed_sparse_quantize_b200 import cp
+    if not dist.is_initialized():          # one rank: a one-rank NCCL group
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(sk.getsockname()[1]))
+        sk.close()
+        import datetime
+        dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+    w = synth.WORKLOADS[CP_WORKLOAD]
+    B, cap, K = w.B, w.cap, w.K
+    seed = args.seed                        # one batch: the same inputs on every rank
+    lo, hi = cp.shards(cap, world)[rank]
+    L = synth.layer_inputs(w, 0, seed, dev)
+    dirs = synth.planted_direction([L["q_I"]]) if w.planted else None
+    k_full, _ = synth.indexer_keys(w, seed, dev, planted_dirs=dirs)
+    k_shard = k_full[:, lo:hi].contiguous()
+    del k_full
+    codes = torch.zeros((B, hi - lo, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, hi - lo, 32), dtype=torch.uint8, device=dev)
+    for b in range(B):
+        src = _main_rows(w, seed, b, dev)[lo:hi].contiguous()
+        csa2.quantize_kv(src[None], torch.zeros(1, dtype=torch.int32, device=dev),
+                         codes[b:b + 1], scales[b:b + 1])
+        del src
+    n_vis = synth.decode_positions(w, dev)
+    ws_i = csa2.new_workspace(csa2.workspace_bytes(0, B, 1, w.H_I, hi - lo, K, synth.POOL_BLOCKS))
+    ws_a = csa2.new_workspace(csa2.workspace_bytes(1, B, 1, w.H, hi - lo, K))
+    out = torch.empty((B, w.H, synth.D_MAIN), dtype=torch.float32, device=dev)
+    tau = 1.0 / math.sqrt(synth.D_MAIN)
+    swa = L["swa"] if rank == 0 else None
+    torch.cuda.empty_cache()
+
+    def step():
+        idx, _pool = cp.select(L["q_I"], L["w"], k_shard, n_vis, lo, K, ws_i,
+                               pool_blocks=synth.POOL_BLOCKS)
+        cp.attend("full", L["q"], codes, scales, idx.view(B, K), lo, swa, out, ws_a, scale=tau)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist, dev)
+    st = [csa2.read_device_status(ws_i), csa2.read_device_status(ws_a)]
+    ms = total / args.steps
+    # per step: prep, scan, Top-K, pool Top-K; candidates, merge (x2), pool candidates, pool
+    # expansion; local indices, the attention's launches, the partials' merge
+    launches = 4 + 5 + 1 + csa2.sparse_attn_decode_launches(B, K, synth.WINDOW) + 1
+    exch = world * B * (K * 8 + synth.POOL_BLOCKS * 8 + w.H * (synth.D_MAIN + 2) * 4)
+    line = {
+        "metric": "CSA2 context-parallel Full layer (scan + pool + Top-512 + attention) "
+                  "queries/s at 1M ctx",
+        "value": B / (ms / 1e3), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "e4m3/fp4/fp16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": CP_WORKLOAD + " (Full layer)", "batch": B,
+                   "compressed_entries": cap, "shard_entries": hi - lo,
+                   "parallelism": f"cp{world} (entries sharded; NCCL all-gather of selections "
+                                  "and attention partials)",
+                   "launch": "eager (NCCL collectives between the library calls)",
+                   "l2": "not flushed: each step streams the shard's indexer keys"},
+        "exchange_bytes_per_step": exch,
+        "gpu_launches": launches * args.steps,
+        "clocks": clk, "device_status": st,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def local_rank():
     return int(os.environ.get("LOCAL_RANK", "0"))
 
@@ -734,6 +829,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the shorter runs of the other workloads (256K, 1M, prefill)")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--cp", action="store_true",
+                    help="context-parallel Full layer of the 1M-context workload over the ranks")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call from Python instead of replaying CUDA graphs")
     args = ap.parse_args()
@@ -757,6 +854,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
         pg = dist
+    if args.cp:
+        return cp_main(args, dev, rank, world, local)
     w = synth.WORKLOADS[args.workload]
     if w.kind == "prefill":
         prefill_main(args, w, dev, rank, world)

@@ -6,7 +6,10 @@ oracle, the lists travel through cp.all_gather_last, and the merge by the oracle
 the Top-K and for the block pool, with planted exact ties at both boundaries.
 
 GPU (one device, shards run one after another): the cp_* kernels. The selection merged from
-G shard scans is bit-identical to the single-scan selection (indices and pool)."""
+G shard scans is bit-identical to the single-scan selection (indices and pool) and passes
+the oracle's Top-K and pool checks; cp.select and cp.attend run over a one-rank NCCL group.
+cp.attend's own logic (local indices, the window on one rank, the exchange) also runs over
+two gloo ranks on CPU with the kernels replaced by oracle stand-ins."""
 import os
 import socket
 
@@ -202,6 +205,18 @@ def test_gpu_sharded_selection_equals_single(G, n_list, K, nblk):
     assert csa2.read_device_status(ws) == 0
     assert torch.equal(idx, ref_idx)
     assert torch.equal(pool, ref_pool)
+    # and against the oracle's whole-context selection (scores over the same keys)
+    from tests.helpers import bits8, check_topk
+    idx_np, pool_np = idx.cpu().numpy(), pool.cpu().numpy()
+    for b, n in enumerate(n_list):
+        s = O.index_scores(bits8(q_I[b, 0]), w[b, 0].cpu().numpy(), bits8(k_I[b, :n]), O.E4M3)
+        check_topk(idx_np[b, 0], s, np.arange(n), K, f"G={G} b={b}")
+        nb = (n + 7) // 8
+        bmax = np.array([s[8 * c:8 * c + 8].max() for c in range(nb)])
+        got = np.unique(pool_np[b, 0][pool_np[b, 0] >= 0] // 8)
+        gb = np.full(nblk, -1)
+        gb[:len(got)] = got
+        check_topk(gb, bmax, np.arange(nb), nblk, f"G={G} pool b={b}")
 
 
 def _select_worker(port, q):
@@ -243,6 +258,60 @@ def test_gpu_select_one_rank_nccl():
     p.join(timeout=60)
     assert p.exitcode == 0
     assert res == (True, True, 0)
+
+
+def _attend_nccl_worker(port, q):
+    """cp.attend over a one-rank NCCL group: the partial path, the exchange and the merge
+    kernel on a GPU, against the oracle."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        import math
+        from fp4_compressed_sparse_quantize_b200 import csa2
+        from tests.helpers import bits16, bits8, oracle_main_rows
+        dev = "cuda"
+        g = torch.Generator().manual_seed(91)
+        B, H, n, K, W = 3, 64, 9000, 512, 128
+        kv = (torch.randn((B, n, 512), generator=g) *
+              torch.exp(torch.randn((B, 1, 512), generator=g))).to(torch.bfloat16)
+        codes = torch.zeros((B, n, 256), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, n, 32), dtype=torch.uint8, device=dev)
+        csa2.quantize_kv(kv.to(dev), torch.zeros(B, dtype=torch.int32, device=dev), codes, scales)
+        rng = np.random.default_rng(9)
+        idx = np.stack([np.sort(rng.choice(n, K, replace=False)) for _ in range(B)]).astype(np.int32)
+        qh = torch.randn((B, H, 512), generator=g).to(torch.bfloat16)
+        swa = torch.randn((B, W, 512), generator=g).to(torch.float8_e4m3fn)
+        tau = 1 / math.sqrt(512)
+        out = torch.empty((B, H, 512), dtype=torch.float32, device=dev)
+        ws = csa2.new_workspace(csa2.workspace_bytes(1, B, 1, H, n, K))
+        cp.attend("full", qh.to(dev), codes, scales, torch.from_numpy(idx).to(dev), 0,
+                  swa.to(dev), out, ws, scale=tau)
+        torch.cuda.synchronize()
+        errs = []
+        for b in range(B):
+            rows = np.concatenate([oracle_main_rows(bits16(kv[b, idx[b]])),
+                                   O.e4m3_array_to_f64(bits8(swa[b])).reshape(W, 512)])
+            ref = O.attention(O.bf16_array_to_f64(bits16(qh[b])).reshape(H, 512), rows, tau)
+            errs.append(float(np.max(np.abs(out[b].cpu().numpy() - ref)) /
+                              math.sqrt(float(np.mean(ref * ref)))))
+        q.put((errs, csa2.read_device_status(ws)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_gpu_attend_one_rank_nccl():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_attend_nccl_worker, args=(_free_port(), q))
+    p.start()
+    errs, st = q.get(timeout=300)
+    p.join(timeout=60)
+    assert p.exitcode == 0
+    assert st == 0
+    assert max(errs) <= 2e-3, errs
 
 
 # ---- attention over shards: partial results merged by the log-sum-exp identity -------------
@@ -345,3 +414,113 @@ def test_gpu_sharded_attention_matches_oracle(G, B, H, n, K, W):
                                O.e4m3_array_to_f64(bits8(swa[b])).reshape(W, 512)])
         ref = O.attention(O.bf16_array_to_f64(bits16(q[b])).reshape(H, 512), rows, tau)
         check_attention(out[b].cpu().numpy(), ref, f"G={G} b={b}")
+
+
+# ---- cp.attend on CPU ranks: the module's plumbing with the kernels stood in for --------------
+
+class _FakeKernels:
+    """CPU stand-ins (from the oracle) for the three library calls cp.attend makes, with the
+    kernels' argument conventions: local indices (-1 off-shard), base-2 (maximum, sum)
+    partials with the unnormalised output, and their log-sum-exp merge."""
+
+    @staticmethod
+    def cp_local_idx(idx, lo, hi, out, stream=None):
+        i = idx.to(torch.int64)
+        out.copy_(torch.where((i >= lo) & (i < hi), i - lo, torch.full_like(i, -1)).to(out.dtype))
+
+    @staticmethod
+    def sparse_attn_decode_partial(mode, q, codes, scales, idx, swa, o_part, ml_part, ws,
+                                   scale=None, swa_valid=None, stream=None):
+        B, H, D = q.shape
+        for b in range(B):
+            sel = [int(i) for i in idx[b] if i >= 0]
+            rows = O.dequant_entries(codes[b, sel].numpy(), scales[b, sel].numpy()) if sel \
+                else np.zeros((0, D))
+            if swa is not None:
+                rows = np.concatenate([rows, O.e4m3_array_to_f64(
+                    swa[b].view(torch.uint8).numpy().ravel()).reshape(-1, D)])
+            qb = O.bf16_array_to_f64(q[b].view(torch.int16).numpy().view(np.uint16)).reshape(H, D)
+            if rows.shape[0] == 0:
+                o_part[b] = 0
+                ml_part[b, 0] = -float("inf")
+                ml_part[b, 1] = 0
+                continue
+            lg2 = scale * (qb @ rows.T) / np.log(2.0)
+            m = lg2.max(axis=1)
+            p = np.exp2(lg2 - m[:, None])
+            o_part[b] = torch.from_numpy(p @ rows)
+            ml_part[b, 0] = torch.from_numpy(m)
+            ml_part[b, 1] = torch.from_numpy(p.sum(axis=1))
+
+    @staticmethod
+    def attn_merge_partials(o_parts, ml_parts, out, stream=None):
+        o = o_parts.double().numpy()
+        m = ml_parts[:, :, 0].double().numpy()
+        l = ml_parts[:, :, 1].double().numpy()
+        M = m.max(axis=0)
+        wgt = np.exp2(m - M)
+        out.copy_(torch.from_numpy((wgt[..., None] * o).sum(axis=0) /
+                                   (wgt * l).sum(axis=0)[..., None]))
+
+
+def _attend_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        for nm in ("cp_local_idx", "sparse_attn_decode_partial", "attn_merge_partials"):
+            setattr(cp.csa2, nm, getattr(_FakeKernels, nm))
+        g = torch.Generator().manual_seed(5)
+        B, H, n, K, W, tau = 2, 8, 1000, 64, 16, 1 / np.sqrt(512)
+        kv = (torch.randn((B, n, 512), generator=g) *
+              torch.exp(torch.randn((B, 1, 512), generator=g))).to(torch.bfloat16)
+        codes = np.zeros((B, n, 256), np.uint8)
+        scales = np.zeros((B, n, 32), np.uint8)
+        for b in range(B):
+            codes[b], scales[b] = O.quantize_entries(
+                kv[b].view(torch.int16).numpy().view(np.uint16))
+        rng = np.random.default_rng(3)
+        idx = np.stack([np.sort(rng.choice(n, K, replace=False)) for _ in range(B)]).astype(np.int32)
+        idx[1, -5:] = -1                              # padded selection
+        qh = torch.randn((B, H, 512), generator=g).to(torch.bfloat16)
+        swa = torch.randn((B, W, 512), generator=g).to(torch.float8_e4m3fn)
+        lo, hi = cp.shards(n, world)[rank]
+        out = torch.empty((B, H, 512), dtype=torch.float32)
+        cp.attend("full", qh, torch.from_numpy(codes[:, lo:hi].copy()),
+                  torch.from_numpy(scales[:, lo:hi].copy()), torch.from_numpy(idx), lo,
+                  swa if rank == 0 else None, out, None, scale=tau)
+        errs = []
+        for b in range(B):
+            sel = [int(i) for i in idx[b] if i >= 0]
+            rows = np.concatenate([O.dequant_entries(codes[b, sel], scales[b, sel]),
+                                   O.e4m3_array_to_f64(swa[b].view(torch.uint8).numpy().ravel()
+                                                       ).reshape(W, 512)])
+            ref = O.attention(O.bf16_array_to_f64(qh[b].view(torch.int16).numpy()
+                                                  .view(np.uint16)).reshape(H, 512), rows, tau)
+            errs.append(float(np.max(np.abs(out[b].double().numpy() - ref)) /
+                              np.sqrt(np.mean(ref * ref))))
+        q.put((rank, errs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_attend_plumbing_equals_whole_context():
+    """cp.attend over two gloo ranks (window rows on rank 0 only): local indices, the
+    partials' exchange through all_gather_stack and the merge reproduce the oracle's
+    attention over the whole selection. The three kernels are replaced by CPU stand-ins
+    with the same conventions, so this tests the module, not the kernels (those are the
+    GPU tests above)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_attend_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=180) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, errs in out:
+        for b, e in enumerate(errs):
+            # fp32 storage of the partials and of the output; a plumbing mistake (a window
+            # counted twice, a lost shard, unshifted indices) is an O(1) error
+            assert e < 1e-5, f"rank {rank} b={b}: {e:.3g}"
