@@ -711,10 +711,12 @@ constexpr int pick_stages() {
 template <int NQ, int ESZ, int G, bool GATHER, bool POOL, bool KF4 = false>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
-    // 384-key tiles for one FP8 query row per tile (fewer barrier waits and commits per key
-    // for the single MMA-issuing thread); two epilogue groups whenever the TMEM accumulators
-    // split evenly between them
-    constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 3 : 1;
+    // 384-key tiles for one FP8 query row per tile and 256-key tiles for two (prefill): the
+    // per-tile hand-over (mbarrier waits behind in-flight commits, the named barrier, the
+    // commits) costs about the same whatever the tile holds, so the tiles are as large as
+    // two accumulators allow; two epilogue groups whenever the TMEM accumulators split
+    // evenly between them
+    constexpr int TM = (G == 1 && !GATHER && ESZ == 1) ? 3 : (G == 2 && !GATHER && ESZ == 1) ? 2 : 1;
     constexpr int kAccCols = TM * NQ;
     constexpr int ACC = kAccCols <= 128 ? 4 : kAccCols <= 256 ? 2 : 1;
     constexpr int EPI = (ACC % 2 == 0 && G <= 2) ? 2 : 1;
@@ -816,7 +818,8 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
 }
 
 int scan_tile_rows(int G, bool gather, int esz) {
-    return (G == 1 && !gather && esz == 1) ? 3 * kTileRows : kTileRows;
+    return (G == 1 && !gather && esz == 1) ? 3 * kTileRows
+         : (G == 2 && !gather && esz == 1) ? 2 * kTileRows : kTileRows;
 }
 
 cudaError_t launch_prep_rows(int rows, int T, int G, const int32_t* n_vis0,
