@@ -207,15 +207,19 @@ def compress_kv(C, Z, ratio, w_proj, dst_off, codes, scales, k_I, latent_out=Non
     _need(codes, torch.uint8, "codes")
     _need(scales, torch.uint8, "scales")
     _need(latent_out, torch.bfloat16, "latent_out")
-    if k_I.dtype not in DTYPE:
-        raise Csa2Error(ERR_ARG, "k_I must be bf16 or float8_e4m3fn")
-    _need(k_I, k_I.dtype, "k_I")
+    if isinstance(k_I, Fp4Keys):
+        kdt, kp = DTYPE_E4M3_FP4KEY, _p(k_I.buf)
+    else:
+        if k_I.dtype not in DTYPE:
+            raise Csa2Error(ERR_ARG, "k_I must be bf16, float8_e4m3fn or Fp4Keys")
+        _need(k_I, k_I.dtype, "k_I")
+        kdt, kp = DTYPE[k_I.dtype], _p(k_I)
     B, n_tok, D = C.shape
     if n_tok % ratio:
         raise Csa2Error(ERR_ARG, "the token count must be a multiple of the ratio")
     st = lib().csa2_compress_kv(B, n_tok // ratio, int(ratio), _p(C), _p(Z), C.stride(1),
-                                C.stride(0), _p(w_proj), DTYPE[k_I.dtype], _p(dst_off),
-                                _p(codes), _p(scales), _p(k_I), codes.shape[1], _p(latent_out),
+                                C.stride(0), _p(w_proj), kdt, _p(dst_off),
+                                _p(codes), _p(scales), kp, codes.shape[1], _p(latent_out),
                                 _p(status), _stream(stream))
     _check(st, "csa2_compress_kv")
 

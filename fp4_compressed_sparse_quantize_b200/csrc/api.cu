@@ -224,7 +224,11 @@ csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, const voi
                                void* stream) {
     if (B < 0 || n_new < 0 || cap < 1 || r < 1 || r > 64) return CSA2_ERR_ARG;
     if ((int64_t)B * n_new == 0) return CSA2_OK;
-    if (key_dtype != CSA2_DTYPE_E4M3 && key_dtype != CSA2_DTYPE_BF16) return CSA2_ERR_ARG;
+    if (key_dtype != CSA2_DTYPE_E4M3 && key_dtype != CSA2_DTYPE_BF16 &&
+        key_dtype != CSA2_DTYPE_E4M3_FP4KEY)
+        return CSA2_ERR_ARG;
+    if (key_dtype == CSA2_DTYPE_E4M3_FP4KEY && (reinterpret_cast<uintptr_t>(k_I) & 31u) != 0)
+        return CSA2_ERR_ARG;
     if (!C || !Z || !w_proj || !dst_off || !codes || !scales || !k_I) return CSA2_ERR_ARG;
     if (ld < CSA2_D_MAIN || ld % 8 != 0 || bstride % 8 != 0 || bstride < 0) return CSA2_ERR_ARG;
     if (B > 1 && bstride < ((int64_t)r * n_new - 1) * ld + CSA2_D_MAIN) return CSA2_ERR_ARG;
@@ -243,6 +247,7 @@ csa2_status_t csa2_compress_kv(int B, int n_new, int r, const void* C, const voi
     l.Z = Z;
     l.w_proj = w_proj;
     l.key_bf16 = key_dtype == CSA2_DTYPE_BF16;
+    l.key_fp4 = key_dtype == CSA2_DTYPE_E4M3_FP4KEY;
     l.dst_off = dst_off;
     l.codes = codes;
     l.scales = scales;

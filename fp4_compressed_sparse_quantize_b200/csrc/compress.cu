@@ -50,8 +50,10 @@ struct CompressDev {
     const int32_t* dst_off;
     uint8_t* codes;
     uint8_t* scales;
-    uint8_t* keys;                // [B][cap][128] E4M3 or bf16
+    uint8_t* keys;                // [B][cap][128] E4M3 or bf16, or compact-key codes [B][cap][64]
+    float* key_scales;            // compact keys: fp32 scale per key [B][cap]
     int key_bf16;
+    int key_fp4;
     int64_t cap;
     __nv_bfloat16* latent;        // [B * n_new][512] or null
     int32_t* status;
@@ -222,7 +224,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int m = warp * 32 + lane;
         const int64_t crow = row_dst[m];
-        if (ok) {
+        if (ok && a.key_fp4) {
+            // compact key of the bf16-rounded projection (csa2_quantize_keys_fp4's decisions):
+            // pass 1 its amax, pass 2 the E2M1 codes under s = amax / 6
+            const uint32_t row_t = tmem + ((uint32_t)(warp * 32) << 16);
+            auto rounded = [](uint32_t u) { return __bfloat162float(__float2bfloat16_rn(__uint_as_float(u))); };
+            float amax = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kDi; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(row_t + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(rounded(v[k])));
+            }
+            const float s = __fdiv_rn(amax, 6.0f);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kDi; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(row_t + c0, v);
+                tmem_ld_wait();
+                uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float x0 = rounded(v[2 * k]), x1 = rounded(v[2 * k + 1]);
+                    const float q0 = (s > 0.f) ? __fdiv_rn(fabsf(x0), s) : 0.f;
+                    const float q1 = (s > 0.f) ? __fdiv_rn(fabsf(x1), s) : 0.f;
+                    uint16_t byte;
+                    asm("{\n\t.reg .b8 t;\n\t"
+                        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+                        "cvt.u16.u8 %0, t;\n\t}"
+                        : "=h"(byte)
+                        : "f"(q1), "f"(q0));
+                    uint32_t bb = byte & 0x77u;
+                    bb |= (__float_as_uint(x0) >> 31) << 3;
+                    bb |= (__float_as_uint(x1) >> 31) << 7;
+                    w[k >> 2] |= bb << (8 * (k & 3));
+                }
+                if (crow >= 0)
+                    *reinterpret_cast<uint2*>(a.keys + crow * (kDi / 2) + c0 / 2) = make_uint2(w[0], w[1]);
+            }
+            if (crow >= 0) a.key_scales[crow] = s;
+        } else if (ok) {
 #pragma unroll 1
             for (int c0 = 0; c0 < kDi; c0 += 16) {
                 uint32_t v[16];
@@ -295,6 +338,10 @@ cudaError_t launch_compress_kv(const CompressLaunch& l, cudaStream_t st) {
     a.scales = l.scales;
     a.keys = reinterpret_cast<uint8_t*>(l.keys);
     a.key_bf16 = l.key_bf16;
+    a.key_fp4 = l.key_fp4;
+    if (l.key_fp4)
+        a.key_scales = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(l.keys) +
+                                                (size_t)l.B * l.cap * CSA2_FP4KEY_CODE_BYTES);
     a.cap = l.cap;
     a.latent = reinterpret_cast<__nv_bfloat16*>(l.latent);
     a.status = l.status;

@@ -73,6 +73,7 @@ struct CompressLaunch {
     const void* Z;
     const void* w_proj;
     int key_bf16;
+    int key_fp4;            // compact 68-byte keys (two-plane buffer in keys)
     const int32_t* dst_off;
     uint8_t* codes;
     uint8_t* scales;

@@ -143,10 +143,13 @@ CSA2_API csa2_status_t csa2_quantize_kv(const void* kv, int B, int n_new, int64_
  *            multiples of 8; 16-byte aligned; finite values.
  *   r        tokens per entry, 1..64.
  *   w_proj   bf16 [128][512], row e = the weights of key channel e; 16-byte aligned.
- *   key_dtype  CSA2_DTYPE_E4M3 or CSA2_DTYPE_BF16: the storage type of k_I.
+ *   key_dtype  CSA2_DTYPE_E4M3 or CSA2_DTYPE_BF16: the storage type of k_I; or
+ *            CSA2_DTYPE_E4M3_FP4KEY: k_I is the two-plane compact-key buffer and each key
+ *            is csa2_quantize_keys_fp4's encoding of the bf16-rounded projection.
  *   dst_off  int32 [B]: entry index of sequence b's first new entry.
  *   codes, scales  the FP4 cache as in csa2_quantize_kv.
- *   k_I      [B][cap][128] in key_dtype: the indexer-key cache.
+ *   k_I      [B][cap][128] in key_dtype: the indexer-key cache (compact keys: 32-byte
+ *            aligned two-plane buffer).
  *   latent_out  nullable bf16 [B][n_new][512]: the pooled bf16 latents x.
  *   status   nullable int32 device word: CSA2_DEV_BAD_INDEX for an entry outside
  *            [0, cap) (that entry is skipped), CSA2_DEV_TIMEOUT for a bounded wait that

@@ -177,3 +177,38 @@ def test_compress_decode_shape_and_prefill_chunk():
     flips, total = _check(Cs, Zs, 2, W, dst, 65536 + 2048, codes, scales, keys, latent,
                           torch.float8_e4m3fn, 2048)
     assert flips <= 1e-3 * total
+
+
+def test_compress_writes_compact_keys():
+    """With compact 68-byte keys the compressor stores csa2_quantize_keys_fp4's encoding of
+    the bf16-rounded projection. The same call with bf16 keys yields that projection exactly
+    (the MMA is deterministic), so the compact keys are compared bit for bit with the
+    oracle's quantiser applied to it."""
+    g = _gen(36)
+    B, n_new, r, cap = 2, 300, 2, 400
+    dst = [0, 57]
+    Cs = torch.randn((B, r * n_new, 512), generator=g).to(torch.bfloat16).to(dev)
+    Zs = (torch.randn((B, r * n_new, 512), generator=g) * 2).to(torch.bfloat16).to(dev)
+    W = (torch.randn((128, 512), generator=g) * 0.06).to(torch.bfloat16).to(dev)
+    d = torch.tensor(dst, dtype=torch.int32, device=dev)
+    outs = []
+    for kind in ("bf16", "fp4"):
+        codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
+        keys = (torch.zeros((B, cap, 128), dtype=torch.bfloat16, device=dev) if kind == "bf16"
+                else C().Fp4Keys(B, cap))
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        C().compress_kv(Cs, Zs, r, W, d, codes, scales, keys, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        outs.append((codes.cpu(), scales.cpu(), keys))
+    (c0, s0, kb), (c1, s1, kf) = outs
+    assert torch.equal(c0, c1) and torch.equal(s0, s1)
+    codes = kf.codes.cpu().numpy()
+    kscale = kf.scales.cpu().numpy()
+    for b in range(B):
+        oc, os_ = O.quantize_keys_fp4(bits16(kb[b, dst[b]:dst[b] + n_new]))
+        np.testing.assert_array_equal(codes[b, dst[b]:dst[b] + n_new], oc, f"codes b={b}")
+        np.testing.assert_array_equal(kscale[b, dst[b]:dst[b] + n_new].view(np.uint32),
+                                      os_.view(np.uint32), f"scales b={b}")
+    assert codes[1, :57].sum() == 0 and kscale[0, n_new:].sum() == 0
