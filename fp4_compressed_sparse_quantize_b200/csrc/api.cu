@@ -322,8 +322,7 @@ csa2_status_t csa2_index_score_topk(csa2_mode_t mode, int B, int T, int H_I,
         qk_dtype != CSA2_DTYPE_E4M3_FP4KEY)
         return CSA2_ERR_ARG;
     const bool key_fp4 = qk_dtype == CSA2_DTYPE_E4M3_FP4KEY;
-    if (key_fp4 && (mode != CSA2_MODE_FULL || (reinterpret_cast<uintptr_t>(k_I) & 31u) != 0))
-        return mode != CSA2_MODE_FULL ? CSA2_ERR_UNSUPPORTED : CSA2_ERR_ARG;
+    if (key_fp4 && (reinterpret_cast<uintptr_t>(k_I) & 31u) != 0) return CSA2_ERR_ARG;
     if (H_I < 1 || H_I > 128) return CSA2_ERR_UNSUPPORTED;
     if (!q_I || !w || !k_I) return CSA2_ERR_ARG;
     if (!aligned16(q_I) || !aligned16(k_I) || !aligned16(w)) return CSA2_ERR_ARG;

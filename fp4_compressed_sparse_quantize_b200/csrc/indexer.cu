@@ -129,6 +129,10 @@ struct GroupCursor {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// 8 bytes (compact-key codes: one 16-code group per 16-byte slot)
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -157,7 +161,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     using L = ScanSmem<NQ, ESZ, STAGES, ACC, G, EPI, POOL, TM>;
     static_assert(ACC % EPI == 0, "each epilogue group owns fixed accumulators");
     static_assert(!GATHER || TM == 1, "gathered tiles are 128 keys");
-    static_assert(!KF4 || (ESZ == 1 && !GATHER), "compact keys: E4M3 queries, contiguous tiles");
+    static_assert(!KF4 || ESZ == 1, "compact keys take E4M3 queries");
     constexpr int kRowsT = L::kRowsT;
     constexpr int kKSteps = (128 * ESZ) / 32;         // 32 bytes of K per MMA instruction
     constexpr uint32_t kSlab = kRowsT * 128;          // bytes of one 128-byte-wide K slab
@@ -302,7 +306,16 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                     const int64_t slot = jt * kRowsT + rl;
                     int pos = (slot < p.P) ? ld_dep(pl + rl) : -1;
                     if (pos >= n_vis) pos = -1;
-                    if (pos >= 0) {
+                    if (pos >= 0 && KF4) {
+                        // compact key: 16 codes (8 bytes) per 16-byte slot, the layout the
+                        // unpacking TMA load gives the contiguous tiles; the other half is 0
+                        const uint8_t* src = p.keys + ((int64_t)b * p.cap + pos) * CSA2_FP4KEY_CODE_BYTES;
+                        const int c = lane & 7;
+                        const uint32_t off = rl * 128 + ((c ^ (rl & 7)) << 4);
+                        cp_async8(dst_u + off, src + c * 8);
+                        asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(dst_u + off + 8), "r"(0u)
+                                     : "memory");
+                    } else if (pos >= 0) {
                         const uint8_t* src = p.keys + ((int64_t)b * p.cap + pos) * (128 * ESZ);
                         for (int h = 0; h < ESZ; ++h) {
                             const int c = lane & 7;         // 16-byte chunk within 128 bytes
@@ -487,7 +500,13 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                 ks[hh] = 1.f;
                 if (KF4) {
                     const int64_t j = jt * kRowsT + hh * 128 + row;
-                    ks[hh] = (j < p.cap) ? ld_dep(p.kscale + (int64_t)(r0 / p.T) * p.cap + j) : 0.f;
+                    const int64_t kb = (int64_t)(r0 / p.T) * p.cap;
+                    if (GATHER) {   // pool slot j of query row r0 holds the entry position
+                        const int pos = (j < p.P) ? ld_dep(p.pool + (int64_t)r0 * p.P + j) : -1;
+                        ks[hh] = (pos >= 0 && pos < p.cap) ? ld_dep(p.kscale + kb + pos) : 0.f;
+                    } else {
+                        ks[hh] = (j < p.cap) ? ld_dep(p.kscale + kb + j) : 0.f;
+                    }
                 }
             }
             aborted = aborted || *abort_flag;
@@ -741,7 +760,7 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
     memset(&mk, 0, sizeof mk);
     memset(&mq, 0, sizeof mq);
     if (!make_map(&mq, a.q, (int64_t)a.rows * a.H_I, esz, NQ)) return cudaErrorInvalidValue;
-    if (a.key_fp4 && (a.gather || esz != 1)) return cudaErrorNotSupported;
+    if (a.key_fp4 && esz != 1) return cudaErrorNotSupported;
     if (!a.gather && !a.key_fp4 &&
         !make_map(&mk, a.k, (int64_t)a.B * a.cap, esz, kTileRows))
         return cudaErrorInvalidValue;
@@ -779,6 +798,14 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
 
     if (a.key_fp4) {
 #define CSA2_SCAN4(NQv, Gv, PO) return launch_scan_t<NQv, 1, Gv, false, PO, true>(mk, mq, p, st)
+#define CSA2_SCAN4G(NQv) return launch_scan_t<NQv, 1, 1, true, false, true>(mk, mq, p, st)
+        if (a.gather) {
+            if (a.G != 1) return cudaErrorNotSupported;
+            if (NQ <= 16) CSA2_SCAN4G(16);
+            if (NQ <= 32) CSA2_SCAN4G(32);
+            if (NQ <= 64) CSA2_SCAN4G(64);
+            CSA2_SCAN4G(128);
+        }
         if (a.G == 1) {
             if (a.pool_build) {
                 if (NQ <= 16) CSA2_SCAN4(16, 1, true);
@@ -793,6 +820,7 @@ cudaError_t launch_index_scan(const ScanLaunch& a, cudaStream_t st) {
         } else if (a.G == 2 && NQ <= 128 && !a.pool_build) {
             CSA2_SCAN4(128, 2, false);
         }
+#undef CSA2_SCAN4G
 #undef CSA2_SCAN4
         return cudaErrorNotSupported;
     }

@@ -78,7 +78,7 @@ typedef enum csa2_dtype {
     CSA2_DTYPE_E4M3 = 1,   /* OCP FP8 E4M3 ("fn": no infinities, max 448) */
     /* E4M3 query with compact 68-byte keys (csa2_quantize_keys_fp4): the key buffer holds
      * two planes, E2M1 codes [B][cap][64] and then fp32 scales [B][cap] starting at byte
-     * B*cap*64; its start must be 32-byte aligned. Full mode only. */
+     * B*cap*64; its start must be 32-byte aligned. Full and Reindex modes. */
     CSA2_DTYPE_E4M3_FP4KEY = 2
 } csa2_dtype_t;
 
@@ -200,8 +200,8 @@ CSA2_API csa2_status_t csa2_quantize_keys_fp4(const void* k, int B, int n_new, i
  *   B, T      sequences and query tokens per sequence (T = 1 for decode).
  *   H_I       indexer heads, 1..128.
  *   qk_dtype  storage type of q_I and k_I; CSA2_DTYPE_E4M3_FP4KEY: E4M3 q_I and compact
- *             68-byte keys (FULL only; the score is the same formula over the keys'
- *             decoded values e2m1(code) * scale).
+ *             68-byte keys (the score is the same formula over the keys' decoded values
+ *             e2m1(code) * scale).
  *   q_I       [B][T][H_I][128];  w  fp32 [B][T][H_I];  k_I  [B][cap][128] (compact keys:
  *             the two-plane buffer described at CSA2_DTYPE_E4M3_FP4KEY).
  *   n_vis0    int32 [B]: visible entries per sequence (decode, q_pos0 == NULL).

@@ -169,13 +169,40 @@ def test_prefill_with_compact_keys():
             check_topk(idx[b, t], s, np.arange(n), K, f"b={b} t={t}")
 
 
-def test_compact_keys_reject_reindex():
-    keys = C().Fp4Keys(1, 64)
-    q_I = torch.zeros((1, 1, 64, 128), dtype=torch.float8_e4m3fn, device=dev)
-    w = torch.zeros((1, 1, 64), device=dev)
-    idx = torch.empty((1, 1, 8), dtype=torch.int32, device=dev)
-    ws = C().new_workspace(C().workspace_bytes(0, 1, 1, 64, 64, 8))
-    with pytest.raises(C().Csa2Error):
-        C().index_score_topk("reindex", q_I, w, keys, 8, idx, ws,
-                             n_vis0=torch.tensor([64], dtype=torch.int32, device=dev),
-                             pool_in=torch.zeros((1, 1, 16), dtype=torch.int32, device=dev))
+def test_reindex_with_compact_keys():
+    """Reindex over compact keys: a second layer's query rescored inside the oracle's pool
+    (pool rows gathered with 8-byte copies into the unpacked operand layout, each key's
+    scale looked up through its pool position)."""
+    g = _gen(45)
+    B, n, H_I, K, nblk = 2, 20000, 64, 512, 512
+    k = _keys_bf16(B, n, g)
+    keys, _ = _compact(k, n, [0, 0])
+    codes = keys.codes.cpu().numpy()
+    kscale = keys.scales.cpu().numpy()
+    q1 = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn)
+    w1 = torch.rand((B, 1, H_I), generator=g)
+    q2 = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn)
+    w2 = torch.rand((B, 1, H_I), generator=g)
+    n_list = [n, n - 13]
+    pool_o = np.stack([O.pool(_oracle_scores(bits8(q1[b, 0]), w1[b, 0].numpy(), codes[b], kscale[b],
+                                             n_list[b])[0], nblk) for b in range(B)])[:, None, :]
+    P = pool_o.shape[-1]
+    idx = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+    sc = torch.zeros((B, 1, P), dtype=torch.float32, device=dev)
+    ws = C().new_workspace(C().workspace_bytes(0, B, 1, H_I, P, K))
+    C().index_score_topk("reindex", q2.to(dev), w2.to(dev), keys, K, idx, ws,
+                         n_vis0=torch.tensor(n_list, dtype=torch.int32, device=dev),
+                         pool_in=torch.from_numpy(pool_o.astype(np.int32)).to(dev), scores_out=sc)
+    torch.cuda.synchronize()
+    assert C().read_device_status(ws) == 0
+    idx = idx.cpu().numpy()
+    sc = sc.cpu().numpy()
+    for b in range(B):
+        slots = np.nonzero(pool_o[b, 0] >= 0)[0]
+        ids = pool_o[b, 0][slots]
+        s2 = O.index_scores_fp4key(bits8(q2[b, 0]), w2[b, 0].numpy(), codes[b], kscale[b], rows=ids)
+        qd = O.e4m3_array_to_f64(bits8(q2[b, 0]).ravel()).reshape(H_I, 128)
+        kd = O.dequant_keys_fp4(codes[b][ids], kscale[b][ids])
+        mag = np.abs(kd) @ np.abs(qd).T @ w2[b, 0].numpy().astype(np.float64)
+        np.testing.assert_array_less(np.abs(sc[b, 0, slots] - s2), 2e-6 * mag + 1e-30)
+        check_topk(idx[b, 0], s2, ids, K, f"reindex b={b}")
