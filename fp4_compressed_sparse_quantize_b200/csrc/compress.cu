@@ -11,18 +11,20 @@
 //   codes, scales = FP4 quantize-on-write of x[j] (as csa2_quantize_kv)
 //   k[j][e] = sum_d W[e][d] * x[j][d], stored as E4M3 (RNE, saturating) or bf16.
 //
-// One CTA per 128 entries (the MMA's M), 8 warps:
-//  1. pooling: warp w takes entries w, w+8, ...; lane l owns channels [16l, 16l+16), i.e.
+// One CTA per 32 entries (the MMA's M is 128; rows 32.. are computed and discarded, the
+// projection being tiny next to the pooling's loads), 8 warps:
+//  1. pooling: warp w takes entries w, w+8, w+16, w+24; lane l owns channels [16l, 16l+16), i.e.
 //     one FP4 scale block. Per token the warp reads the 1 KiB latent and logit rows in one
-//     coalesced sweep; the softmax (max, then exp-weighted sums) runs in fp32 per channel.
+//     coalesced sweep (for up to 4 tokens, all of an entry's rows in one batch of loads);
+//     the softmax (max, then exp-weighted sums) runs in fp32 per channel.
 //     The bf16 latent goes to the global FP4 cache (codes + scale, this lane's block) and
 //     into shared memory as the MMA's A operand (K-major, 128-byte swizzle, 8 slabs of
 //     64 channels);
 //  2. projection: one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
 //     M = 128 entries, N = 64 key channels, K = 512, twice (W's two halves are TMA-loaded
 //     in turn into one 64 KiB buffer);
-//  3. epilogue: warps 0-3 read their TMEM lane quadrant (one entry per thread), convert
-//     and store the 128-channel key row.
+//  3. epilogue: warp 0 reads TMEM lanes 0-31 (one entry per thread), converts and stores
+//     the 128-channel key row.
 #include "csa2_common.cuh"
 #include "csa2_internal.h"
 #include "fp4_block.cuh"
@@ -30,7 +32,8 @@
 namespace csa2 {
 namespace {
 
-constexpr int kM = 128;                    // entries per CTA
+constexpr int kM = 128;                    // MMA rows (A operand rows in shared memory)
+constexpr int kE = 32;                     // entries per CTA (rows kE.. of the MMA unused)
 constexpr int kD = 512;                    // latent channels
 constexpr int kDi = 128;                   // indexer-key channels
 constexpr int kThreads = 256;
@@ -105,8 +108,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- 1. pooling, FP4 write and the A operand ----------------------------------------
     const int64_t total = (int64_t)a.B * a.n_new;
-    for (int m = warp; m < kM; m += kThreads / 32) {
-        const int64_t g = (int64_t)blockIdx.x * kM + m;
+    if (threadIdx.x >= kE && threadIdx.x < kM) row_dst[threadIdx.x] = -1;
+    for (int m = warp; m < kE; m += kThreads / 32) {
+        const int64_t g = (int64_t)blockIdx.x * kE + m;
         int64_t crow = -1;
         int b = 0, j = 0;
         if (g < total) {
@@ -128,27 +132,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             float zmax[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) zmax[k] = -INFINITY;
-            for (int t = 0; t < a.r; ++t) {
-                const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
-                float z[16];
-                bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
-            }
             float den[16], num[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) den[k] = num[k] = 0.f;
-            for (int t = 0; t < a.r; ++t) {
-                const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
-                const uint4* cp = reinterpret_cast<const uint4*>(cc + (tok0 + t) * a.ld);
-                float z[16], c[16];
-                bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
-                bf16x16_to_float(ld_dep(cp), ld_dep(cp + 1), c);
+            if (a.r <= 4) {
+                // up to 4 tokens: every latent and logit row of the entry in one batch of loads
+                uint4 zr[4][2], cr[4][2];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float e = expf(z[k] - zmax[k]);
-                    den[k] += e;
-                    num[k] = fmaf(e, c[k], num[k]);
+                for (int t = 0; t < 4; ++t) {
+                    if (t < a.r) {
+                        const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
+                        const uint4* cp = reinterpret_cast<const uint4*>(cc + (tok0 + t) * a.ld);
+                        zr[t][0] = ld_dep(zp);
+                        zr[t][1] = ld_dep(zp + 1);
+                        cr[t][0] = ld_dep(cp);
+                        cr[t][1] = ld_dep(cp + 1);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (t < a.r) {
+                        float z[16];
+                        bf16x16_to_float(zr[t][0], zr[t][1], z);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (t < a.r) {
+                        float z[16], c[16];
+                        bf16x16_to_float(zr[t][0], zr[t][1], z);
+                        bf16x16_to_float(cr[t][0], cr[t][1], c);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const float e = expf(z[k] - zmax[k]);
+                            den[k] += e;
+                            num[k] = fmaf(e, c[k], num[k]);
+                        }
+                    }
+                }
+            } else {
+                for (int t = 0; t < a.r; ++t) {
+                    const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
+                    float z[16];
+                    bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
+                }
+                for (int t = 0; t < a.r; ++t) {
+                    const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
+                    const uint4* cp = reinterpret_cast<const uint4*>(cc + (tok0 + t) * a.ld);
+                    float z[16], c[16];
+                    bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
+                    bf16x16_to_float(ld_dep(cp), ld_dep(cp + 1), c);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float e = expf(z[k] - zmax[k]);
+                        den[k] += e;
+                        num[k] = fmaf(e, c[k], num[k]);
+                    }
                 }
             }
 #pragma unroll
@@ -217,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
 
     // ---- 3. epilogue: one entry per thread of warps 0-3 ------------------------------------
-    if (warp < 4) {
+    if (warp < (kE + 31) / 32) {
         bool ok = !*stuck && mbar_wait(mdone1, 0, a.status);
         ok = __all_sync(0xffffffffu, ok);   // tcgen05.ld below is warp-collective
         if (!ok) *stuck = 1;
@@ -348,7 +391,7 @@ cudaError_t launch_compress_kv(const CompressLaunch& l, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(compress_kv_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDynBytes);
     if (e != cudaSuccess) return e;
-    const int64_t grid = (entries + kM - 1) / kM;
+    const int64_t grid = (entries + kE - 1) / kE;
     return launch_pdl(compress_kv_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)kDynBytes,
                       st, mw, a);
 }
