@@ -102,5 +102,31 @@ def test_host_validation_rejects_without_launch(lib):
     assert q(P, 1, 1, 500, 512, P, P, P, 10, None, None) == csa2.ERR_ARG   # ld_kv < 512
     assert q(odd, 1, 1, 512, 512, P, P, P, 10, None, None) == csa2.ERR_ARG
     assert q(None, 0, 1, 512, 512, P, P, P, 10, None, None) == csa2.OK     # nothing to do
+    # compressor + projection: (B, n_new, r, C, Z, ld, bstride, w_proj, key_dtype, dst_off,
+    # codes, scales, k_I, cap, latent_out, status, stream)
+    c = lib.csa2_compress_kv
+    ok = (1, 4, 2, P, P, 512, 8 * 512, P, 1, P, P, P, P, 100, None, None, None)
+
+    def cz(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return c(*a)
+    assert cz(_2=0) == csa2.ERR_ARG and cz(_2=65) == csa2.ERR_ARG      # ratio outside 1..64
+    assert cz(_5=504) == csa2.ERR_ARG                                   # ld < 512
+    assert cz(_3=odd) == csa2.ERR_ARG and cz(_7=None) == csa2.ERR_ARG   # misaligned C, no W
+    assert cz(_8=7) == csa2.ERR_ARG                                     # unknown key type
+    assert cz(_8=2, _12=_ptr(0x10010)) == csa2.ERR_ARG                  # compact keys: 32-B aligned
+    assert cz(_14=odd) == csa2.ERR_ARG                                  # misaligned latent_out
+    assert cz(_1=0) == csa2.OK                                          # nothing to do
+    # compact-key quantiser: (k, B, n_new, ld, bstride, dst_off, keys, cap, status, stream)
+    kq = lib.csa2_quantize_keys_fp4
+    assert kq(P, 1, 4, 120, 1024, P, P, 100, None, None) == csa2.ERR_ARG   # ld < 128
+    assert kq(odd, 1, 4, 128, 1024, P, P, 100, None, None) == csa2.ERR_ARG
+    assert kq(P, 1, 4, 128, 1024, P, _ptr(0x10010), 100, None, None) == csa2.ERR_ARG
+    assert kq(P, 1, 0, 128, 1024, P, P, 100, None, None) == csa2.OK
+    # compact keys in index_score_topk: the key buffer must be 32-byte aligned
+    assert call(dt=2, k=_ptr(0x10010)) == csa2.ERR_ARG
+    assert call(dt=3) == csa2.ERR_ARG
     assert lib.csa2_read_device_status(None, None, None) == csa2.ERR_ARG
     assert lib.csa2_debug_bounded_wait(P, 0, None) == csa2.ERR_ARG
