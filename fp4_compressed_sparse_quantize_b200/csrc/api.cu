@@ -476,7 +476,7 @@ static csa2_status_t attn_common(bool prefill, int B, int T, int H, const void* 
     if (H > 64 || W > 1024 || K > 65536) return CSA2_ERR_UNSUPPORTED;
     const bool part = o_part != nullptr;
     if (part) {
-        if (!ml_part || !aligned16(o_part) || prefill || K + W < 1) return CSA2_ERR_ARG;
+        if (!ml_part || !aligned16(o_part) || prefill) return CSA2_ERR_ARG;
         out = o_part;   // only checked for alignment below; the result goes to o_part/ml_part
     }
     if (!q || !out || !ws) return !ws ? CSA2_ERR_WORKSPACE : CSA2_ERR_ARG;

@@ -1,4 +1,4 @@
-// Fused gather + exact FP4 dequantisation + joint sparse / sliding-window attention on the
+// Decode: gather + exact FP4 dequantisation + joint sparse / sliding-window attention on the
 // 5th-generation tensor cores (tcgen05, TMEM accumulators).
 //
 // "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression" (AI summary),
@@ -21,23 +21,18 @@
 // accumulated together (~22-bit probabilities: one fp16 rounding of P alone costs ~2e-3 of
 // the output RMS on heavy-tailed channels). All accumulation is fp32 in TMEM.
 //
-// One CTA owns one query row (all heads, padded to 64) and a range of 128-row chunks of
-// the concatenated [selected entries | window rows] list:
-//   1. every thread gathers its share of the chunk's rows (FP4 codes + scales, or E4M3
-//      window rows), dequantises to fp16 and stores them into X [128 rows x 512] laid out
-//      in 128-byte-swizzled slabs of 64 channels; the query Q [64 x 512] likewise;
-//   2. one thread issues S^T = X Q^T (M = 128 rows, N = 64 heads, K = 512): 32 tcgen05.mma;
-//   3. four warps read S^T from TMEM (one row per thread) into a transposed shared tile;
-//      256 threads take (head, 32-row quarter) slices for the softmax and write P (high and
-//      low fp16 parts) as the K-major B operand [64 heads x 128 rows];
-//   4. one thread issues O^T += X^T P^T (M = 128 channels per tile, 4 tiles, N = 64 heads,
-//      K = 128 rows) reading the SAME X tile as an MN-major A operand;
-//   5. eight warps read O^T from TMEM (one channel per thread) and write the output, or
-//      the (max, sum, output) partial that a merge kernel combines when the rows of a query
-//      were split over several CTAs.
-// A CTA with several chunks (prefill) first sweeps them for the exact per-head maximum,
-// then sweeps again to accumulate P x V, so no accumulator is ever rescaled.
+// Kernels (prefill has its own kernel, attention_prefill.cu):
+//   attn_stage_kernel   one warp per row: every selected FP4 row and window row of every
+//                       query dequantised to fp16 rows [Q][K + W][512], and each query's
+//                       heads rescaled to fp16 with their logit factors;
+//   attn_decode_kernel  one CTA per (query, split of at most 160 rows): TMA loads of the
+//                       staged rows and query, S = Q X^T with the 64 heads as M, softmax,
+//                       [O_hi; O_lo] = [P_hi; P_lo] X, and either the splits' merge inside
+//                       a thread-block cluster (distributed shared memory) or (max, sum,
+//                       output) partials that attn_combine_kernel merges;
+//   attn_empty_kernel   queries with no row at all (K + W == 0).
 #include <cuda.h>
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <cudaTypedefs.h>
@@ -47,7 +42,6 @@
 
 namespace csa2 {
 
-constexpr int kRows = 128;     // rows per chunk (MMA M of S^T, K of O^T)
 constexpr int kD = 512;        // latent channels
 constexpr int kHeads = 64;     // heads per CTA (MMA N), padded
 
@@ -68,7 +62,7 @@ struct TcAttnDev {
     float* out;
     float* partial;          // O [Q * nsplit][H][512]
     float* partial_ml;       // (m, l) [Q * nsplit][2][H]
-    int nsplit, nchunks, chunks_per_split;
+    int nsplit;
     bool part;               // decode: write (m, l, unnormalised O) partials even for one split
     int32_t* status;
     // staged decode: rows / query already dequantised by attn_stage_kernel
@@ -76,26 +70,10 @@ struct TcAttnDev {
     const float* st_qf;        // [Q][64] logit factors
 };
 
+// one 64-channel slab of the query operand: [64 heads x 128 bytes]
 struct TcSmem {
-    static constexpr int kX = 0;                          // 8 slabs x [128 rows x 128 B]
-    static constexpr int kXSlab = kRows * 128;            // 16 KiB
-    static constexpr int kQ = kX + 8 * kXSlab;            // 8 slabs x [64 rows x 128 B]
     static constexpr int kQSlab = kHeads * 128;           // 8 KiB
-    // after S^T is computed the Q region holds the transposed logits and P
-    static constexpr int kS = kQ;                         // fp32 [64 heads][128 rows]
-    static constexpr int kPhi = kS + kHeads * kRows * 4;  // 2 slabs x [64 x 128 B]
-    static constexpr int kPlo = kPhi + 2 * kQSlab;
-    static constexpr int kMisc = kQ + 8 * kQSlab;
-    static constexpr int kQf = kMisc;                     // 64 floats
-    static constexpr int kM = kQf + 256;                  // 64 floats
-    static constexpr int kL = kM + 256;                   // 64 floats
-    static constexpr int kValid = kL + 256;               // 128 ints
-    static constexpr int kBar = kValid + 512;             // 3 mbarriers
-    static constexpr int kTmem = kBar + 24;
-    static constexpr int kBytes = kTmem + 16;
-    static constexpr int kAlloc = kBytes + 1024;
 };
-static_assert(TcSmem::kPlo + 2 * TcSmem::kQSlab <= TcSmem::kMisc, "P fits in the Q region");
 
 // byte offset of 16-byte chunk `c` (0..7) of row `r` inside one 128-byte-wide slab
 __device__ __forceinline__ uint32_t slab_off(int r, int c) {
@@ -119,135 +97,6 @@ __device__ __forceinline__ uint32_t e2m1x2_to_h2_tc(uint32_t byte) {
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// Logit tile S[r][h] (fp32, 64 heads per row) with the 16-byte chunk (4 heads) index XOR-ed
-// by ((r / 32) * 2) ^ (r mod 8): one thread per row writes it with 16-byte stores, and the
-// (head, 32-row quarter)-per-thread reads of the softmax touch 32 distinct banks.
-__device__ __forceinline__ int s_swz(int r) { return ((r >> 5) << 1) ^ (r & 7); }
-__device__ __forceinline__ int s_idx(int h, int r) {
-    return r * kHeads + ((((h >> 2) ^ s_swz(r)) & 15) << 2) + (h & 3);
-}
-
-// Gather + dequantise rows [ch*128, ch*128+128) of query row `qrow` into X (all 256 threads:
-// two threads per row, 16 groups of 16 channels each). Records per-row validity.
-__device__ __forceinline__ void load_chunk(const TcAttnDev& a, int qrow, int b, int t, int ch,
-                                           uint32_t sX, int* rvalid) {
-    const int tid = threadIdx.x;
-    const int i = tid >> 1, part = tid & 1;      // row within the chunk, half of its channels
-    const int g = ch * kRows + i;
-    int kind = 0;
-    const uint8_t* src_codes = nullptr;
-    const uint8_t* src_scales = nullptr;
-    const uint8_t* src_swa = nullptr;
-    if (g < a.K) {
-        const int32_t e = ld_dep(a.idx + (int64_t)qrow * a.K + g);
-        if (e >= 0 && e < a.cap) {
-            kind = 1;
-            const int64_t ent = (int64_t)b * a.cap + e;
-            src_codes = a.codes + ent * CSA2_ENTRY_CODE_BYTES + part * 128;
-            src_scales = a.scales + ent * CSA2_ENTRY_SCALE_BYTES + part * 16;
-        } else if (e != -1 && part == 0) {
-            set_status(a.status, CSA2_DEV_BAD_INDEX);
-        }
-    } else if (g < a.K + a.W) {
-        const int v = g - a.K;   // window row 0..W-1, oldest first
-        int64_t srow;
-        bool ok;
-        if (!a.prefill) {
-            const int nv = a.swa_valid ? ld_dep(a.swa_valid + b) : a.W;
-            ok = v >= a.W - nv;
-            srow = (int64_t)b * a.W + v;
-        } else {
-            const int64_t rw = t + v;
-            const int64_t pos =
-                (a.q_pos0 ? (int64_t)ld_dep(a.q_pos0 + b) : (int64_t)(a.W - 1)) - (a.W - 1) + rw;
-            ok = pos >= 0;
-            srow = (int64_t)b * (a.W - 1 + a.T) + rw;
-        }
-        if (ok) {
-            kind = 2;
-            src_swa = a.swa + srow * kD + part * 256;
-        }
-    }
-    if (part == 0) rvalid[i] = kind;
-    // issue every load of this thread before converting
-    uint4 raw[16];
-    uint4 sc4 = make_uint4(0, 0, 0, 0);
-    if (kind == 1) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) raw[k] = ld_dep(reinterpret_cast<const uint4*>(src_codes) + k);
-        sc4 = ld_dep(reinterpret_cast<const uint4*>(src_scales));
-    } else if (kind == 2) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) raw[k] = ld_dep(reinterpret_cast<const uint4*>(src_swa) + k);
-    }
-    const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
-    // 16 groups of 16 channels: group gl covers channels 256*part + 16*gl
-#pragma unroll
-    for (int gl = 0; gl < 16; ++gl) {
-        uint32_t hv[8];
-        if (kind == 1) {
-            const uint4 cb = raw[gl >> 1];
-            const uint32_t w0 = (gl & 1) ? cb.z : cb.x, w1 = (gl & 1) ? cb.w : cb.y;
-            const uint32_t sbyte = (scw[gl >> 2] >> (8 * (gl & 3))) & 0xFFu;
-            const __half2 s2 = __half2half2(__float2half_rn(e4m3_to_float((uint8_t)sbyte)));
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t byte = ((k < 4 ? w0 : w1) >> (8 * (k & 3))) & 0xFFu;
-                uint32_t h2 = e2m1x2_to_h2_tc(byte);
-                hv[k] = h2_bits(__hmul2(*reinterpret_cast<__half2*>(&h2), s2));
-            }
-        } else if (kind == 2) {
-            const uint4 eb = raw[gl];
-            const uint32_t ew[4] = {eb.x, eb.y, eb.z, eb.w};
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                hv[k] = h2_bits(e4m3x2_to_half2((uint16_t)(ew[k >> 1] >> (16 * (k & 1)))));
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) hv[k] = 0u;
-        }
-        const int c0 = 256 * part + 16 * gl;         // first channel of the group
-        const uint32_t slab = sX + (c0 >> 6) * TcSmem::kXSlab;
-        const int cc = (c0 & 63) >> 3;               // 16-byte chunk within the slab row
-        st_shared_v4(slab + slab_off(i, cc), hv[0], hv[1], hv[2], hv[3]);
-        st_shared_v4(slab + slab_off(i, cc + 1), hv[4], hv[5], hv[6], hv[7]);
-    }
-}
-
-// S^T = X Q^T into TMEM columns [0, 64)
-__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sX, uint32_t sQ) {
-    constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u);
-#pragma unroll 4
-    for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint64_t ad = sw128_desc(sX + (kk >> 2) * TcSmem::kXSlab + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = sw128_desc(sQ + (kk >> 2) * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
-        mma_f16(tmem, ad, bd, idesc, kk > 0);
-    }
-}
-
-// O^T (+)= X^T P^T for both P parts into TMEM columns [64, 320)
-__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t sX, uint32_t sPhi,
-                                         uint32_t sPlo, bool accumulate) {
-    constexpr uint32_t idesc = make_idesc(kRows, kHeads, 0u, 0u, /*a MN-major*/ 1u, 0u);
-#pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-            const uint32_t sP = part ? sPlo : sPhi;
-#pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk) {
-                // A: channels [128m, 128m+128) x rows [16kk, 16kk+16), MN-major: the two
-                // 64-channel halves are adjacent slabs (LBO), 8-row groups 1 KiB apart (SBO)
-                const uint64_t ad =
-                    sw128_desc(sX + (2 * m) * TcSmem::kXSlab + kk * 16 * 128, TcSmem::kXSlab, 1024);
-                const uint64_t bd =
-                    sw128_desc(sP + (kk >> 2) * TcSmem::kQSlab + (kk & 3) * 32, 16, 1024);
-                mma_f16(tmem + kHeads + 64 * m, ad, bd, idesc,
-                        (accumulate || part > 0 || kk > 0) ? 1u : 0u);
-            }
-        }
-    }
-}
 
 // Decode pre-pass: every selected main-KV row and window row of every query, dequantised to
 // fp16 rows [Q][K + W][512] (exact), plus each query's heads rescaled to fp16 [Q][64][512] and
@@ -343,314 +192,6 @@ __global__ void __launch_bounds__(256) attn_stage_kernel(const TcAttnDev a, __ha
     if (lane == 0) qfg[b * kHeads + h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
 }
 
-template <bool STAGED>
-__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                                                         const __grid_constant__ CUtensorMap tmap_q,
-                                                         const __grid_constant__ CUtensorMap tmap_o,
-                                                         const TcAttnDev a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    using L = TcSmem;
-    const uint32_t sX = smem_u32(sm + L::kX), sQ = smem_u32(sm + L::kQ),
-                   sPhi = smem_u32(sm + L::kPhi), sPlo = smem_u32(sm + L::kPlo);
-    float* Ssm = reinterpret_cast<float*>(sm + L::kS);
-    float* qf = reinterpret_cast<float*>(sm + L::kQf);
-    float* m_s = reinterpret_cast<float*>(sm + L::kM);
-    float* l_s = reinterpret_cast<float*>(sm + L::kL);
-    int* rvalid = reinterpret_cast<int*>(sm + L::kValid);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::kTmem);
-
-    grid_dep_launch();
-    grid_dep_wait();
-    const int qrow = blockIdx.x, split = blockIdx.y;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = qrow / a.T, t = qrow - b * a.T;
-    const int c_begin = split * a.chunks_per_split;
-    const int c_end = min(a.nchunks, c_begin + a.chunks_per_split);
-
-    // staged rows and query of chunk ch: 8 + 8 TMA boxes of [rows x 64 channels] on bar[2]
-    auto issue_loads = [&](int ch) {
-        mbar_arrive_expect_tx(&bar[2], 8u * L::kXSlab + 8u * L::kQSlab);
-        const int32_t xrow = qrow * (a.K + a.W) + ch * kRows;
-#pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-            tma_load_2d(sm + L::kX + j * L::kXSlab, &tmap_x, &bar[2], 64 * j, xrow);
-            tma_load_2d(sm + L::kQ + j * L::kQSlab, &tmap_q, &bar[2], 64 * j, qrow * kHeads);
-        }
-    };
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        mbar_init(&bar[2], 1);
-        fence_mbar_init();
-        if constexpr (STAGED) issue_loads(c_begin);   // overlaps the TMEM allocation below
-    }
-    // the first chunk's row kinds and logit factors, fetched before the setup barrier
-    int pre_valid = 0;
-    float pre_qf = 0.f;
-    if constexpr (STAGED) {
-        const int r0 = c_begin * kRows + tid;
-        if (tid < kRows && r0 < a.K + a.W)
-            pre_valid = ld_dep(a.st_valid + (int64_t)qrow * (a.K + a.W) + r0);
-        if (tid < kHeads) pre_qf = ld_dep(a.st_qf + qrow * kHeads + tid);
-    }
-    bool first_chunk = true;
-    if (warp == 0) tmem_alloc(tmem_holder, 512);
-    if (tid < kHeads) m_s[tid] = -INFINITY;
-
-    // ---- query: per-head power-of-two rescale into fp16, K-major swizzled slabs --------
-    // (1) the raw bf16 rows [64 heads x 1 KiB] are fetched asynchronously into the Q tile,
-    // overlapping the row gather; (2) every thread reads its (head, 128-channel quarter) into
-    // registers, the block syncs, and the scaled fp16 values are written back swizzled.
-    auto q_prefetch = [&]() {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int c = tid + 256 * k;          // 16-byte chunk of the 64 KiB tile
-            const int h = c >> 6, off = (c & 63) * 16;
-            const uint32_t dst = sQ + h * 1024 + off;
-            if (h < a.H)
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                             "l"(reinterpret_cast<const uint8_t*>(a.q + ((int64_t)qrow * a.H + h) * kD) + off)
-                             : "memory");
-            else
-                st_shared_v4(dst, 0u, 0u, 0u, 0u);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    auto q_convert = [&]() {
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();
-        const int h = tid >> 2, qq = tid & 3;   // channels [128 qq, 128 qq + 128) of head h
-        uint4 raw[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-            raw[k] = *reinterpret_cast<const uint4*>(sm + L::kQ + h * 1024 + qq * 256 + k * 16);
-        float amax = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)),
-                                         fabsf(__uint_as_float(w4[e] & 0xFFFF0000u))));
-        }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        int shift = 0;
-        if (amax > 0.f) {
-            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-            shift = min(126, max(-126, 14 - ex));
-        }
-        const float mul = __int_as_float((127 + shift) << 23);   // 2^shift, exact
-        __syncthreads();   // every raw read is done before the swizzled writes begin
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-            uint32_t hw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                hw[e] = h2_bits(__floats2half2_rn(__uint_as_float(w4[e] << 16) * mul,
-                                                  __uint_as_float(w4[e] & 0xFFFF0000u) * mul));
-            // channels 128 qq + 8 k .. +8: slab 2 qq + k / 8, chunk k % 8
-            st_shared_v4(sQ + (2 * qq + (k >> 3)) * L::kQSlab + slab_off(h, k & 7), hw[0], hw[1],
-                         hw[2], hw[3]);
-        }
-        if (qq == 0) qf[h] = a.scale * 1.4426950408889634f * __int_as_float((127 - shift) << 23);
-    };
-
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
-    const uint32_t quad = (uint32_t)(32 * (warp & 3)) << 16;
-    uint32_t phase[3] = {0u, 0u, 0u};
-    bool ok = true;
-
-    // wait on barrier i (all threads), bounded
-    auto wait_bar = [&](int i) {
-        if (ok && !mbar_wait(&bar[i], phase[i], a.status)) ok = false;
-        phase[i] ^= 1u;
-    };
-
-    // S^T for chunk ch -> transposed logits Ssm[h][r] (log2 domain, -inf for empty rows)
-    auto scores = [&](int ch) {
-        if constexpr (STAGED) {
-            // rows and query already in fp16 (the first chunk's loads went out at the start)
-            if (first_chunk) {
-                if (tid < kRows) rvalid[tid] = pre_valid;
-                if (tid < kHeads) qf[tid] = pre_qf;
-                first_chunk = false;
-            } else {
-                if (tid == 0) issue_loads(ch);
-                if (tid < kRows) {
-                    const int r = ch * kRows + tid;
-                    rvalid[tid] =
-                        (r < a.K + a.W) ? ld_dep(a.st_valid + (int64_t)qrow * (a.K + a.W) + r) : 0;
-                }
-                if (tid < kHeads) qf[tid] = ld_dep(a.st_qf + qrow * kHeads + tid);
-            }
-            wait_bar(2);
-            __syncthreads();
-        } else {
-            q_prefetch();
-            load_chunk(a, qrow, b, t, ch, sX, rvalid);
-            q_convert();
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncthreads();
-        }
-        if (tid == 0) {
-            tc_fence_after();
-            issue_s(tmem, sX, sQ);
-            mma_commit(&bar[0]);
-        }
-        wait_bar(0);
-        tc_fence_after();
-        if (warp < 4) {
-            const int r = 32 * warp + lane;
-            const bool valid = rvalid[r] != 0;
-            uint32_t v[4][16];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld16(tmem + quad + 16 * c, v[c]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {   // heads 4 c4 .. 4 c4 + 3
-                float4 o;
-                const float4 f = *reinterpret_cast<const float4*>(qf + 4 * c4);
-                o.x = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 0]) * f.x : -INFINITY;
-                o.y = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 1]) * f.y : -INFINITY;
-                o.z = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 2]) * f.z : -INFINITY;
-                o.w = valid ? __uint_as_float(v[c4 >> 2][4 * (c4 & 3) + 3]) * f.w : -INFINITY;
-                *reinterpret_cast<float4*>(Ssm + r * kHeads + (((c4 ^ s_swz(r)) & 15) << 2)) = o;
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-    };
-
-    const int h = tid >> 2, qq = tid & 3;   // softmax slice: head h, rows [32 qq, +32)
-    float l_acc = 0.f;
-
-    // ---- pass 1 (several chunks only): exact per-head maximum ---------------------------
-    if (c_end - c_begin > 1) {
-        for (int ch = c_begin; ch < c_end; ++ch) {
-            scores(ch);
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, Ssm[s_idx(h, 32 * qq + j)]);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            if (qq == 0) m_s[h] = fmaxf(m_s[h], mx);
-            __syncthreads();
-        }
-    }
-
-    // ---- pass 2: softmax numerators and P x V -------------------------------------------
-    for (int ch = c_begin; ch < c_end; ++ch) {
-        scores(ch);
-        float sv[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sv[j] = Ssm[s_idx(h, 32 * qq + j)];
-        float m;
-        if (c_end - c_begin > 1) {
-            m = m_s[h];
-        } else {
-            m = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) m = fmaxf(m, sv[j]);
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        }
-        const float base = (m == -INFINITY) ? 0.f : m;
-        uint32_t hi[16], lo[16];
-        float ls = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float p0 = exp2f(sv[2 * j] - base), p1 = exp2f(sv[2 * j + 1] - base);
-            ls += p0 + p1;
-            const __half2 ph = __floats2half2_rn(p0, p1);
-            hi[j] = h2_bits(ph);
-            lo[j] = h2_bits(__floats2half2_rn(p0 - __low2float(ph), p1 - __high2float(ph)));
-        }
-        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-        l_acc += ls;
-        if (qq == 0 && c_end - c_begin == 1) m_s[h] = m;
-        __syncthreads();   // every thread has read its logits before P overwrites the tile
-        // P[h][rows 32qq .. 32qq+31]: slab qq/2, chunks 4(qq%2) .. +4, row h
-        {
-            const uint32_t ohi = sPhi + (qq >> 1) * L::kQSlab, olo = sPlo + (qq >> 1) * L::kQSlab;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int cc = 4 * (qq & 1) + c;
-                st_shared_v4(ohi + slab_off(h, cc), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                st_shared_v4(olo + slab_off(h, cc), lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-            }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            issue_pv(tmem, sX, sPhi, sPlo, ch > c_begin);
-            mma_commit(&bar[1]);
-        }
-        wait_bar(1);
-        tc_fence_after();
-        __syncthreads();   // X and the Q region may be rewritten by the next chunk
-    }
-    if (qq == 0) {
-        l_s[h] = l_acc;
-        qf[h] = l_acc > 0.f ? 1.f / l_acc : 0.f;   // the logit factors are no longer needed
-    }
-    __syncthreads();
-
-    // ---- epilogue: O^T tiles (warps 0-3: tiles 0,1; warps 4-7: tiles 2,3) -> shared memory
-    // as [heads][128 channels] fp32 per tile (the X region is free), then one bulk tensor
-    // store per tile: the normalised output (one split) or the partial output of this split
-    float* osm = reinterpret_cast<float*>(sm + L::kX);
-    const int oblk = a.nsplit == 1 ? qrow : qrow * a.nsplit + split;
-    if (ok) {
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-            const int tile = 2 * (warp >> 2) + tt;
-            const int cl = 32 * (warp & 3) + lane;   // channel within the tile
-            uint32_t v[4][16];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) tmem_ld16(tmem + quad + kHeads + 64 * tile + 16 * k, v[k]);
-            tmem_ld_wait();
-            float* dst = osm + tile * (kHeads * 128) + cl;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int hh = 16 * k + e;
-                    float x = __uint_as_float(v[k][e]);
-                    if (a.nsplit == 1) x *= qf[hh];
-                    dst[hh * 128] = x;
-                }
-        }
-        if (a.nsplit > 1 && warp == 0) {
-            float* ml = a.partial_ml + (int64_t)oblk * 2 * a.H;
-            for (int hh = lane; hh < a.H; hh += 32) {
-                ml[hh] = m_s[hh];
-                ml[a.H + hh] = l_s[hh];
-            }
-        }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && ok) {
-#pragma unroll 1
-        for (int tile = 0; tile < 4; ++tile)
-            tma_store_3d(&tmap_o, osm + tile * (kHeads * 128), 128 * tile, 0, oblk);
-        bulk_commit();
-        bulk_wait_all();
-    }
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
-}
 
 // ---- decode: one CTA per (query, split of at most 160 rows) ------------------------------
 // The rows of a decode query are split evenly (a multiple of 32 per split, at most
@@ -1039,6 +580,25 @@ __global__ void __launch_bounds__(256, 1) attn_decode_kernel(const __grid_consta
     if (warp == 0 && !mma_stuck) tmem_dealloc(tmem, 512);
 }
 
+// Queries with no row at all (K + W == 0): the softmax of an empty set contributes nothing,
+// so the output is zero; a partial result is (maximum -inf, sum 0, output 0), which the
+// partial merge weighs by zero.
+__global__ void __launch_bounds__(256) attn_empty_kernel(float* o, float* ml, int Q, int H) {
+    grid_dep_launch();
+    grid_dep_wait();
+    const int64_t n4 = (int64_t)Q * H * kD / 4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x)
+        reinterpret_cast<float4*>(o)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ml)
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)Q * H;
+             i += (int64_t)gridDim.x * blockDim.x) {
+            const int64_t q = i / H, h = i - q * H;
+            ml[q * 2 * H + h] = -INFINITY;
+            ml[q * 2 * H + H + h] = 0.f;
+        }
+}
+
 // [rows][512] fp16 matrix, box = 64 channels x box_rows, 128-byte swizzle
 static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
     auto enc = tensor_map_encoder();
@@ -1052,18 +612,6 @@ static bool fp16_rows_map(CUtensorMap* m, const void* base, int64_t rows, int bo
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [blocks][H][512] fp32 output or partial output, box = 128 channels x H heads x 1 block
-static bool out_map(CUtensorMap* m, void* base, int H, int64_t blocks) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)blocks};
-    cuuint64_t strides[2] = {(cuuint64_t)(kD * 4), (cuuint64_t)H * kD * 4};
-    cuuint32_t box[3] = {128u, (cuuint32_t)H, 1u};
-    cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // [blocks][H][512] fp32, box = 32 channels x H heads x 1 block, 128-byte swizzle
 static bool out_map_sw(CUtensorMap* m, void* base, int H, int64_t blocks) {
@@ -1150,19 +698,20 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merg
     a.partial_ml = (l.nsplit > 1 || a.part) ? l.partial + (int64_t)l.Q * l.nsplit * l.H * kD
                                             : nullptr;
     a.nsplit = l.nsplit;
-    a.nchunks = (l.K + l.W + kRows - 1) / kRows;
-    if (a.nchunks < 1) a.nchunks = 1;
-    a.chunks_per_split = (a.nchunks + l.nsplit - 1) / l.nsplit;
     a.status = l.status;
-    const int smem = TcSmem::kAlloc;
     dim3 grid((unsigned)l.Q, (unsigned)l.nsplit);
-    CUtensorMap mx, mq, mo;
+    CUtensorMap mx, mq;
     memset(&mx, 0, sizeof mx);
     memset(&mq, 0, sizeof mq);
-    if (l.nsplit > 1 ? !out_map(&mo, l.partial, l.H, (int64_t)l.Q * l.nsplit)
-                     : !out_map(&mo, l.out, l.H, l.Q))
-        return cudaErrorInvalidValue;
-    if (!l.prefill && l.stage && l.K + l.W > 0) {
+    if (l.K + l.W == 0) {
+        // no row at all: the output (or partial) of an empty softmax, final as written
+        *merged = true;
+        const int64_t n = (int64_t)l.Q * l.H;
+        const int blocks = (int)std::min<int64_t>((n * kD / 4 + 255) / 256, 4096);
+        return launch_pdl(attn_empty_kernel, dim3((unsigned)std::max(blocks, 1)), dim3(256), 0, st,
+                          a.part ? l.o_part : l.out, a.part ? l.ml_part : nullptr, l.Q, l.H);
+    }
+    if (!l.prefill && l.stage) {
         // staged decode: pre-pass, then one CTA per (query, split)
         const int rows = l.K + l.W;
         const int rps = attention_rows_per_split(rows, l.nsplit);
@@ -1223,10 +772,7 @@ cudaError_t launch_attention_tc(const AttnLaunch& l, cudaStream_t st, bool* merg
         return launch_pdl(attn_decode_kernel<false>, grid, dim3(256), (size_t)dsmem, st, mx, mq,
                           mos, a, rps);
     }
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(attn_tc_kernel<false>, grid, dim3(256), (size_t)smem, st, mx, mq, mo, a);
+    return cudaErrorInvalidValue;   // decode always has a staging area (api.cu)
 }
 
 }  // namespace csa2

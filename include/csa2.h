@@ -379,8 +379,9 @@ CSA2_API csa2_status_t csa2_cp_local_idx(int64_t n, const int32_t* idx, int64_t 
  * (its shard's selected entries, and the window rows on one shard only), left as a partial
  * result for csa2_attn_merge_partials: o_part fp32 [B][H][512] = sum_i 2^(l_i - m) x_i and
  * ml_part fp32 [B][2][H] = (m, sum_i 2^(l_i - m)), with l_i the logits in base-2 units
- * (scale * log2(e) * <q_h, x_i>); a head with no rows gives (-inf, 0) and a zero o_part.
- * Same arguments and checks as csa2_sparse_attn_decode, K + W >= 1, the same workspace.
+ * (scale * log2(e) * <q_h, x_i>); a head with no rows (all indices -1, or K = W = 0 for a
+ * shard that holds nothing) gives (-inf, 0) and a zero o_part, which the merge weighs 0.
+ * Same arguments and checks as csa2_sparse_attn_decode, the same workspace.
  * [TDG Compressed Sparse Attention 2 (CSA2)]: one softmax over the selected entries and the
  * window rows; splitting the rows and merging partials is the exact log-sum-exp identity.
  *

@@ -291,6 +291,30 @@ def test_attention_decode(B, H, K, W, n):
         check_attention(out[b].cpu().numpy(), ref, f"b={b}")
 
 
+def test_attention_decode_with_no_rows():
+    """K = 0 and W = 0: the softmax of an empty set contributes nothing. The output is zero
+    (the oracle's value), and a partial result is (maximum -inf, sum 0, output 0)."""
+    g = _gen(61)
+    B, H = 3, 64
+    q = torch.randn((B, H, 512), generator=g).to(torch.bfloat16).to(dev)
+    codes = torch.zeros((B, 8, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, 8, 32), dtype=torch.uint8, device=dev)
+    idx = torch.empty((B, 0), dtype=torch.int32, device=dev)
+    out = torch.full((B, H, 512), 7.0, dtype=torch.float32, device=dev)
+    ws = C().new_workspace(C().workspace_bytes(1, B, 1, H, 8, 0))
+    C().sparse_attn_decode("full", q, codes, scales, idx, None, out, ws)
+    o = torch.full((B, H, 512), 7.0, dtype=torch.float32, device=dev)
+    ml = torch.full((B, 2, H), 7.0, dtype=torch.float32, device=dev)
+    C().sparse_attn_decode_partial("full", q, codes, scales, idx, None, o, ml, ws)
+    torch.cuda.synchronize()
+    assert C().read_device_status(ws) == 0
+    ref = O.attention(O.bf16_array_to_f64(bits16(q[0])).reshape(H, 512), np.zeros((0, 512)), 0.1)
+    assert np.all(ref == 0.0)
+    assert torch.count_nonzero(out).item() == 0
+    assert torch.count_nonzero(o).item() == 0
+    assert torch.all(ml[:, 0] == -float("inf")) and torch.all(ml[:, 1] == 0)
+
+
 def test_attention_reuse_equals_full_and_bad_index_flag():
     B, H, K, W, n = 2, 64, 512, 128, 2000
     kv, codes, scales, idx, q, swa = _attn_case(B, H, K, W, n, seed=77)
