@@ -90,6 +90,13 @@ __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
 }
+// The two halves of cluster_sync_all, for work placed between them.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // shared::cluster address of `p` (this CTA's shared memory) in CTA `rank` of the cluster
 __device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
     uint32_t r;
@@ -105,6 +112,17 @@ __device__ __forceinline__ uint64_t ld_peer_u64(uint32_t addr) {
     uint64_t v;
     asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ void st_peer_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_peer_u64(uint32_t addr, uint64_t v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_peer_u32(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
 }
 __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
     float4 v;

@@ -11,18 +11,23 @@
 //
 // Radix select on an order-preserving 32-bit key of the fp32 score, extended to a unique
 // 64-bit composite  (key << 32) | ~id  so that "larger composite" is the required order.
-// Rows of up to 262,144 elements take one 1024-thread CTA each (topk_row_kernel: the steps
-// below, all in shared memory). Longer rows (the 1M-entry Full layer) are split over CTAs,
-// grid = chunks x rows:
-//   1. the scan kernel already histogrammed the top 12 key bits of every row, which fixes
-//      the threshold digit d0: fewer than K elements lie above it;
-//   2. every CTA classifies its chunk: elements above d0 are sure winners, elements on d0
-//      are candidates; both are appended to per-row lists (one atomic per list per CTA);
-//   3. the last CTA of a row to finish (threadfence + counter, no waiting) finds the exact
-//      `need`-th best candidate by 8-bit radix refinement over the candidate list (in shared
-//      memory when it fits, else in global memory, else over the row itself when even the
-//      list overflowed), marks the winners and chosen candidates in a shared bitmap of ids,
-//      and emits the set bits in ascending order.
+// The scan kernel already histogrammed the top 12 key bits of every row, which fixes the
+// threshold digit d0: fewer than K elements lie above it. Elements above d0 are sure
+// winners, elements on d0 are candidates, and the exact `need`-th best candidate is found
+// by 8-bit radix refinement. Three kernels:
+//   topk_bitmap_kernel  rows by position of up to 262,144 elements (Full layers, the pool's
+//                       block maxima): one CTA, or a cluster of CTAs, per row; picks are
+//                       marked in a bitmap of positions (see the kernel);
+//   topk_gather_kernel  rows of gathered ids (Reindex over the pool): one 1024-thread CTA
+//                       per row, winner and candidate lists in shared memory, picks ordered
+//                       through a bitmap of ids;
+//   topk_kernel         longer rows (the 1M-entry Full layer), grid = chunks x rows: every
+//                       CTA classifies its chunk into per-row lists (one atomic per list per
+//                       CTA); the last CTA of a row to finish (threadfence + counter, no
+//                       waiting) refines over the candidate list (in shared memory when it
+//                       fits, else in global memory, else over the row itself when even the
+//                       list overflowed) and emits the set bits of a bitmap of ids in
+//                       ascending order.
 #include "csa2_common.cuh"
 #include "csa2_internal.h"
 
@@ -434,23 +439,13 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
 // single SM keeps far more bytes in flight that way than with per-thread loads. With ids
 // (Reindex: short rows) the elements are read 8 per thread per batch.
 constexpr int kRowThreads = 1024;
-constexpr int kRowPer = 16;                  // elements per thread per chunk (no ids)
-constexpr int kRowChunk = kRowThreads * kRowPer;   // 16384 elements = 64 KiB
 constexpr int kRowPerIds = 8;                // elements per thread per batch (ids)
 constexpr int kRowCands = 4096;
 constexpr int64_t kRowMaxN = 262144;
-constexpr int kRowCluster = 4;               // CTAs per row for few long rows
 constexpr size_t kRowOffHist = 0;                                   // u32[4096]
 constexpr size_t kRowOffCand = kRowOffHist + 4 * kBinsT;            // u64[kRowCands]
 constexpr size_t kRowOffWin = kRowOffCand + 8 * kRowCands;          // u32[kMaxK]
-constexpr size_t kRowOffBar = kRowOffWin + 4 * kMaxK;               // 3 mbarriers
-constexpr size_t kRowOffBm = kRowOffBar + 64;                       // bitmap or pick list
-// after the bitmap (no ids): two chunk buffers, 64 KiB each, 128-byte aligned
-constexpr size_t kRowChunkBytes = (size_t)kRowChunk * 4;
-__host__ __device__ constexpr size_t row_chunk_offset(int bitmap_words) {
-    return (kRowOffBm + (bitmap_words > 0 ? (size_t)bitmap_words * 4 : (size_t)kMaxK * 4) + 127) &
-           ~(size_t)127;
-}
+constexpr size_t kRowOffBm = kRowOffWin + 4 * kMaxK;                // bitmap or pick list
 
 // Exclusive prefix sum of v over the 1024 threads (thread order); `total` gets the sum.
 // Uses wsum[0..32); ends with a barrier, so wsum may be reused right away.
@@ -620,8 +615,8 @@ __device__ __forceinline__ void row_threshold(const RowState& S, const uint32_t 
     __syncthreads();
 }
 
-// Refinement, picks and the ordered output of one row, after every element was classified.
-template <bool GATHER>
+// Refinement, picks and the ordered output of one gathered row, after every element was
+// classified.
 __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t n,
                              uint32_t id_lim, bool many, int d0, uint32_t above, int ccap) {
     const int tid = threadIdx.x;
@@ -643,13 +638,9 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
         auto cand = [&](int64_t i, uint64_t& c) -> bool {
             if (from_row) {
                 const uint32_t kk = elem_key(a, r, i);
-                uint32_t id = (uint32_t)i;
-                if (GATHER) {
-                    const int32_t v = ld_dep(a.ids + (int64_t)r * a.ld + i);
-                    if (v < 0 || (uint32_t)v >= id_lim) return false;
-                    id = (uint32_t)v;
-                }
-                c = ((uint64_t)kk << 32) | (uint64_t)(~id);
+                const int32_t v = ld_dep(a.ids + (int64_t)r * a.ld + i);
+                if (v < 0 || (uint32_t)v >= id_lim) return false;
+                c = ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)v);
                 return (int)(kk >> 20) == d0;
             }
             c = i < kRowCands ? S.cand_s[i] : __ldcg(gcand + i);
@@ -759,14 +750,10 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
     for (int i = npick * mult + tid; i < K * mult; i += kRowThreads) o[i] = -1;
 }
 
-// CL > 1: a cluster of CL CTAs shares one row. Every CTA finds d0 and classifies its own
-// contiguous part of the row into its own lists; CTA 0 then gathers the other CTAs' lists
-// through distributed shared memory and finishes the row alone.
-template <bool GATHER, int CL>
-__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev a) {
-    static_assert(!GATHER || CL == 1, "gather rows are short: one CTA each");
-    // with a cluster, every CTA's candidate list lives in shared memory only
-    const int ccap = CL > 1 ? 0 : a.ccap;
+// Rows of gathered ids (Reindex over the candidate pool): one CTA per row, elements read in
+// batches of 8 per thread with plain loads, classified into winner and candidate lists.
+__global__ void __launch_bounds__(kRowThreads, 1) topk_gather_kernel(const TopkDev a) {
+    const int ccap = a.ccap;
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ uint32_t wsum[40];
     __shared__ int dig_s[4];
@@ -779,16 +766,14 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
     S.wsum = wsum;
     S.dig_s = dig_s;
     S.tot_s = tot_s;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + kRowOffBar);
-    const int r = CL > 1 ? (int)blockIdx.y : (int)blockIdx.x;
-    const uint32_t crank = CL > 1 ? cluster_rank() : 0u;
+    const int r = (int)blockIdx.x;
     const int tid = threadIdx.x;
     grid_dep_launch();
     grid_dep_wait();
     const int64_t n = row_len(a, r);
     const int K = a.K;
-    const uint32_t id_lim = GATHER ? (uint32_t)max(0, ld_dep(a.id_limit + r)) : 0xFFFFFFFFu;
-    const bool use_bm = a.bitmap_words > 0 && crank == 0;
+    const uint32_t id_lim = (uint32_t)max(0, ld_dep(a.id_limit + r));
+    const bool use_bm = a.bitmap_words > 0;
     const int nwords = a.bitmap_words;
     if (tid == 0) {
         tot_s[0] = tot_s[1] = 0u;
@@ -798,149 +783,355 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(const TopkDev 
     bool many;
     int d0;
     uint32_t above;
+    constexpr int PER = kRowPerIds;
+    constexpr int BATCH = kRowThreads * PER;
+    uint32_t key[PER], id[PER];
+    auto load = [&](int64_t base) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = base + (int64_t)k * kRowThreads + tid;
+            key[k] = i < n ? elem_key(a, r, i) : 0u;
+            id[k] = i < n ? (uint32_t)ld_dep(a.ids + (int64_t)r * a.ld + i) : 0xFFFFFFFFu;
+        }
+    };
+    load(0);
+    const uint4 h4 = reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kBinsT)[kRowThreads - 1 - tid];
+    if (use_bm)
+        for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
+    const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
+    row_threshold(S, b4, K, many, d0, above);
+    for (int64_t base = 0; base < n; base += BATCH) {
+        if (base > 0) load(base);
+        uint32_t valid = 0;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = base + (int64_t)k * kRowThreads + tid;
+            if (i < n && (int32_t)id[k] >= 0 && id[k] < id_lim) valid |= 1u << k;
+        }
+        row_classify<PER>(a, S, r, key, [&](int k) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (j == k) v = id[j];
+            return v;
+        }, valid, many, d0, ccap);
+    }
+    row_finalize(a, S, r, n, id_lim, many, d0, above, ccap);
+}
 
-    if constexpr (GATHER) {
-        // ---- ids: plain loads, 8 elements per thread per batch ------------------------------
-        constexpr int PER = kRowPerIds;
-        constexpr int BATCH = kRowThreads * PER;
-        uint32_t key[PER], id[PER];
-        auto load = [&](int64_t base) {
+// ---- rows by position: picks marked in a bitmap of positions ---------------------------------
+// One row per CTA, or per cluster of CL CTAs that split it into word-aligned parts. The
+// elements stream through registers in rounds of NT x 32; a warp's 32 consecutive positions
+// are one bitmap word, built with a ballot. Winners (first digit above d0) are marked as they
+// are read; candidates (first digit d0) go to a list through one warp-aggregated atomic per
+// warp and digit. Bitmap, list and counters live in the shared memory of the row's first CTA
+// (the others write them through distributed shared memory); that CTA then finds the exact
+// `need`-th best candidate by 8-bit radix refinement and emits the set bits in ascending
+// order. No list of winners is kept, so the block-wide steps are d0, the refinement passes
+// and the final prefix sum.
+constexpr int kBmPer = 32;                    // elements per thread per round
+constexpr int kBmCands = 4096;                // candidates kept in shared memory
+constexpr int64_t kBmMaxN = 262144;
+constexpr size_t kBmOffHist = 0;                                   // u32[4096]
+constexpr size_t kBmOffCand = kBmOffHist + 4 * kBinsT;             // u64[kBmCands]
+constexpr size_t kBmOffBm = kBmOffCand + 8 * (size_t)kBmCands;     // u32[kBmMaxN / 32]
+constexpr size_t kBmSmem = kBmOffBm + 4 * (size_t)(kBmMaxN / 32);
+
+// Exclusive prefix sum of v over the NT threads of the block (thread order); `total` gets
+// the sum. Uses wsum[0..33); ends with a barrier.
+template <int NT>
+__device__ __forceinline__ uint32_t bm_excl_scan(uint32_t v, uint32_t* wsum, uint32_t& total) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
 #pragma unroll
-            for (int k = 0; k < PER; ++k) {
-                const int64_t i = base + (int64_t)k * kRowThreads + tid;
-                key[k] = i < n ? elem_key(a, r, i) : 0u;
-                id[k] = i < n ? (uint32_t)ld_dep(a.ids + (int64_t)r * a.ld + i) : 0xFFFFFFFFu;
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t x = lane < NW ? wsum[lane] : 0u;
+        uint32_t xi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += u;
+        }
+        if (lane < NW) wsum[lane] = xi - x;
+        if (lane == 31) wsum[32] = xi;
+    }
+    __syncthreads();
+    const uint32_t res = wsum[warp] + incl - v;
+    total = wsum[32];
+    __syncthreads();
+    return res;
+}
+
+template <int NT, int CL>
+__global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDev a) {
+    static_assert(NT % 32 == 0 && kBinsT % NT == 0, "block size");
+    constexpr int BPT = kBinsT / NT;              // first-digit bins per thread
+    constexpr int64_t RS = (int64_t)NT * kBmPer;  // elements per round
+    extern __shared__ __align__(16) uint8_t dsm[];
+    uint32_t* hist = reinterpret_cast<uint32_t*>(dsm + kBmOffHist);
+    uint64_t* cand = reinterpret_cast<uint64_t*>(dsm + kBmOffCand);
+    uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + kBmOffBm);
+    __shared__ uint32_t wsum[40];
+    __shared__ int dig_s[4];
+    __shared__ uint32_t cnt_s[2];   // candidates, winners
+    __shared__ __align__(8) uint64_t bar;
+    const int r = CL > 1 ? (int)blockIdx.y : (int)blockIdx.x;
+    const uint32_t crank = CL > 1 ? cluster_rank() : 0u;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.K;
+    grid_dep_launch();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        cnt_s[0] = cnt_s[1] = 0u;
+        dig_s[0] = -1;
+        dig_s[1] = 0;
+    }
+    __syncthreads();
+    // the first CTA's counters are set before any CTA of the cluster adds to them
+    if constexpr (CL > 1) cluster_arrive();
+    grid_dep_wait();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar, 4u * kBinsT);
+        bulk_load(hist, a.hist + (int64_t)r * kBinsT, 4u * kBinsT, &bar);
+    }
+    int64_t n = row_len(a, r);
+    n = n < 0 ? 0 : (n > a.ld ? a.ld : n);
+    // this CTA's part [p0, p1) of the row, word aligned
+    const int64_t part = CL > 1 ? ((((n + CL - 1) / CL) + 31) & ~(int64_t)31) : n;
+    const int64_t p0 = (int64_t)crank * part < n ? (int64_t)crank * part : n;
+    const int64_t p1 = p0 + part < n ? p0 + part : n;
+    const int nrounds = (int)((p1 - p0 + RS - 1) / RS);
+    // raw bits; the order-preserving key is formed where it is used, so that no thread
+    // waits for these loads before the histogram step
+    uint32_t raw[kBmPer];
+    const uint32_t* src = a.scores ? reinterpret_cast<const uint32_t*>(a.scores) : a.keys;
+    auto load_round = [&](int64_t base) {
+#pragma unroll
+        for (int j = 0; j < kBmPer; ++j) {
+            const int64_t e = base + (int64_t)j * NT + tid;
+            raw[j] = e < p1 ? ld_dep(src + (int64_t)r * a.ld + e) : 0u;
+        }
+    };
+    auto key_of = [&](uint32_t v) { return a.scores ? score_key(__uint_as_float(v)) : v; };
+    if (nrounds > 0) load_round(p0);   // in flight while the histogram arrives
+
+    // ---- d0: the first digit that holds the K-th best element (every CTA) -------------------
+    mbar_wait(&bar, 0, a.status);
+    uint32_t b[BPT], local = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {   // thread 0 owns the highest bins, highest first
+        b[j] = hist[kBinsT - 1 - BPT * tid - j];
+        local += b[j];
+    }
+    uint32_t total;
+    const uint32_t excl = bm_excl_scan<NT>(local, wsum, total);
+    if (excl < (uint32_t)K && excl + local >= (uint32_t)K) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+            if (acc < (uint32_t)K && acc + b[j] >= (uint32_t)K) {
+                dig_s[0] = kBinsT - 1 - BPT * tid - j;
+                dig_s[1] = (int)acc;
             }
-        };
-        load(0);
-        const uint4 h4 = reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kBinsT)[kRowThreads - 1 - tid];
-        if (use_bm)
-            for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
-        const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
-        row_threshold(S, b4, K, many, d0, above);
-        for (int64_t base = 0; base < n; base += BATCH) {
-            if (base > 0) load(base);
-            uint32_t valid = 0;
+            acc += b[j];
+        }
+    }
+    __syncthreads();
+    const bool many = total >= (uint32_t)K;
+    const int d0 = many ? dig_s[0] : -1;
+    const uint32_t above = many ? (uint32_t)dig_s[1] : total;
+
+    // ---- classify: winners into the bitmap, candidates into the list ----------------------------
+    // (addresses in the first CTA of the cluster; plain shared memory without a cluster)
+    uint32_t bm0 = 0, cand0 = 0, cnt0 = 0;
+    if constexpr (CL > 1) {
+        cluster_wait();
+        bm0 = peer_addr(bm, 0);
+        cand0 = peer_addr(cand, 0);
+        cnt0 = peer_addr(cnt_s, 0);
+    }
+    uint32_t nwin_w = 0;   // lane 0: this warp's winners
+    for (int rd = 0; rd < nrounds; ++rd) {
+        const int64_t base = p0 + (int64_t)rd * RS;
+        if (rd > 0) load_round(base);
+        // winners' words, and the warp's candidate count
+        uint32_t ncw = 0;
 #pragma unroll
-            for (int k = 0; k < PER; ++k) {
-                const int64_t i = base + (int64_t)k * kRowThreads + tid;
-                if (i < n && (int32_t)id[k] >= 0 && id[k] < id_lim) valid |= 1u << k;
+        for (int j = 0; j < kBmPer; ++j) {
+            if (base + (int64_t)j * NT >= p1) break;                 // the same for every warp
+            const int64_t e0 = base + (int64_t)j * NT + warp * 32;   // the warp's first position
+            const bool ok = e0 + lane < p1;
+            const int dig = (int)(key_of(raw[j]) >> 20);
+            const uint32_t wb = __ballot_sync(0xffffffffu, ok && (!many || dig > d0));
+            ncw += (uint32_t)__popc(__ballot_sync(0xffffffffu, ok && many && dig == d0));
+            if (lane == 0 && e0 < p1) {
+                if constexpr (CL > 1) st_peer_u32(bm0 + 4u * (uint32_t)(e0 >> 5), wb);
+                else bm[e0 >> 5] = wb;
+                nwin_w += __popc(wb);
             }
-            row_classify<PER>(a, S, r, key, [&](int k) {
-                uint32_t v = 0;
+        }
+        if (ncw == 0) continue;
+        // one atomic per warp reserves its candidates' slots
+        uint32_t q = 0;
+        if (lane == 0) {
+            if constexpr (CL > 1) q = atom_add_peer_u32(cnt0, ncw);
+            else q = atomicAdd(&cnt_s[0], ncw);
+        }
+        q = __shfl_sync(0xffffffffu, q, 0);
 #pragma unroll
-                for (int j = 0; j < PER; ++j)
-                    if (j == k) v = id[j];
-                return v;
-            }, valid, many, d0, ccap);
-        }
-    } else {
-        // ---- positions: histogram and elements through bulk copies -------------------------
-        // Elements [h0, h0 + nbulk) arrive in 64 KiB chunks (16-byte aligned source, whole
-        // 16-byte units); the few before h0 and after the last unit are read directly.
-        uint8_t* cbuf = dsm + row_chunk_offset(nwords);
-        const uint8_t* rowp = a.scores ? reinterpret_cast<const uint8_t*>(a.scores + (int64_t)r * a.ld)
-                                       : reinterpret_cast<const uint8_t*>(a.keys + (int64_t)r * a.ld);
-        const int64_t lead = (int64_t)(((16u - (reinterpret_cast<uintptr_t>(rowp) & 15u)) & 15u) >> 2);
-        const int h0 = (int)(lead < n ? lead : n);
-        const int64_t nbulk_all = ((n - h0) >> 2) << 2;   // whole 16-byte units
-        const int64_t ntail = n - h0 - nbulk_all;          // < 4
-        // this CTA's part [pb, pb + nbulk) of the bulk elements (4-element granularity)
-        const int64_t part = (((nbulk_all >> 2) + CL - 1) / CL) << 2;
-        const int64_t pb = (int64_t)crank * part < nbulk_all ? (int64_t)crank * part : nbulk_all;
-        const int64_t nbulk = (pb + part < nbulk_all ? pb + part : nbulk_all) - pb;
-        const int nch = (int)((nbulk + kRowChunk - 1) / kRowChunk);
-        bool ok = true;
-        auto issue = [&](int c) {
-            const int64_t e0 = (int64_t)c * kRowChunk;
-            const int64_t left = nbulk - e0;
-            const uint32_t bytes = (uint32_t)((left < kRowChunk ? left : (int64_t)kRowChunk) * 4);
-            mbar_arrive_expect_tx(&bar[1 + (c & 1)], bytes);
-            bulk_load(cbuf + (size_t)(c & 1) * kRowChunkBytes, rowp + (h0 + pb + e0) * 4, bytes,
-                      &bar[1 + (c & 1)]);
-        };
-        if (tid == 0) {
-            mbar_init(&bar[0], 1);
-            mbar_init(&bar[1], 1);
-            mbar_init(&bar[2], 1);
-            fence_mbar_init();
-            mbar_arrive_expect_tx(&bar[0], 4u * kBinsT);
-            bulk_load(S.hist, a.hist + (int64_t)r * kBinsT, 4u * kBinsT, &bar[0]);
-            for (int c = 0; c < min(nch, 2); ++c) issue(c);
-        }
-        // the stray head / tail elements: one per thread among the first few threads
-        uint32_t xkey = 0u;
-        int64_t xi = -1;
-        if (crank == 0) {
-            if (tid < h0) xi = tid;
-            else if (tid - h0 < ntail) xi = h0 + nbulk_all + (tid - h0);
-        }
-        if (xi >= 0) xkey = elem_key(a, r, xi);
-        if (use_bm)
-            for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
-        __syncthreads();   // barrier initialisation is visible to every waiting thread
-        if (!mbar_wait(&bar[0], 0, a.status)) ok = false;
-        const uint4 h4 = reinterpret_cast<const uint4*>(S.hist)[kRowThreads - 1 - tid];
-        const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
-        row_threshold(S, b4, K, many, d0, above);   // ends with a barrier: hist is free again
-        for (int c = 0; c < max(nch, 1); ++c) {
-            uint32_t key[kRowPer + 1];
-            uint32_t valid = 0;
-            const int64_t e0 = (int64_t)c * kRowChunk;
-            if (c < nch) {
-                if (!mbar_wait(&bar[1 + (c & 1)], (uint32_t)((c >> 1) & 1), a.status)) ok = false;
-                const uint32_t* buf = reinterpret_cast<const uint32_t*>(cbuf + (size_t)(c & 1) * kRowChunkBytes);
-#pragma unroll
-                for (int k = 0; k < kRowPer; ++k) {
-                    const int64_t e = e0 + (int64_t)k * kRowThreads + tid;
-                    const uint32_t raw = e < nbulk ? buf[k * kRowThreads + tid] : 0u;
-                    key[k] = a.scores ? score_key(__uint_as_float(raw)) : raw;
-                    if (e < nbulk) valid |= 1u << k;
+        for (int j = 0; j < kBmPer; ++j) {
+            if (base + (int64_t)j * NT >= p1) break;
+            const int64_t e = base + (int64_t)j * NT + warp * 32 + lane;
+            const uint32_t kk = key_of(raw[j]);
+            const bool c = e < p1 && (int)(kk >> 20) == d0;
+            const uint32_t cb = __ballot_sync(0xffffffffu, c);
+            if (c) {
+                const uint32_t qi = q + __popc(cb & ((1u << lane) - 1u));
+                const uint64_t comp = ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)e);
+                if (qi < (uint32_t)kBmCands) {
+                    if constexpr (CL > 1) st_peer_u64(cand0 + 8u * qi, comp);
+                    else cand[qi] = comp;
                 }
-            } else {
-#pragma unroll
-                for (int k = 0; k < kRowPer; ++k) key[k] = 0u;
             }
-            key[kRowPer] = xkey;
-            if (c == 0 && xi >= 0) valid |= 1u << kRowPer;
-            const uint32_t idb = (uint32_t)(h0 + pb + e0 + tid);
-            row_classify<kRowPer + 1>(a, S, r, key, [&](int k) {
-                return k < kRowPer ? idb + (uint32_t)k * kRowThreads : (uint32_t)xi;
-            }, valid, many, d0, ccap);
-            // every thread has read buffer (c & 1): refill it with chunk c + 2
-            if (tid == 0 && ok && c + 2 < nch) issue(c + 2);
+            q += (uint32_t)__popc(cb);
         }
+    }
+    if (lane == 0 && nwin_w) {
+        if constexpr (CL > 1) atom_add_peer_u32(cnt0 + 4u, nwin_w);
+        else atomicAdd(&cnt_s[1], nwin_w);
     }
     if constexpr (CL > 1) {
-        // every CTA's lists are complete; CTA 0 appends the others' lists to its own
-        cluster_sync_all();
-        if (crank == 0) {
-            uint32_t wbase = tot_s[0], cbase = tot_s[1];
-            __syncthreads();
-#pragma unroll 1
-            for (uint32_t k = 1; k < (uint32_t)CL; ++k) {
-                const uint32_t nw = ld_peer_u32(peer_addr(&tot_s[0], k));
-                const uint32_t nc = ld_peer_u32(peer_addr(&tot_s[1], k));
-                const uint32_t rw = peer_addr(S.win_s, k), rc = peer_addr(S.cand_s, k);
-                for (uint32_t i = tid; i < nw; i += kRowThreads)
-                    if (wbase + i < (uint32_t)K && i < (uint32_t)K) S.win_s[wbase + i] = ld_peer_u32(rw + 4 * i);
-                for (uint32_t i = tid; i < nc; i += kRowThreads)
-                    if (cbase + i < (uint32_t)kRowCands && i < (uint32_t)kRowCands)
-                        S.cand_s[cbase + i] = ld_peer_u64(rc + 8 * i);
-                wbase += nw;
-                cbase += nc;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                tot_s[0] = wbase;
-                tot_s[1] = cbase;
-            }
-            __syncthreads();
-        }
-        cluster_sync_all();   // the other CTAs' lists have been read: they may exit
+        // every part is in the first CTA's shared memory; the others are done
+        cluster_arrive();
+        cluster_wait();
         if (crank != 0) return;
+    } else {
+        __syncthreads();
     }
-    row_finalize<GATHER>(a, S, r, n, id_lim, many, d0, above, ccap);
+    const uint32_t ncand = cnt_s[0], nwin_all = cnt_s[1];
+    if (tid == 0 && (nwin_all > (uint32_t)K || (many && nwin_all != above)))
+        set_status(a.status, CSA2_DEV_BAD_COUNT);
+
+    // ---- the exact `need`-th best candidate -------------------------------------------------------
+    if (many) {
+        const uint32_t need = (uint32_t)K - above;
+        const bool from_row = ncand > (uint32_t)kBmCands;   // list overflowed: read the row again
+        const int64_t nsrc = from_row ? n : (int64_t)ncand;
+        auto cnd = [&](int64_t i, uint64_t& c) -> bool {
+            if (from_row) {
+                const uint32_t kk = elem_key(a, r, i);
+                c = ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)i);
+                return (int)(kk >> 20) == d0;
+            }
+            c = cand[i];
+            return true;
+        };
+        uint64_t prefix = (uint64_t)d0;
+        int shift = 52;
+        uint32_t rem = need;
+        bool found = true;
+        while (shift > 0) {
+            const int nb = shift < 8 ? shift : 8;
+            for (int i = tid; i < 256; i += NT) hist[i] = 0u;
+            __syncthreads();
+            for (int64_t i = tid; i < nsrc; i += NT) {
+                uint64_t c;
+                if (cnd(i, c) && (c >> shift) == prefix)
+                    atomicAdd(&hist[(c >> (shift - nb)) & ((1u << nb) - 1u)], 1u);
+            }
+            __syncthreads();
+            if (tid < 32) warp_find_digit256(hist, rem, dig_s);
+            __syncthreads();
+            const int d = dig_s[0];
+            const uint32_t ab = (uint32_t)dig_s[1], inbin = (uint32_t)dig_s[2];
+            __syncthreads();   // dig_s is rewritten by the next pass
+            if (d < 0) {
+                if (tid == 0) set_status(a.status, CSA2_DEV_BAD_COUNT);
+                found = false;
+                break;
+            }
+            rem -= ab;
+            prefix = (prefix << nb) | (uint64_t)d;
+            shift -= nb;
+            if (inbin == rem) break;   // the whole bin is taken
+        }
+        if (found) {
+            const uint64_t T = prefix << shift;
+            for (int64_t i = tid; i < nsrc; i += NT) {
+                uint64_t c;
+                if (cnd(i, c) && c >= T) {
+                    const uint32_t id = ~(uint32_t)(c & 0xFFFFFFFFu);
+                    atomicOr(&bm[id >> 5], 1u << (id & 31));
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- emit the set bits in ascending position order -------------------------------------------
+    const int64_t nwords = (n + 31) >> 5;
+    const int32_t lim = a.expand8 ? ld_dep(a.expand_limit + r) : 0;
+    int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
+    const int64_t per = (nwords + NT - 1) / NT;
+    const int64_t w0 = tid * per, w1 = w0 + per < nwords ? w0 + per : nwords;
+    uint32_t cntb = 0;
+    for (int64_t wi = w0; wi < w1; ++wi) cntb += __popc(bm[wi]);
+    uint32_t tot;
+    uint32_t off = bm_excl_scan<NT>(cntb, wsum, tot);
+    const int npick = (int)min(tot, (uint32_t)K);
+    for (int64_t wi = w0; wi < w1; ++wi) {
+        uint32_t m = bm[wi];
+        while (m) {
+            const int bit = __ffs(m) - 1;
+            m &= m - 1;
+            const uint32_t slot = off++;
+            if (slot >= (uint32_t)K) continue;
+            const int64_t id = wi * 32 + bit;
+            if (!a.expand8) {
+                o[slot] = (int32_t)id;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int64_t pos = id * 8 + e;
+                    o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
+                }
+            }
+        }
+    }
+    const int mult = a.expand8 ? 8 : 1;
+    for (int i = npick * mult + tid; i < K * mult; i += NT) o[i] = -1;
+}
+
+template <int NT, int CL>
+static cudaError_t launch_bitmap(const TopkDev& a, int R, cudaStream_t st) {
+    auto kern = topk_bitmap_kernel<NT, CL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBmSmem);
+    if (e != cudaSuccess) return e;
+    if (CL == 1) return launch_pdl(kern, dim3((unsigned)R), dim3(NT), kBmSmem, st, a);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(CL, (unsigned)R);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = kBmSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
@@ -967,40 +1158,27 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     // ids are < id_bound: a bitmap of that many bits orders the picks when it fits
     const int64_t words = (l.id_bound + 31) / 32;
     cudaError_t e;
-    if (l.max_n <= kRowMaxN) {
-        // ids: the bitmap may cover up to 2^20 ids; positions: ids < max_n <= 2^18, and the
-        // two 64 KiB chunk buffers follow the bitmap
+    if (!l.ids && l.max_n <= kBmMaxN) {
+        // Few rows: a cluster per row spreads the reading over more SMs, within one wave:
+        // 1024-thread CTAs (one per SM) while four per row fit, else 512-thread CTAs (two
+        // per SM), with at least 4,096 elements per CTA.
+        const int sms = device_sm_count();
+        if (l.max_n >= 4 * 8192 && l.R * 4 <= sms) return launch_bitmap<1024, 4>(a, l.R, st);
+        if (l.max_n >= 8 * 4096 && l.R * 8 <= 2 * sms) return launch_bitmap<512, 8>(a, l.R, st);
+        if (l.max_n >= 4 * 4096 && l.R * 4 <= 2 * sms) return launch_bitmap<512, 4>(a, l.R, st);
+        if (l.max_n >= 2 * 4096 && l.R * 2 <= 2 * sms) return launch_bitmap<512, 2>(a, l.R, st);
+        return launch_bitmap<512, 1>(a, l.R, st);
+    }
+    if (l.ids && l.max_n <= kRowMaxN) {
+        // the bitmap of ids may cover up to 2^20 ids
         a.bitmap_words = (l.id_bound > 0 && words * 4 <= 128 * 1024) ? (int)words : 0;
-        size_t rsmem = kRowOffBm + (a.bitmap_words > 0 ? (size_t)a.bitmap_words * 4
-                                                        : (size_t)kMaxK * 4);
-        if (!l.ids) rsmem = row_chunk_offset(a.bitmap_words) + 2 * kRowChunkBytes;
+        const size_t rsmem = kRowOffBm + (a.bitmap_words > 0 ? (size_t)a.bitmap_words * 4
+                                                              : (size_t)kMaxK * 4);
         if (rsmem > 227 * 1024) return cudaErrorInvalidValue;
-        // few long rows: a cluster of kRowCluster CTAs per row spreads the classification
-        if (!l.ids && l.max_n >= 4 * kRowChunk / 2 && l.R * kRowCluster <= 2 * device_sm_count()) {
-            auto kern = topk_row_kernel<false, kRowCluster>;
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
-            if (e != cudaSuccess) return e;
-            cudaLaunchConfig_t cfg;
-            memset(&cfg, 0, sizeof cfg);
-            cfg.gridDim = dim3(kRowCluster, (unsigned)l.R);
-            cfg.blockDim = dim3(kRowThreads);
-            cfg.dynamicSmemBytes = rsmem;
-            cfg.stream = st;
-            cudaLaunchAttribute attr[2];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = kRowCluster;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[1].val.programmaticStreamSerializationAllowed = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 2;
-            return cudaLaunchKernelEx(&cfg, kern, a);
-        }
-        auto kern = l.ids ? topk_row_kernel<true, 1> : topk_row_kernel<false, 1>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+        e = cudaFuncSetAttribute(topk_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)rsmem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3((unsigned)l.R), dim3(kRowThreads), rsmem, st, a);
+        return launch_pdl(topk_gather_kernel, dim3((unsigned)l.R), dim3(kRowThreads), rsmem, st, a);
     }
     a.bitmap_words = (l.id_bound > 0 && words * 4 <= 64 * 1024) ? (int)words : 0;
     const size_t smem = (size_t)kSmemCands * 8 +
