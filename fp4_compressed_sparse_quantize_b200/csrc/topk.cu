@@ -57,6 +57,7 @@ struct TopkDev {
     uint64_t* cands;
     int ccap;
     int bitmap_words;        // > 0: order the picks through a shared bitmap of ids
+    int ring;                // topk_bitmap_kernel: chunk buffers in flight
     int32_t* status;
 };
 
@@ -820,25 +821,34 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_gather_kernel(const TopkD
 }
 
 // ---- rows by position: picks marked in a bitmap of positions ---------------------------------
-// One row per CTA, or per cluster of CL CTAs that split it into word-aligned parts. The
-// elements stream through registers in rounds of NT x 32; a warp's 32 consecutive positions
-// are one bitmap word, built with a ballot. Winners (first digit above d0) are marked as they
-// are read; candidates (first digit d0) go to a list through one warp-aggregated atomic per
-// warp and digit. Bitmap, list and counters live in the shared memory of the row's first CTA
-// (the others write them through distributed shared memory); that CTA then finds the exact
-// `need`-th best candidate by 8-bit radix refinement and emits the set bits in ascending
-// order. No list of winners is kept, so the block-wide steps are d0, the refinement passes
-// and the final prefix sum.
-constexpr int kBmPer = 32;                    // elements per thread per round
+// One row per CTA, or per cluster of CL CTAs that split it into parts. Each CTA's part
+// streams into shared memory by bulk copies (a ring of `ring` chunks of NT x 8 elements; a
+// single SM keeps far more bytes in flight that way than with per-thread loads); the few
+// elements before the first and after the last 16-byte unit are read directly. Winners
+// (first digit above d0) are set in a bitmap of positions as they are read; candidates
+// (first digit d0) go to a list through one warp-aggregated atomic per warp and chunk.
+// Bitmap, list and counters live in the shared memory of the row's first CTA (the others
+// write them through distributed shared memory); that CTA then finds the exact `need`-th
+// best candidate by 8-bit radix refinement and emits the set bits in ascending order. No list
+// of winners is kept, so the block-wide steps are d0, one barrier per chunk, the refinement
+// passes and the final prefix sum.
+constexpr int kBmPer = 8;                     // elements per thread per chunk
 constexpr int kBmCands = 4096;                // candidates kept in shared memory
 constexpr int64_t kBmMaxN = 262144;
 constexpr size_t kBmOffHist = 0;                                   // u32[4096]
 constexpr size_t kBmOffCand = kBmOffHist + 4 * kBinsT;             // u64[kBmCands]
-constexpr size_t kBmOffBm = kBmOffCand + 8 * (size_t)kBmCands;     // u32[kBmMaxN / 32]
-constexpr size_t kBmSmem = kBmOffBm + 4 * (size_t)(kBmMaxN / 32);
+constexpr size_t kBmOffBm = kBmOffCand + 8 * (size_t)kBmCands;     // u32[bitmap words]
+__host__ __device__ constexpr size_t bm_off_ring(int words) {
+    return (kBmOffBm + 4 * (size_t)words + 127) & ~(size_t)127;
+}
+__host__ __device__ constexpr size_t bm_chunk_bytes(int nt) { return (size_t)nt * kBmPer * 4; }
+__host__ __device__ constexpr size_t bm_off_bar(int words, int nt, int ring) {
+    return bm_off_ring(words) + (size_t)ring * bm_chunk_bytes(nt);
+}
+__host__ __device__ constexpr size_t bm_smem(int words, int nt, int ring) {
+    return bm_off_bar(words, nt, ring) + 8 * (size_t)(ring + 1);
+}
 
-// Exclusive prefix sum of v over the NT threads of the block (thread order); `total` gets
-// the sum. Uses wsum[0..33); ends with a barrier.
 template <int NT>
 __device__ __forceinline__ uint32_t bm_excl_scan(uint32_t v, uint32_t* wsum, uint32_t& total) {
     constexpr int NW = NT / 32;
@@ -872,59 +882,69 @@ __device__ __forceinline__ uint32_t bm_excl_scan(uint32_t v, uint32_t* wsum, uin
 template <int NT, int CL>
 __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDev a) {
     static_assert(NT % 32 == 0 && kBinsT % NT == 0, "block size");
-    constexpr int BPT = kBinsT / NT;              // first-digit bins per thread
-    constexpr int64_t RS = (int64_t)NT * kBmPer;  // elements per round
+    constexpr int BPT = kBinsT / NT;                    // first-digit bins per thread
+    constexpr int CE = NT * kBmPer;                     // elements per chunk
     extern __shared__ __align__(16) uint8_t dsm[];
+    const int words = a.bitmap_words, ring = a.ring;
     uint32_t* hist = reinterpret_cast<uint32_t*>(dsm + kBmOffHist);
     uint64_t* cand = reinterpret_cast<uint64_t*>(dsm + kBmOffCand);
     uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + kBmOffBm);
+    const uint32_t* buf = reinterpret_cast<const uint32_t*>(dsm + bm_off_ring(words));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + bm_off_bar(words, NT, ring));
     __shared__ uint32_t wsum[40];
     __shared__ int dig_s[4];
     __shared__ uint32_t cnt_s[2];   // candidates, winners
-    __shared__ __align__(8) uint64_t bar;
     const int r = CL > 1 ? (int)blockIdx.y : (int)blockIdx.x;
     const uint32_t crank = CL > 1 ? cluster_rank() : 0u;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int K = a.K;
     grid_dep_launch();
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        for (int i = 0; i <= ring; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
         cnt_s[0] = cnt_s[1] = 0u;
         dig_s[0] = -1;
         dig_s[1] = 0;
     }
+    for (int i = tid; i < words; i += NT) bm[i] = 0u;
     __syncthreads();
-    // the first CTA's counters are set before any CTA of the cluster adds to them
+    // the first CTA's bitmap and counters are cleared before any CTA of the cluster writes
     if constexpr (CL > 1) cluster_arrive();
     grid_dep_wait();
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar, 4u * kBinsT);
-        bulk_load(hist, a.hist + (int64_t)r * kBinsT, 4u * kBinsT, &bar);
-    }
+
     int64_t n = row_len(a, r);
     n = n < 0 ? 0 : (n > a.ld ? a.ld : n);
-    // this CTA's part [p0, p1) of the row, word aligned
-    const int64_t part = CL > 1 ? ((((n + CL - 1) / CL) + 31) & ~(int64_t)31) : n;
+    n = n < (int64_t)words * 32 ? n : (int64_t)words * 32;
+    // this CTA's part [p0, p1) of the row
+    const int64_t part = CL > 1 ? ((n + CL - 1) / CL) : n;
     const int64_t p0 = (int64_t)crank * part < n ? (int64_t)crank * part : n;
     const int64_t p1 = p0 + part < n ? p0 + part : n;
-    const int nrounds = (int)((p1 - p0 + RS - 1) / RS);
-    // raw bits; the order-preserving key is formed where it is used, so that no thread
-    // waits for these loads before the histogram step
-    uint32_t raw[kBmPer];
     const uint32_t* src = a.scores ? reinterpret_cast<const uint32_t*>(a.scores) : a.keys;
-    auto load_round = [&](int64_t base) {
-#pragma unroll
-        for (int j = 0; j < kBmPer; ++j) {
-            const int64_t e = base + (int64_t)j * NT + tid;
-            raw[j] = e < p1 ? ld_dep(src + (int64_t)r * a.ld + e) : 0u;
-        }
+    const uint32_t* rowp = src + (int64_t)r * a.ld;
+    // whole 16-byte units [b0, b1) by bulk copies; [p0, b0) and [b1, p1) read directly
+    const int64_t lead = (int64_t)(((16u - (reinterpret_cast<uintptr_t>(rowp + p0) & 15u)) & 15u) >> 2);
+    const int64_t b0 = p0 + lead < p1 ? p0 + lead : p1;
+    const int64_t b1 = b0 + ((p1 - b0) & ~(int64_t)3);
+    const int nch = (int)((b1 - b0 + CE - 1) / CE);
+    auto issue = [&](int c) {
+        const int64_t e0 = b0 + (int64_t)c * CE;
+        const int64_t cnt = b1 - e0 < CE ? b1 - e0 : CE;
+        const int slot = c % ring;
+        mbar_arrive_expect_tx(&bar[1 + slot], (uint32_t)(cnt * 4));
+        bulk_load(const_cast<uint32_t*>(buf) + (size_t)slot * CE, rowp + e0, (uint32_t)(cnt * 4), &bar[1 + slot]);
     };
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], 4u * kBinsT);
+        bulk_load(hist, a.hist + (int64_t)r * kBinsT, 4u * kBinsT, &bar[0]);
+        for (int c = 0; c < nch && c < ring; ++c) issue(c);
+    }
+    // the stray elements: one per thread among the first few
+    const int64_t xi = tid < b0 - p0 ? p0 + tid : (tid - (b0 - p0) < p1 - b1 ? b1 + (tid - (b0 - p0)) : -1);
+    const uint32_t xraw = xi >= 0 ? ld_dep(rowp + xi) : 0u;
     auto key_of = [&](uint32_t v) { return a.scores ? score_key(__uint_as_float(v)) : v; };
-    if (nrounds > 0) load_round(p0);   // in flight while the histogram arrives
 
     // ---- d0: the first digit that holds the K-th best element (every CTA) -------------------
-    mbar_wait(&bar, 0, a.status);
+    bool ok = mbar_wait(&bar[0], 0, a.status);
     uint32_t b[BPT], local = 0;
 #pragma unroll
     for (int j = 0; j < BPT; ++j) {   // thread 0 owns the highest bins, highest first
@@ -958,55 +978,74 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
         cand0 = peer_addr(cand, 0);
         cnt0 = peer_addr(cnt_s, 0);
     }
-    uint32_t nwin_w = 0;   // lane 0: this warp's winners
-    for (int rd = 0; rd < nrounds; ++rd) {
-        const int64_t base = p0 + (int64_t)rd * RS;
-        if (rd > 0) load_round(base);
-        // winners' words, and the warp's candidate count
+    auto set_bit = [&](int64_t pos) {
+        if constexpr (CL > 1) red_or_peer_u32(bm0 + 4u * (uint32_t)(pos >> 5), 1u << (pos & 31));
+        else atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+    };
+    auto put_cand = [&](uint32_t q, uint64_t c) {
+        if (q >= (uint32_t)kBmCands) return;
+        if constexpr (CL > 1) st_peer_u64(cand0 + 8u * q, c);
+        else cand[q] = c;
+    };
+    auto reserve = [&](uint32_t cnt) -> uint32_t {
+        if constexpr (CL > 1) return atom_add_peer_u32(cnt0, cnt);
+        else return atomicAdd(&cnt_s[0], cnt);
+    };
+    uint32_t nwin_t = 0;   // this thread's winners
+    if (xi >= 0) {
+        const uint32_t kk = key_of(xraw);
+        const int dig = (int)(kk >> 20);
+        if (!many || dig > d0) {
+            set_bit(xi);
+            ++nwin_t;
+        } else if (dig == d0) {
+            put_cand(reserve(1u), ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)xi));
+        }
+    }
+    for (int c = 0; c < nch; ++c) {
+        const int slot = c % ring;
+        if (!mbar_wait(&bar[1 + slot], (uint32_t)((c / ring) & 1), a.status)) ok = false;
+        const int64_t e0 = b0 + (int64_t)c * CE;
+        const int cnt = (int)(b1 - e0 < CE ? b1 - e0 : CE);
+        const uint32_t* cb_ = buf + (size_t)slot * CE;
+        uint32_t key[kBmPer];
         uint32_t ncw = 0;
 #pragma unroll
         for (int j = 0; j < kBmPer; ++j) {
-            if (base + (int64_t)j * NT >= p1) break;                 // the same for every warp
-            const int64_t e0 = base + (int64_t)j * NT + warp * 32;   // the warp's first position
-            const bool ok = e0 + lane < p1;
-            const int dig = (int)(key_of(raw[j]) >> 20);
-            const uint32_t wb = __ballot_sync(0xffffffffu, ok && (!many || dig > d0));
-            ncw += (uint32_t)__popc(__ballot_sync(0xffffffffu, ok && many && dig == d0));
-            if (lane == 0 && e0 < p1) {
-                if constexpr (CL > 1) st_peer_u32(bm0 + 4u * (uint32_t)(e0 >> 5), wb);
-                else bm[e0 >> 5] = wb;
-                nwin_w += __popc(wb);
+            const int i = j * NT + tid;
+            key[j] = i < cnt ? key_of(cb_[i]) : 0u;
+            const int dig = (int)(key[j] >> 20);
+            if (i < cnt && (!many || dig > d0)) {
+                set_bit(e0 + i);
+                ++nwin_t;
             }
+            ncw += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < cnt && many && dig == d0));
         }
-        if (ncw == 0) continue;
-        // one atomic per warp reserves its candidates' slots
-        uint32_t q = 0;
-        if (lane == 0) {
-            if constexpr (CL > 1) q = atom_add_peer_u32(cnt0, ncw);
-            else q = atomicAdd(&cnt_s[0], ncw);
-        }
-        q = __shfl_sync(0xffffffffu, q, 0);
+        __syncthreads();   // every thread has read the slot: refill it
+        if (tid == 0 && ok && c + ring < nch) issue(c + ring);
+        if (ncw) {
+            // one atomic per warp reserves its candidates' slots
+            uint32_t q = 0;
+            if (lane == 0) q = reserve(ncw);
+            q = __shfl_sync(0xffffffffu, q, 0);
 #pragma unroll
-        for (int j = 0; j < kBmPer; ++j) {
-            if (base + (int64_t)j * NT >= p1) break;
-            const int64_t e = base + (int64_t)j * NT + warp * 32 + lane;
-            const uint32_t kk = key_of(raw[j]);
-            const bool c = e < p1 && (int)(kk >> 20) == d0;
-            const uint32_t cb = __ballot_sync(0xffffffffu, c);
-            if (c) {
-                const uint32_t qi = q + __popc(cb & ((1u << lane) - 1u));
-                const uint64_t comp = ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)e);
-                if (qi < (uint32_t)kBmCands) {
-                    if constexpr (CL > 1) st_peer_u64(cand0 + 8u * qi, comp);
-                    else cand[qi] = comp;
-                }
+            for (int j = 0; j < kBmPer; ++j) {
+                const int i = j * NT + tid;
+                const bool isc = i < cnt && many && (int)(key[j] >> 20) == d0;
+                const uint32_t cb = __ballot_sync(0xffffffffu, isc);
+                if (isc)
+                    put_cand(q + __popc(cb & ((1u << lane) - 1u)),
+                             ((uint64_t)key[j] << 32) | (uint64_t)(~(uint32_t)(e0 + i)));
+                q += (uint32_t)__popc(cb);
             }
-            q += (uint32_t)__popc(cb);
         }
     }
-    if (lane == 0 && nwin_w) {
-        if constexpr (CL > 1) atom_add_peer_u32(cnt0 + 4u, nwin_w);
-        else atomicAdd(&cnt_s[1], nwin_w);
+    // this warp's winners
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nwin_t += __shfl_xor_sync(0xffffffffu, nwin_t, o);
+    if (lane == 0 && nwin_t) {
+        if constexpr (CL > 1) atom_add_peer_u32(cnt0 + 4u, nwin_t);
+        else atomicAdd(&cnt_s[1], nwin_t);
     }
     if constexpr (CL > 1) {
         // every part is in the first CTA's shared memory; the others are done
@@ -1111,16 +1150,25 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
 }
 
 template <int NT, int CL>
-static cudaError_t launch_bitmap(const TopkDev& a, int R, cudaStream_t st) {
+static cudaError_t launch_bitmap(TopkDev a, int64_t max_n, int R, cudaStream_t st) {
+    // bitmap words for the longest row; as many chunk buffers as fit beside it (two per SM
+    // for 512-thread CTAs: at most 113 KiB each), between 2 and 4
+    a.bitmap_words = (int)((max_n + 127) / 128 * 4);
+    const size_t cap = NT == 512 ? 113 * 1024 : 227 * 1024;
+    int ring = 4;
+    while (ring > 2 && bm_smem(a.bitmap_words, NT, ring) > cap) --ring;
+    a.ring = ring;
+    const size_t smem = bm_smem(a.bitmap_words, NT, ring);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
     auto kern = topk_bitmap_kernel<NT, CL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBmSmem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (CL == 1) return launch_pdl(kern, dim3((unsigned)R), dim3(NT), kBmSmem, st, a);
+    if (CL == 1) return launch_pdl(kern, dim3((unsigned)R), dim3(NT), smem, st, a);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3(CL, (unsigned)R);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = kBmSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1155,6 +1203,8 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     a.cands = l.cands;
     a.ccap = l.ccap;
     a.status = l.status;
+    a.bitmap_words = 0;
+    a.ring = 0;
     // ids are < id_bound: a bitmap of that many bits orders the picks when it fits
     const int64_t words = (l.id_bound + 31) / 32;
     cudaError_t e;
@@ -1163,11 +1213,11 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
         // 1024-thread CTAs (one per SM) while four per row fit, else 512-thread CTAs (two
         // per SM), with at least 4,096 elements per CTA.
         const int sms = device_sm_count();
-        if (l.max_n >= 4 * 8192 && l.R * 4 <= sms) return launch_bitmap<1024, 4>(a, l.R, st);
-        if (l.max_n >= 8 * 4096 && l.R * 8 <= 2 * sms) return launch_bitmap<512, 8>(a, l.R, st);
-        if (l.max_n >= 4 * 4096 && l.R * 4 <= 2 * sms) return launch_bitmap<512, 4>(a, l.R, st);
-        if (l.max_n >= 2 * 4096 && l.R * 2 <= 2 * sms) return launch_bitmap<512, 2>(a, l.R, st);
-        return launch_bitmap<512, 1>(a, l.R, st);
+        if (l.max_n >= 4 * 8192 && l.R * 4 <= sms) return launch_bitmap<1024, 4>(a, l.max_n, l.R, st);
+        if (l.max_n >= 8 * 4096 && l.R * 8 <= 2 * sms) return launch_bitmap<512, 8>(a, l.max_n, l.R, st);
+        if (l.max_n >= 4 * 4096 && l.R * 4 <= 2 * sms) return launch_bitmap<512, 4>(a, l.max_n, l.R, st);
+        if (l.max_n >= 2 * 4096 && l.R * 2 <= 2 * sms) return launch_bitmap<512, 2>(a, l.max_n, l.R, st);
+        return launch_bitmap<512, 1>(a, l.max_n, l.R, st);
     }
     if (l.ids && l.max_n <= kRowMaxN) {
         // the bitmap of ids may cover up to 2^20 ids
