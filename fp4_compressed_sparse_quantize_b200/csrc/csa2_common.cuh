@@ -119,13 +119,8 @@ __device__ __forceinline__ void st_peer_u32(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void st_peer_u64(uint32_t addr, uint64_t v) {
     asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
-__device__ __forceinline__ void red_or_peer_u32(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared::cluster.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t atom_add_peer_u32(uint32_t addr, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
-    return old;
+__device__ __forceinline__ void red_add_peer_u32(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
     float4 v;

@@ -833,11 +833,12 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_gather_kernel(const TopkD
 // of winners is kept, so the block-wide steps are d0, one barrier per chunk, the refinement
 // passes and the final prefix sum.
 constexpr int kBmPer = 8;                     // elements per thread per chunk
-constexpr int kBmCands = 4096;                // candidates kept in shared memory
+constexpr int kBmCands = 3968;                // candidates kept in shared memory
 constexpr int64_t kBmMaxN = 262144;
 constexpr size_t kBmOffHist = 0;                                   // u32[4096]
 constexpr size_t kBmOffCand = kBmOffHist + 4 * kBinsT;             // u64[kBmCands]
-constexpr size_t kBmOffBm = kBmOffCand + 8 * (size_t)kBmCands;     // u32[bitmap words]
+constexpr size_t kBmOffH2 = kBmOffCand + 8 * (size_t)kBmCands;     // u32[256]
+constexpr size_t kBmOffBm = kBmOffH2 + 4 * 256;                      // u32[bitmap words]
 __host__ __device__ constexpr size_t bm_off_ring(int words) {
     return (kBmOffBm + 4 * (size_t)words + 127) & ~(size_t)127;
 }
@@ -889,11 +890,15 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
     uint32_t* hist = reinterpret_cast<uint32_t*>(dsm + kBmOffHist);
     uint64_t* cand = reinterpret_cast<uint64_t*>(dsm + kBmOffCand);
     uint32_t* bm = reinterpret_cast<uint32_t*>(dsm + kBmOffBm);
+    // the candidates' next 8 key bits, counted as they are found: the first refinement
+    // pass's histogram
+    uint32_t* h2 = reinterpret_cast<uint32_t*>(dsm + kBmOffH2);
     const uint32_t* buf = reinterpret_cast<const uint32_t*>(dsm + bm_off_ring(words));
     uint64_t* bar = reinterpret_cast<uint64_t*>(dsm + bm_off_bar(words, NT, ring));
     __shared__ uint32_t wsum[40];
     __shared__ int dig_s[4];
-    __shared__ uint32_t cnt_s[2];   // candidates, winners
+    __shared__ uint32_t cnt_s[2];   // this CTA's candidates and winners
+    __shared__ uint32_t part_s[16]; // first CTA: every CTA's candidate, then winner count
     const int r = CL > 1 ? (int)blockIdx.y : (int)blockIdx.x;
     const uint32_t crank = CL > 1 ? cluster_rank() : 0u;
     const int tid = threadIdx.x, lane = tid & 31;
@@ -906,19 +911,22 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
         dig_s[0] = -1;
         dig_s[1] = 0;
     }
-    for (int i = tid; i < words; i += NT) bm[i] = 0u;
+    for (int i = tid; i < 256; i += NT) h2[i] = 0u;
     __syncthreads();
-    // the first CTA's bitmap and counters are cleared before any CTA of the cluster writes
+    // every CTA of the cluster has started before any writes another's shared memory (the
+    // matching wait comes after the classification)
     if constexpr (CL > 1) cluster_arrive();
     grid_dep_wait();
 
     int64_t n = row_len(a, r);
     n = n < 0 ? 0 : (n > a.ld ? a.ld : n);
     n = n < (int64_t)words * 32 ? n : (int64_t)words * 32;
-    // this CTA's part [p0, p1) of the row
-    const int64_t part = CL > 1 ? ((n + CL - 1) / CL) : n;
+    // this CTA's part [p0, p1) of the row: whole bitmap words, so that every CTA builds its
+    // own words in its own shared memory
+    const int64_t part = CL > 1 ? ((((n + CL - 1) / CL) + 31) & ~(int64_t)31) : n;
     const int64_t p0 = (int64_t)crank * part < n ? (int64_t)crank * part : n;
     const int64_t p1 = p0 + part < n ? p0 + part : n;
+    for (int64_t wi = (p0 >> 5) + tid; wi < ((p1 + 31) >> 5); wi += NT) bm[wi] = 0u;   // own words
     const uint32_t* src = a.scores ? reinterpret_cast<const uint32_t*>(a.scores) : a.keys;
     const uint32_t* rowp = src + (int64_t)r * a.ld;
     // whole 16-byte units [b0, b1) by bulk copies; [p0, b0) and [b1, p1) read directly
@@ -971,26 +979,16 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
 
     // ---- classify: winners into the bitmap, candidates into the list ----------------------------
     // (addresses in the first CTA of the cluster; plain shared memory without a cluster)
-    uint32_t bm0 = 0, cand0 = 0, cnt0 = 0;
-    if constexpr (CL > 1) {
-        cluster_wait();
-        bm0 = peer_addr(bm, 0);
-        cand0 = peer_addr(cand, 0);
-        cnt0 = peer_addr(cnt_s, 0);
-    }
-    auto set_bit = [&](int64_t pos) {
-        if constexpr (CL > 1) red_or_peer_u32(bm0 + 4u * (uint32_t)(pos >> 5), 1u << (pos & 31));
-        else atomicOr(&bm[pos >> 5], 1u << (pos & 31));
-    };
+    // Every CTA marks its own words of the bitmap and fills its own part of the candidate
+    // list in its own shared memory, both at the places they take in the first CTA; the
+    // others copy them there once classified.
+    constexpr uint32_t RC = (uint32_t)(kBmCands / CL);
+    auto set_bit = [&](int64_t pos) { atomicOr(&bm[pos >> 5], 1u << (pos & 31)); };
     auto put_cand = [&](uint32_t q, uint64_t c) {
-        if (q >= (uint32_t)kBmCands) return;
-        if constexpr (CL > 1) st_peer_u64(cand0 + 8u * q, c);
-        else cand[q] = c;
+        atomicAdd(&h2[(uint32_t)(c >> 44) & 0xFFu], 1u);
+        if (q < RC) cand[crank * RC + q] = c;
     };
-    auto reserve = [&](uint32_t cnt) -> uint32_t {
-        if constexpr (CL > 1) return atom_add_peer_u32(cnt0, cnt);
-        else return atomicAdd(&cnt_s[0], cnt);
-    };
+    auto reserve = [&](uint32_t cnt) -> uint32_t { return atomicAdd(&cnt_s[0], cnt); };
     uint32_t nwin_t = 0;   // this thread's winners
     if (xi >= 0) {
         const uint32_t kk = key_of(xraw);
@@ -1043,51 +1041,91 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
     // this warp's winners
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nwin_t += __shfl_xor_sync(0xffffffffu, nwin_t, o);
-    if (lane == 0 && nwin_t) {
-        if constexpr (CL > 1) atom_add_peer_u32(cnt0 + 4u, nwin_t);
-        else atomicAdd(&cnt_s[1], nwin_t);
-    }
+    if (lane == 0 && nwin_t) atomicAdd(&cnt_s[1], nwin_t);
+    __syncthreads();
     if constexpr (CL > 1) {
+        cluster_wait();
+        if (crank != 0) {
+            // this CTA's words, candidates and counts into the first CTA
+            const int64_t w0 = p0 >> 5, w1 = (p1 + 31) >> 5;
+            const uint32_t bm0 = peer_addr(bm, 0), cand0 = peer_addr(cand, 0);
+            for (int64_t wi = w0 + tid; wi < w1; wi += NT) st_peer_u32(bm0 + 4u * (uint32_t)wi, bm[wi]);
+            const uint32_t nc = min(cnt_s[0], RC);
+            for (uint32_t i = tid; i < nc; i += NT)
+                st_peer_u64(cand0 + 8u * (crank * RC + i), cand[crank * RC + i]);
+            const uint32_t h20 = peer_addr(h2, 0);
+            for (int i = tid; i < 256; i += NT)
+                if (h2[i]) red_add_peer_u32(h20 + 4u * i, h2[i]);
+            if (tid == 0) {
+                st_peer_u32(peer_addr(&part_s[crank], 0), cnt_s[0]);
+                st_peer_u32(peer_addr(&part_s[CL + crank], 0), cnt_s[1]);
+            }
+        } else if (tid == 0) {
+            part_s[0] = cnt_s[0];
+            part_s[CL] = cnt_s[1];
+        }
         // every part is in the first CTA's shared memory; the others are done
         cluster_arrive();
         cluster_wait();
         if (crank != 0) return;
-    } else {
-        __syncthreads();
     }
-    const uint32_t ncand = cnt_s[0], nwin_all = cnt_s[1];
+    auto part_cands = [&](int k) { return CL > 1 ? part_s[k] : cnt_s[0]; };
+    uint32_t ncand = 0, nwin_all = 0;
+    bool over = false;
+#pragma unroll
+    for (int k = 0; k < CL; ++k) {
+        const uint32_t c = part_cands(k);
+        ncand += c;
+        over |= c > RC;
+        nwin_all += CL > 1 ? part_s[CL + k] : cnt_s[1];
+    }
     if (tid == 0 && (nwin_all > (uint32_t)K || (many && nwin_all != above)))
         set_status(a.status, CSA2_DEV_BAD_COUNT);
 
     // ---- the exact `need`-th best candidate -------------------------------------------------------
     if (many) {
         const uint32_t need = (uint32_t)K - above;
-        const bool from_row = ncand > (uint32_t)kBmCands;   // list overflowed: read the row again
+        const bool from_row = over;   // a part of the list overflowed: read the row again
         const int64_t nsrc = from_row ? n : (int64_t)ncand;
+        // candidate i of the list: the parts follow one another
+        uint32_t pc[CL];
+#pragma unroll
+        for (int k = 0; k < CL; ++k) pc[k] = part_cands(k);
         auto cnd = [&](int64_t i, uint64_t& c) -> bool {
             if (from_row) {
                 const uint32_t kk = elem_key(a, r, i);
                 c = ((uint64_t)kk << 32) | (uint64_t)(~(uint32_t)i);
                 return (int)(kk >> 20) == d0;
             }
-            c = cand[i];
+            uint32_t j = (uint32_t)i, slot = j;
+#pragma unroll
+            for (int k = 0; k < CL; ++k) {
+                if (j < pc[k]) {
+                    slot = (uint32_t)k * RC + j;
+                    break;
+                }
+                j -= pc[k];
+            }
+            c = cand[slot];
             return true;
         };
         uint64_t prefix = (uint64_t)d0;
         int shift = 52;
         uint32_t rem = need;
         bool found = true;
-        while (shift > 0) {
+        for (int pass = 0; shift > 0; ++pass) {
             const int nb = shift < 8 ? shift : 8;
-            for (int i = tid; i < 256; i += NT) hist[i] = 0u;
-            __syncthreads();
-            for (int64_t i = tid; i < nsrc; i += NT) {
-                uint64_t c;
-                if (cnd(i, c) && (c >> shift) == prefix)
-                    atomicAdd(&hist[(c >> (shift - nb)) & ((1u << nb) - 1u)], 1u);
+            if (pass > 0) {   // the first pass's histogram is h2
+                for (int i = tid; i < 256; i += NT) hist[i] = 0u;
+                __syncthreads();
+                for (int64_t i = tid; i < nsrc; i += NT) {
+                    uint64_t c;
+                    if (cnd(i, c) && (c >> shift) == prefix)
+                        atomicAdd(&hist[(c >> (shift - nb)) & ((1u << nb) - 1u)], 1u);
+                }
+                __syncthreads();
             }
-            __syncthreads();
-            if (tid < 32) warp_find_digit256(hist, rem, dig_s);
+            if (tid < 32) warp_find_digit256(pass > 0 ? hist : h2, rem, dig_s);
             __syncthreads();
             const int d = dig_s[0];
             const uint32_t ab = (uint32_t)dig_s[1], inbin = (uint32_t)dig_s[2];
