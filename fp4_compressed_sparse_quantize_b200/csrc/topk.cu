@@ -926,7 +926,9 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
     const int64_t part = CL > 1 ? ((((n + CL - 1) / CL) + 31) & ~(int64_t)31) : n;
     const int64_t p0 = (int64_t)crank * part < n ? (int64_t)crank * part : n;
     const int64_t p1 = p0 + part < n ? p0 + part : n;
-    for (int64_t wi = (p0 >> 5) + tid; wi < ((p1 + 31) >> 5); wi += NT) bm[wi] = 0u;   // own words
+    // this CTA's words [w0, w1): its part starts on a word boundary unless it is empty
+    const int64_t pw0 = p0 >> 5, pw1 = p1 > p0 ? (p1 + 31) >> 5 : pw0;
+    for (int64_t wi = pw0 + tid; wi < pw1; wi += NT) bm[wi] = 0u;
     const uint32_t* src = a.scores ? reinterpret_cast<const uint32_t*>(a.scores) : a.keys;
     const uint32_t* rowp = src + (int64_t)r * a.ld;
     // whole 16-byte units [b0, b1) by bulk copies; [p0, b0) and [b1, p1) read directly
@@ -1047,9 +1049,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
         cluster_wait();
         if (crank != 0) {
             // this CTA's words, candidates and counts into the first CTA
-            const int64_t w0 = p0 >> 5, w1 = (p1 + 31) >> 5;
             const uint32_t bm0 = peer_addr(bm, 0), cand0 = peer_addr(cand, 0);
-            for (int64_t wi = w0 + tid; wi < w1; wi += NT) st_peer_u32(bm0 + 4u * (uint32_t)wi, bm[wi]);
+            for (int64_t wi = pw0 + tid; wi < pw1; wi += NT) st_peer_u32(bm0 + 4u * (uint32_t)wi, bm[wi]);
             const uint32_t nc = min(cnt_s[0], RC);
             for (uint32_t i = tid; i < nc; i += NT)
                 st_peer_u64(cand0 + 8u * (crank * RC + i), cand[crank * RC + i]);

@@ -135,7 +135,10 @@ def _full_decode(q_I, w, k_I, n_vis, K, pool_blocks=0):
 
 @pytest.mark.parametrize("dtype,H_I,K", [(torch.bfloat16, 8, 64), (torch.float8_e4m3fn, 64, 512),
                                          (torch.float8_e4m3fn, 16, 32)])
-@pytest.mark.parametrize("n_list", [[1, 7, 16], [511, 512, 513], [4096, 1000, 129]])
+@pytest.mark.parametrize("n_list", [[1, 7, 16], [511, 512, 513], [4096, 1000, 129],
+                                    # long rows split over a cluster, beside short rows whose
+                                    # later parts are empty
+                                    [40000, 9, 70], [20000, 5, 4100]])
 def test_full_decode_scores_and_topk(dtype, H_I, K, n_list):
     g = _gen(sum(n_list) + H_I)
     B = len(n_list)
