@@ -80,6 +80,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     }
 }
 
+// ---- flags between the warps of a CTA ------------------------------------------------
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+// Waits until the shared flag is nonzero (nonzero = true; returns it) or zero (returns 0),
+// or until *stop is set by another warp (returns -1), bounded like mbar_wait (returns -1 and
+// sets CSA2_DEV_TIMEOUT when the limit passes).
+__device__ __forceinline__ int flag_wait(const int* f, bool nonzero, const volatile int* stop,
+                                         int32_t* status, uint64_t limit_ns = kWaitLimitNs) {
+    uint64_t t0 = 0;
+#pragma unroll 1
+    for (uint32_t i = 0;; ++i) {
+        const int v = ld_acquire_cta(f);
+        if ((v != 0) == nonzero) return v;
+        if (*stop) return -1;
+        if (i == 256) t0 = global_timer_ns();
+        if (i > 256 && (i & 63) == 0 && global_timer_ns() - t0 > limit_ns) {
+            set_status(status, CSA2_DEV_TIMEOUT);
+            return -1;
+        }
+    }
+}
+
 // ---- cluster helpers (distributed shared memory) -------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;

@@ -199,6 +199,8 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
     // set when the wait for this CTA's last MMA commit gave up: MMAs may still be in flight,
     // so neither TMEM nor the shared-memory operands may be released or reused
     volatile int* mma_stuck = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 16);
+    // the waiter's verdicts for the MMA issuer, two tiles deep: 0 = empty, 1 = go, 2 = stop
+    int* go_ring = reinterpret_cast<int*>(smem + L::kMiscOff + 24);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -221,6 +223,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         mbar_init(done_bar, 1);
         *abort_flag = 0;
         *mma_stuck = 0;
+        go_ring[0] = go_ring[1] = 0;
         fence_mbar_init();
     }
     if (warp >= kEpiWarp0) {
@@ -342,11 +345,11 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         // ------------------------------------------------------------ MMA issue (warp 1)
         // and its barrier waits (warp 2). An mbarrier wait by the thread whose MMAs and
         // commits are still in flight costs a few hundred cycles even on a completed phase,
-        // so the issuing thread never waits on an mbarrier: warp 2 waits for tile t+1's key
-        // tile, accumulator and query slot while warp 1 issues tile t, and the two meet at a
-        // named barrier once per tile. The waiter's verdict (go / abort) crosses with it, so
-        // both warps always take the same number of hand-overs.
-        volatile int* go_flag = abort_flag + 1;
+        // so the issuing thread never waits on an mbarrier: warp 2 waits for the key tile,
+        // accumulator and query slot of each tile and posts its verdict (go / stop) in a
+        // two-slot ring, up to two tiles ahead of warp 1, which reads the verdict with an
+        // acquiring load and issues. Both walk the same tile sequence, and every wait on the
+        // ring is bounded.
         const bool waiter = warp == 2;
         GroupCursor cur;
         cur.init(p.prefix, ngroups, t0);
@@ -360,25 +363,33 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
             const int qs_new = newgroup ? (qcount & 1) : qs;
             const int s = (int)(it % STAGES);
             const int a = (int)(it % ACC);
+            int* slot = go_ring + (int)(it & 1);
             if (waiter) {
                 bool ok = true;
                 if (lane == 0) {
                     ok = !*abort_flag;
+                    // the issuer has taken the verdict of tile it - 2
+                    if (ok) ok = flag_wait(slot, false, abort_flag, p.status) == 0;
                     if (ok && newgroup)
                         ok = mbar_wait(&qfull[qs_new], (uint32_t)((qcount >> 1) & 1), p.status);
                     if (ok) ok = mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), p.status);
                     if (ok) ok = mbar_wait(&accempty[a], (uint32_t)(((it / ACC) & 1) ^ 1), p.status);
                     if (!ok) *abort_flag = 1;
-                    *go_flag = ok ? 1 : 0;
+                    st_release_cta(slot, ok ? 1 : 2);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                named_bar_sync(15, 64);
                 if (!ok) break;
             } else {
                 // the previous row group's query slot is free once this thread's MMAs are done
                 if (lane == 0 && newgroup && qg >= 0) mma_commit(&qempty[qs]);
-                named_bar_sync(15, 64);
-                if (!*go_flag) break;
+                int v = 0;
+                if (lane == 0) {
+                    v = flag_wait(slot, true, abort_flag, p.status);
+                    if (v != 1) *abort_flag = 1;
+                    st_release_cta(slot, 0);
+                }
+                v = __shfl_sync(0xffffffffu, v, 0);
+                if (v != 1) break;
                 if (lane == 0) {
                     tc_fence_after();
                     // descriptor start addresses advance in 16-byte units
