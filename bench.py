@@ -46,8 +46,8 @@ SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csr
 # dram__bytes_write.sum` (summary in profiles/), valid only for the indexer.cu it was taken
 # on: {workload: (sha1 of indexer.cu, bytes per launch)}.
 SCAN_TRAFFIC = {
-    "decode_full_b32_ctx64k_r2": ("142becb2fc943407bedee0561cf40e1ae3746235",
-                                  134709248 + 3598848),
+    "decode_full_b32_ctx64k_r2": ("0fdccf3561f73aa507efd6d197853de125eac5af",
+                                  134705152 + 3618048),
 }
 
 
