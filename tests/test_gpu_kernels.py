@@ -189,6 +189,33 @@ def test_topk_degenerate_all_equal_scores():
     assert np.all(scores[0, 0] == 0.0)
 
 
+def test_topk_tied_maximum_overflowing_one_cluster_part():
+    """The row's best key repeated 3,000 times: exact ties at the top, so the K lowest of
+    those positions win. Rows of 40,000 entries split over a 4-CTA cluster (parts of ~10,000):
+    row 0 puts every copy in the first part, row 1 straddles the first two parts; either way
+    one part holds more candidates than its share of the list, and the selection goes back
+    to the row."""
+    g = _gen(9)
+    n, K = 40000, 512
+    k_I = torch.randn((2, n, 128), generator=g).to(torch.float8_e4m3fn)
+    q_I = torch.randn((2, 1, 64, 128), generator=g).to(torch.float8_e4m3fn)
+    w = torch.rand((2, 1, 64), generator=g)
+    starts = [0, 9000]
+    for b in range(2):
+        s = O.index_scores(raw_qk(q_I[b, 0]), w[b, 0].numpy(), raw_qk(k_I[b]), O.E4M3)
+        best = int(np.argmax(s))
+        k_I[b, starts[b]:starts[b] + 3000] = k_I[b, best]
+    idx, scores, _, st = _full_decode(q_I, w, k_I, [n, n], K)
+    assert st == 0
+    for b in range(2):
+        copies = np.arange(starts[b], starts[b] + 3000)
+        assert np.all(scores[b, 0, copies] == scores[b, 0, copies[0]])
+        assert np.all(scores[b, 0] <= scores[b, 0, copies[0]])
+        want = np.sort(np.concatenate([copies, np.nonzero(scores[b, 0] == scores[b, 0, copies[0]])[0]]))
+        want = np.unique(want)[:K]
+        np.testing.assert_array_equal(idx[b, 0], want)
+
+
 def test_topk_many_ties_mixed():
     """Integer-valued scores with heavy ties: one-hot keys and a one-head query."""
     g = _gen(8)
