@@ -46,7 +46,7 @@ SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csr
 # dram__bytes_write.sum` (summary in profiles/), valid only for the indexer.cu it was taken
 # on: {workload: (sha1 of indexer.cu, bytes per launch)}.
 SCAN_TRAFFIC = {
-    "decode_full_b32_ctx64k_r2": ("0fdccf3561f73aa507efd6d197853de125eac5af",
+    "decode_full_b32_ctx64k_r2": ("d4aec0c726679d57f6541074179e0477938198ac",
                                   134705152 + 3618048),
 }
 

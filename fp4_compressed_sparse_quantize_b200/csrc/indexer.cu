@@ -19,8 +19,9 @@
 //               row group.
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128 keys,
 //               N = G queries x H_I heads, K = 128 channels) into a TMEM accumulator ring.
-//   warp 2      does warp 1's mbarrier waits one tile ahead and hands each tile over at a
-//               named barrier (a wait behind in-flight MMA commits is slow).
+//   warp 2      does warp 1's mbarrier waits (a wait behind in-flight MMA commits is slow)
+//               and posts a go / stop verdict per tile in a two-slot flag ring, up to two
+//               tiles ahead of warp 1.
 //   then EPI    epilogue groups of 4 warps: tcgen05.ld of one key row per thread,
 //               ReLU-weighted head sum in fp32, coalesced score stores, shared-memory
 //               histogram of the top 12 key bits per query row (first radix-select digit),
@@ -742,7 +743,7 @@ template <int NQ, int ESZ, int G, bool GATHER, bool POOL, bool KF4 = false>
 static cudaError_t launch_scan_t(const CUtensorMap& mk, const CUtensorMap& mq,
                                  const ScanParams& p, cudaStream_t st) {
     // 384-key tiles for one FP8 query row per tile and 256-key tiles for two (prefill): the
-    // per-tile hand-over (mbarrier waits behind in-flight commits, the named barrier, the
+    // per-tile hand-over (mbarrier waits behind in-flight commits, the verdict, the
     // commits) costs about the same whatever the tile holds, so the tiles are as large as
     // two accumulators allow; two epilogue groups whenever the TMEM accumulators split
     // evenly between them
