@@ -616,6 +616,73 @@ __device__ __forceinline__ void row_threshold(const RowState& S, const uint32_t 
     __syncthreads();
 }
 
+// Emits the set bits of bm[0, nwords) in ascending order into output slots [0, K): the bit's
+// index, or the 8 positions of that block (positions >= lim as -1) with expand8; pads the
+// remaining slots with -1. Groups of 32 words are read by whole warps, one word per lane
+// (conflict-free), and each warp owns a contiguous run of groups; a warp-level prefix sum
+// gives every word its first slot. Block-wide (contains barriers); wsum takes 33 words.
+template <int NT>
+__device__ void emit_bitmap(const uint32_t* bm, int64_t nwords, int K, int32_t* o, bool expand8,
+                            int32_t lim, uint32_t* wsum) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t ngroups = (nwords + 31) >> 5;
+    const int64_t gpw = (ngroups + NW - 1) / NW;
+    const int64_t g0 = warp * gpw, g1 = g0 + gpw < ngroups ? g0 + gpw : ngroups;
+    auto word = [&](int64_t g) { const int64_t wi = g * 32 + lane; return wi < nwords ? bm[wi] : 0u; };
+    uint32_t wtot = 0;
+    for (int64_t g = g0; g < g1; ++g) wtot += __reduce_add_sync(0xffffffffu, (uint32_t)__popc(word(g)));
+    if (lane == 0) wsum[warp] = wtot;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t x = lane < NW ? wsum[lane] : 0u;
+        uint32_t xi = x;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, xi, d);
+            if (lane >= d) xi += u;
+        }
+        if (lane < NW) wsum[lane] = xi - x;
+        if (lane == 31) wsum[32] = xi;
+    }
+    __syncthreads();
+    uint32_t base = wsum[warp];
+    const uint32_t total = wsum[32];
+    for (int64_t g = g0; g < g1 && base < (uint32_t)K; ++g) {
+        uint32_t w = word(g);
+        const uint32_t pc = (uint32_t)__popc(w);
+        uint32_t incl = pc;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        uint32_t slot = base + incl - pc;
+        const int64_t wbase = (g * 32 + lane) * 32;
+        while (w) {
+            const int bit = __ffs(w) - 1;
+            w &= w - 1;
+            if (slot < (uint32_t)K) {
+                const int64_t id = wbase + bit;
+                if (!expand8) {
+                    o[slot] = (int32_t)id;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int64_t pos = id * 8 + e;
+                        o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
+                    }
+                }
+            }
+            ++slot;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int npick = (int)(total < (uint32_t)K ? total : (uint32_t)K);
+    const int mult = expand8 ? 8 : 1;
+    for (int i = npick * mult + (int)threadIdx.x; i < K * mult; i += NT) o[i] = -1;
+}
+
 // Refinement, picks and the ordered output of one gathered row, after every element was
 // classified.
 __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t n,
@@ -717,24 +784,12 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
             }
         }
     };
-    int npick;
     if (use_bm) {
-        const int per = (nwords + kRowThreads - 1) / kRowThreads;
-        const int w0 = tid * per, w1 = min(nwords, w0 + per);
-        uint32_t cntb = 0;
-        for (int wi = w0; wi < w1; ++wi) cntb += __popc(S.bm[wi]);
-        uint32_t tot;
-        uint32_t off = row_excl_scan(cntb, S.wsum, tot);
-        npick = (int)min(tot, (uint32_t)K);
-        for (int wi = w0; wi < w1; ++wi) {
-            uint32_t m = S.bm[wi];
-            while (m) {
-                const int b = __ffs(m) - 1;
-                m &= m - 1;
-                emit(off++, (int64_t)wi * 32 + b);
-            }
-        }
-    } else {
+        emit_bitmap<kRowThreads>(S.bm, nwords, K, o, a.expand8, lim, S.wsum);
+        return;
+    }
+    int npick;
+    {
         // winners occupy [0, nwin), candidates were appended from tot_s[0] = nwin_all on
         npick = (int)min(many ? S.tot_s[0] : nwin, (uint32_t)K);
         for (int i = tid; i < npick; i += kRowThreads) {
@@ -1155,37 +1210,9 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
     }
 
     // ---- emit the set bits in ascending position order -------------------------------------------
-    const int64_t nwords = (n + 31) >> 5;
     const int32_t lim = a.expand8 ? ld_dep(a.expand_limit + r) : 0;
-    int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
-    const int64_t per = (nwords + NT - 1) / NT;
-    const int64_t w0 = tid * per, w1 = w0 + per < nwords ? w0 + per : nwords;
-    uint32_t cntb = 0;
-    for (int64_t wi = w0; wi < w1; ++wi) cntb += __popc(bm[wi]);
-    uint32_t tot;
-    uint32_t off = bm_excl_scan<NT>(cntb, wsum, tot);
-    const int npick = (int)min(tot, (uint32_t)K);
-    for (int64_t wi = w0; wi < w1; ++wi) {
-        uint32_t m = bm[wi];
-        while (m) {
-            const int bit = __ffs(m) - 1;
-            m &= m - 1;
-            const uint32_t slot = off++;
-            if (slot >= (uint32_t)K) continue;
-            const int64_t id = wi * 32 + bit;
-            if (!a.expand8) {
-                o[slot] = (int32_t)id;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int64_t pos = id * 8 + e;
-                    o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
-                }
-            }
-        }
-    }
-    const int mult = a.expand8 ? 8 : 1;
-    for (int i = npick * mult + tid; i < K * mult; i += NT) o[i] = -1;
+    emit_bitmap<NT>(bm, (n + 31) >> 5, K, a.out + (int64_t)r * K * (a.expand8 ? 8 : 1), a.expand8, lim,
+                    wsum);
 }
 
 template <int NT, int CL>
