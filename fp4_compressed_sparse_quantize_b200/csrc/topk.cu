@@ -174,6 +174,111 @@ __device__ __forceinline__ bool cand_at(const TopkDev& a, int r, const CandSourc
     return (int)(c >> 52) == s.d0;
 }
 
+// Warp 0 only: over bins h[0..256) (counts), find d with above(d) < rem <= above(d) + h[d],
+// above(d) = sum of h[e] for e > d. Writes d (or -1 when the total is < rem), above(d) and
+// h[d] into out[0..3).
+__device__ __forceinline__ void warp_find_digit256(const uint32_t* h, uint32_t rem, int* out) {
+    const int lane = threadIdx.x & 31;
+    uint32_t b[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {   // lane 0 owns the 8 highest bins, highest first
+        b[j] = h[255 - 8 * lane - j];
+        sum += b[j];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    const uint32_t excl = incl - sum;
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0 && total < rem) {
+        out[0] = -1;
+        out[1] = (int)total;
+        out[2] = 0;
+    }
+    if (excl < rem && incl >= rem) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (acc < rem && acc + b[j] >= rem) {
+                out[0] = 255 - 8 * lane - j;
+                out[1] = (int)acc;
+                out[2] = (int)b[j];
+            }
+            acc += b[j];
+        }
+    }
+}
+
+// Emits the set bits of bm[0, nwords) in ascending order into output slots [0, K): the bit's
+// index, or the 8 positions of that block (positions >= lim as -1) with expand8; pads the
+// remaining slots with -1. Groups of 32 words are read by whole warps, one word per lane
+// (conflict-free), and each warp owns a contiguous run of groups; a warp-level prefix sum
+// gives every word its first slot. Block-wide (contains barriers); wsum takes 33 words.
+template <int NT>
+__device__ void emit_bitmap(const uint32_t* bm, int64_t nwords, int K, int32_t* o, bool expand8,
+                            int32_t lim, uint32_t* wsum) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t ngroups = (nwords + 31) >> 5;
+    const int64_t gpw = (ngroups + NW - 1) / NW;
+    const int64_t g0 = warp * gpw, g1 = g0 + gpw < ngroups ? g0 + gpw : ngroups;
+    auto word = [&](int64_t g) { const int64_t wi = g * 32 + lane; return wi < nwords ? bm[wi] : 0u; };
+    uint32_t wtot = 0;
+    for (int64_t g = g0; g < g1; ++g) wtot += __reduce_add_sync(0xffffffffu, (uint32_t)__popc(word(g)));
+    if (lane == 0) wsum[warp] = wtot;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t x = lane < NW ? wsum[lane] : 0u;
+        uint32_t xi = x;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, xi, d);
+            if (lane >= d) xi += u;
+        }
+        if (lane < NW) wsum[lane] = xi - x;
+        if (lane == 31) wsum[32] = xi;
+    }
+    __syncthreads();
+    uint32_t base = wsum[warp];
+    const uint32_t total = wsum[32];
+    for (int64_t g = g0; g < g1 && base < (uint32_t)K; ++g) {
+        uint32_t w = word(g);
+        const uint32_t pc = (uint32_t)__popc(w);
+        uint32_t incl = pc;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        uint32_t slot = base + incl - pc;
+        const int64_t wbase = (g * 32 + lane) * 32;
+        while (w) {
+            const int bit = __ffs(w) - 1;
+            w &= w - 1;
+            if (slot < (uint32_t)K) {
+                const int64_t id = wbase + bit;
+                if (!expand8) {
+                    o[slot] = (int32_t)id;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int64_t pos = id * 8 + e;
+                        o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
+                    }
+                }
+            }
+            ++slot;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int npick = (int)(total < (uint32_t)K ? total : (uint32_t)K);
+    const int mult = expand8 ? 8 : 1;
+    for (int i = npick * mult + (int)threadIdx.x; i < K * mult; i += NT) o[i] = -1;
+}
+
 // Smallest composite T such that exactly `need` candidates are >= T (composites are
 // unique). 8-bit radix refinement below the known top 12 bits; stops as soon as the chosen
 // bin is taken whole.
@@ -192,14 +297,17 @@ __device__ uint64_t refine_threshold(const TopkDev& a, int r, const CandSource& 
                 atomicAdd(&hist256[(c >> (shift - nb)) & ((1u << nb) - 1u)], 1u);
         }
         __syncthreads();
-        int d;
-        uint32_t ab;
-        if (!find_digit(hist256, 1 << nb, rem, d, ab, red)) {
+        // one warp scans the (zero-padded) 256 bins
+        int* dig = reinterpret_cast<int*>(red);
+        if (threadIdx.x < 32) warp_find_digit256(hist256, rem, dig);
+        __syncthreads();
+        const int d = dig[0];
+        const uint32_t ab = (uint32_t)dig[1], inbin = (uint32_t)dig[2];
+        __syncthreads();
+        if (d < 0) {
             set_status(a.status, CSA2_DEV_BAD_COUNT);  // counts disagree: take everything
             return 0ull;
         }
-        const uint32_t inbin = hist256[d];
-        __syncthreads();
         rem -= ab;
         prefix = (prefix << nb) | (uint64_t)d;
         shift -= nb;
@@ -208,7 +316,7 @@ __device__ uint64_t refine_threshold(const TopkDev& a, int r, const CandSource& 
     return prefix << shift;
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkDev a) {
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ uint32_t red[40];
     __shared__ uint32_t hist256[256];
@@ -231,75 +339,82 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
     const bool many = find_digit(a.hist + (int64_t)r * kBinsT, kBinsT, (uint32_t)K, d0, above, red);
 
     // ---- 1. classify this CTA's chunk and append winners / candidates -------------------
+    // All of the chunk's scores are loaded first; they are then classified and appended in
+    // batches of 8 per thread (one pair of list atomics per batch), which keeps the register
+    // count low enough for several CTAs per SM.
     if (start < end) {
         const unsigned lt = (1u << lane) - 1u;
         constexpr int kPer = kCollectChunk / kThreads;
-        uint64_t comp[kPer];
-        uint32_t valid = 0;
-        if (a.scores && !a.ids) {
-            float sv[kPer];
+        constexpr int kB = 8;
+        const bool plain = a.scores && !a.ids;
+        float sv[kPer];
+        if (plain) {
             const float* row = a.scores + (int64_t)r * a.ld;
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const int64_t i = start + (int64_t)k * kThreads + tid;
                 sv[k] = (i < end) ? ld_dep(row + i) : 0.f;
             }
+        }
 #pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                const int64_t i = start + (int64_t)k * kThreads + tid;
-                comp[k] = ((uint64_t)score_key(sv[k]) << 32) | (uint64_t)(~(uint32_t)i);
-                if (i < end) valid |= 1u << k;
-            }
-        } else {
+        for (int b0 = 0; b0 < kPer; b0 += kB) {
+            uint64_t comp[kB];
+            uint32_t valid = 0;
 #pragma unroll
-            for (int k = 0; k < kPer; ++k) {
-                const int64_t i = start + (int64_t)k * kThreads + tid;
+            for (int k = 0; k < kB; ++k) {
+                const int64_t i = start + (int64_t)(b0 + k) * kThreads + tid;
                 comp[k] = 0;
-                if (i < end && load_elem(a, r, i, comp[k])) valid |= 1u << k;
+                if (plain) {
+                    comp[k] = ((uint64_t)score_key(sv[b0 + k]) << 32) | (uint64_t)(~(uint32_t)i);
+                    if (i < end) valid |= 1u << k;
+                } else if (i < end && load_elem(a, r, i, comp[k])) {
+                    valid |= 1u << k;
+                }
             }
-        }
-        uint32_t mw[kPer], mc[kPer];
-        uint32_t cw = 0, cc = 0;
+            uint32_t mw[kB], mc[kB];
+            uint32_t cw = 0, cc = 0;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const bool ok = (valid >> k) & 1u;
-            const int dig = (int)(comp[k] >> 52);
-            mw[k] = __ballot_sync(0xffffffffu, ok && (!many || dig > d0));
-            mc[k] = __ballot_sync(0xffffffffu, ok && many && dig == d0);
-            cw += __popc(mw[k]);
-            cc += __popc(mc[k]);
-        }
-        if (lane == 0) {
-            wsum[0][wid] = cw;
-            wsum[1][wid] = cc;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            uint32_t tw = 0, tc = 0;
-            for (int w = 0; w < kThreads / 32; ++w) {
-                const uint32_t a0 = wsum[0][w], a1 = wsum[1][w];
-                wsum[0][w] = tw;
-                wsum[1][w] = tc;
-                tw += a0;
-                tc += a1;
+            for (int k = 0; k < kB; ++k) {
+                const bool ok = (valid >> k) & 1u;
+                const int dig = (int)(comp[k] >> 52);
+                mw[k] = __ballot_sync(0xffffffffu, ok && (!many || dig > d0));
+                mc[k] = __ballot_sync(0xffffffffu, ok && many && dig == d0);
+                cw += __popc(mw[k]);
+                cc += __popc(mc[k]);
             }
-            wbase[0] = tw ? atomicAdd(cnt + 0, tw) : 0u;
-            wbase[1] = tc ? atomicAdd(cnt + 1, tc) : 0u;
-        }
-        __syncthreads();
-        uint32_t pw = wbase[0] + wsum[0][wid], pc = wbase[1] + wsum[1][wid];
+            if (lane == 0) {
+                wsum[0][wid] = cw;
+                wsum[1][wid] = cc;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t tw = 0, tc = 0;
+                for (int w = 0; w < kThreads / 32; ++w) {
+                    const uint32_t a0 = wsum[0][w], a1 = wsum[1][w];
+                    wsum[0][w] = tw;
+                    wsum[1][w] = tc;
+                    tw += a0;
+                    tc += a1;
+                }
+                wbase[0] = tw ? atomicAdd(cnt + 0, tw) : 0u;
+                wbase[1] = tc ? atomicAdd(cnt + 1, tc) : 0u;
+            }
+            __syncthreads();
+            uint32_t pw = wbase[0] + wsum[0][wid], pc = wbase[1] + wsum[1][wid];
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            if ((mw[k] >> lane) & 1u) {
-                const uint32_t pos = pw + __popc(mw[k] & lt);
-                if (pos < (uint32_t)K) a.winners[(int64_t)r * K + pos] = comp[k];
+            for (int k = 0; k < kB; ++k) {
+                if ((mw[k] >> lane) & 1u) {
+                    const uint32_t pos = pw + __popc(mw[k] & lt);
+                    if (pos < (uint32_t)K) a.winners[(int64_t)r * K + pos] = comp[k];
+                }
+                if ((mc[k] >> lane) & 1u) {
+                    const uint32_t pos = pc + __popc(mc[k] & lt);
+                    if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp[k];
+                }
+                pw += __popc(mw[k]);
+                pc += __popc(mc[k]);
             }
-            if ((mc[k] >> lane) & 1u) {
-                const uint32_t pos = pc + __popc(mc[k] & lt);
-                if (pos < (uint32_t)a.ccap) a.cands[(int64_t)r * a.ccap + pos] = comp[k];
-            }
-            pw += __popc(mw[k]);
-            pc += __popc(mc[k]);
+            __syncthreads();   // wsum and wbase are rewritten by the next batch
         }
     }
 
@@ -361,72 +476,43 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const TopkDev a) {
     __syncthreads();
 
     // ---- 3. emit the picks in ascending order ---------------------------------------------
-    int npick;
-    uint32_t off = 0;
-    int w0 = 0, w1 = 0;
-    if (use_bm) {
-        const int per = (nwords + kThreads - 1) / kThreads;
-        w0 = tid * per;
-        w1 = min(nwords, w0 + per);
-        uint32_t cntb = 0;
-        for (int wi = w0; wi < w1; ++wi) cntb += __popc(bm[wi]);
-        uint32_t incl = cntb;
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
-        }
-        if (lane == 31) red[wid] = incl;
-        __syncthreads();
-        if (tid == 0) {
-            uint32_t acc = 0;
-            for (int w = 0; w < kThreads / 32; ++w) {
-                const uint32_t t = red[w];
-                red[w] = acc;
-                acc += t;
-            }
-            npick_s = acc;
-        }
-        __syncthreads();
-        off = red[wid] + incl - cntb;
-        npick = (int)min(npick_s, (uint32_t)K);
-    } else {
-        // rank each pick among the (distinct) picks
-        npick = (int)min(npick_s, (uint32_t)K);
-        int32_t* sorted = reinterpret_cast<int32_t*>(cand_s);
-        for (int i = tid; i < npick; i += kThreads) {
-            const int32_t v = picks[i];
-            int rank = 0;
-            for (int j = 0; j < npick; ++j) rank += (picks[j] < v) | ((picks[j] == v) & (j < i));
-            sorted[rank] = v;
-        }
-        __syncthreads();
-        picks = sorted;
-    }
     const int32_t lim = a.expand8 ? ld_dep(a.expand_limit + r) : 0;
     int32_t* o = a.out + (int64_t)r * K * (a.expand8 ? 8 : 1);
-    auto emit = [&](uint32_t slot, int64_t id) {
-        if (slot >= (uint32_t)K) return;
+    if (use_bm) {
+        emit_bitmap<kThreads>(bm, nwords, K, o, a.expand8, lim, red);
+        return;
+    }
+    // bitonic sort of the (distinct) picks, padded to a power of two (at most kMaxK)
+    const int npick = (int)min(npick_s, (uint32_t)K);
+    int p2 = 1;
+    while (p2 < npick) p2 <<= 1;
+    for (int i = npick + tid; i < p2; i += kThreads) picks[i] = INT32_MAX;
+    __syncthreads();
+    for (int k = 2; k <= p2; k <<= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < p2; i += kThreads) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int32_t x = picks[i], y = picks[l];
+                    if ((x > y) == ((i & k) == 0)) {
+                        picks[i] = y;
+                        picks[l] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    for (int i = tid; i < npick; i += kThreads) {
+        const int32_t id = picks[i];
         if (!a.expand8) {
-            o[slot] = (int32_t)id;
+            o[i] = id;
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int64_t pos = id * 8 + e;
-                o[slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
+                const int64_t pos = (int64_t)id * 8 + e;
+                o[(int64_t)i * 8 + e] = pos < lim ? (int32_t)pos : -1;
             }
         }
-    };
-    if (use_bm) {
-        for (int wi = w0; wi < w1; ++wi) {
-            uint32_t m = bm[wi];
-            while (m) {
-                const int b = __ffs(m) - 1;
-                m &= m - 1;
-                emit(off++, (int64_t)wi * 32 + b);
-            }
-        }
-    } else {
-        for (int i = tid; i < npick; i += kThreads) emit((uint32_t)i, picks[i]);
     }
     const int mult = a.expand8 ? 8 : 1;
     for (int i = npick * mult + tid; i < K * mult; i += kThreads) o[i] = -1;
@@ -475,44 +561,6 @@ __device__ __forceinline__ uint32_t row_excl_scan(uint32_t v, uint32_t* wsum, ui
     total = wsum[32];
     __syncthreads();
     return r;
-}
-
-// Warp 0 only: over bins h[0..256) (counts), find d with above(d) < rem <= above(d) + h[d],
-// above(d) = sum of h[e] for e > d. Writes d (or -1 when the total is < rem), above(d) and
-// h[d] into out[0..3).
-__device__ __forceinline__ void warp_find_digit256(const uint32_t* h, uint32_t rem, int* out) {
-    const int lane = threadIdx.x & 31;
-    uint32_t b[8], sum = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {   // lane 0 owns the 8 highest bins, highest first
-        b[j] = h[255 - 8 * lane - j];
-        sum += b[j];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-    }
-    const uint32_t excl = incl - sum;
-    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-    if (lane == 0 && total < rem) {
-        out[0] = -1;
-        out[1] = (int)total;
-        out[2] = 0;
-    }
-    if (excl < rem && incl >= rem) {
-        uint32_t acc = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (acc < rem && acc + b[j] >= rem) {
-                out[0] = 255 - 8 * lane - j;
-                out[1] = (int)acc;
-                out[2] = (int)b[j];
-            }
-            acc += b[j];
-        }
-    }
 }
 
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
@@ -614,73 +662,6 @@ __device__ __forceinline__ void row_threshold(const RowState& S, const uint32_t 
     d0 = many ? S.dig_s[0] : -1;
     above = many ? (uint32_t)S.dig_s[1] : total;
     __syncthreads();
-}
-
-// Emits the set bits of bm[0, nwords) in ascending order into output slots [0, K): the bit's
-// index, or the 8 positions of that block (positions >= lim as -1) with expand8; pads the
-// remaining slots with -1. Groups of 32 words are read by whole warps, one word per lane
-// (conflict-free), and each warp owns a contiguous run of groups; a warp-level prefix sum
-// gives every word its first slot. Block-wide (contains barriers); wsum takes 33 words.
-template <int NT>
-__device__ void emit_bitmap(const uint32_t* bm, int64_t nwords, int K, int32_t* o, bool expand8,
-                            int32_t lim, uint32_t* wsum) {
-    constexpr int NW = NT / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t ngroups = (nwords + 31) >> 5;
-    const int64_t gpw = (ngroups + NW - 1) / NW;
-    const int64_t g0 = warp * gpw, g1 = g0 + gpw < ngroups ? g0 + gpw : ngroups;
-    auto word = [&](int64_t g) { const int64_t wi = g * 32 + lane; return wi < nwords ? bm[wi] : 0u; };
-    uint32_t wtot = 0;
-    for (int64_t g = g0; g < g1; ++g) wtot += __reduce_add_sync(0xffffffffu, (uint32_t)__popc(word(g)));
-    if (lane == 0) wsum[warp] = wtot;
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t x = lane < NW ? wsum[lane] : 0u;
-        uint32_t xi = x;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t u = __shfl_up_sync(0xffffffffu, xi, d);
-            if (lane >= d) xi += u;
-        }
-        if (lane < NW) wsum[lane] = xi - x;
-        if (lane == 31) wsum[32] = xi;
-    }
-    __syncthreads();
-    uint32_t base = wsum[warp];
-    const uint32_t total = wsum[32];
-    for (int64_t g = g0; g < g1 && base < (uint32_t)K; ++g) {
-        uint32_t w = word(g);
-        const uint32_t pc = (uint32_t)__popc(w);
-        uint32_t incl = pc;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t u = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += u;
-        }
-        uint32_t slot = base + incl - pc;
-        const int64_t wbase = (g * 32 + lane) * 32;
-        while (w) {
-            const int bit = __ffs(w) - 1;
-            w &= w - 1;
-            if (slot < (uint32_t)K) {
-                const int64_t id = wbase + bit;
-                if (!expand8) {
-                    o[slot] = (int32_t)id;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int64_t pos = id * 8 + e;
-                        o[(int64_t)slot * 8 + e] = pos < lim ? (int32_t)pos : -1;
-                    }
-                }
-            }
-            ++slot;
-        }
-        base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    const int npick = (int)(total < (uint32_t)K ? total : (uint32_t)K);
-    const int mult = expand8 ? 8 : 1;
-    for (int i = npick * mult + (int)threadIdx.x; i < K * mult; i += NT) o[i] = -1;
 }
 
 // Refinement, picks and the ordered output of one gathered row, after every element was
