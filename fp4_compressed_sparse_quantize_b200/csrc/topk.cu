@@ -1045,7 +1045,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
         const int cnt = (int)(b1 - e0 < CE ? b1 - e0 : CE);
         const uint32_t* cb_ = buf + (size_t)slot * CE;
         uint32_t key[kBmPer];
-        uint32_t ncw = 0;
+        uint32_t nc_t = 0;   // this thread's candidates in the chunk
 #pragma unroll
         for (int j = 0; j < kBmPer; ++j) {
             const int i = j * NT + tid;
@@ -1055,8 +1055,9 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_bitmap_kernel(const TopkDe
                 set_bit(e0 + i);
                 ++nwin_t;
             }
-            ncw += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < cnt && many && dig == d0));
+            nc_t += (i < cnt && many && dig == d0) ? 1u : 0u;
         }
+        const uint32_t ncw = __reduce_add_sync(0xffffffffu, nc_t);
         __syncthreads();   // every thread has read the slot: refill it
         if (tid == 0 && ok && c + ring < nch) issue(c + ring);
         if (ncw) {
