@@ -20,7 +20,7 @@
 //                       marked in a bitmap of positions (see the kernel);
 //   topk_gather_kernel  rows of gathered ids (Reindex over the pool): one 1024-thread CTA
 //                       per row, winner and candidate lists in shared memory, picks ordered
-//                       through a bitmap of ids;
+//                       by a bitonic sort;
 //   topk_kernel         longer rows (the 1M-entry Full layer), grid = chunks x rows: every
 //                       CTA classifies its chunk into per-row lists (one atomic per list per
 //                       CTA); the last CTA of a row to finish (threadfence + counter, no
@@ -532,7 +532,7 @@ constexpr int64_t kRowMaxN = 262144;
 constexpr size_t kRowOffHist = 0;                                   // u32[4096]
 constexpr size_t kRowOffCand = kRowOffHist + 4 * kBinsT;            // u64[kRowCands]
 constexpr size_t kRowOffWin = kRowOffCand + 8 * kRowCands;          // u32[kMaxK]
-constexpr size_t kRowOffBm = kRowOffWin + 4 * kMaxK;                // bitmap or pick list
+constexpr size_t kRowOffBm = kRowOffWin + 4 * kMaxK;                // pick list
 
 // Exclusive prefix sum of v over the 1024 threads (thread order); `total` gets the sum.
 // Uses wsum[0..32); ends with a barrier, so wsum may be reused right away.
@@ -582,7 +582,7 @@ struct RowState {
     uint32_t* hist;     // 4096 bins (the histogram, later 256-bin refinement counts)
     uint64_t* cand_s;   // candidates (composites), first kRowCands
     uint32_t* win_s;    // winner ids
-    uint32_t* bm;       // bitmap of picked ids, or the pick list
+    uint32_t* bm;       // the pick list (ids)
     uint32_t* wsum;
     int* dig_s;
     uint32_t* tot_s;    // running winner / candidate counts
@@ -670,8 +670,6 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
                              uint32_t id_lim, bool many, int d0, uint32_t above, int ccap) {
     const int tid = threadIdx.x;
     const int K = a.K;
-    const bool use_bm = a.bitmap_words > 0;
-    const int nwords = a.bitmap_words;
     const uint32_t nwin_all = S.tot_s[0], ncand = S.tot_s[1];
     const uint32_t nwin = min(nwin_all, (uint32_t)K);
     if (tid == 0 && (nwin_all > (uint32_t)K || (many && nwin_all != above)))
@@ -730,24 +728,14 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
             uint64_t c;
             if (cand(i, c) && c >= T) {
                 const uint32_t id = ~(uint32_t)(c & 0xFFFFFFFFu);
-                if (use_bm) {
-                    if ((int)(id >> 5) < nwords) atomicOr(&S.bm[id >> 5], 1u << (id & 31));
-                } else {
-                    const uint32_t pos = atomicAdd(&S.tot_s[0], 1u);
-                    if (pos < (uint32_t)K) S.bm[pos] = id;
-                }
+                const uint32_t pos = atomicAdd(&S.tot_s[0], 1u);
+                if (pos < (uint32_t)K) S.bm[pos] = id;
             }
         }
     }
     // winners
-    for (uint32_t i = tid; i < nwin; i += kRowThreads) {
-        const uint32_t id = S.win_s[i];
-        if (use_bm) {
-            if ((int)(id >> 5) < nwords) atomicOr(&S.bm[id >> 5], 1u << (id & 31));
-        } else {
-            S.bm[i] = id;   // slots [0, nwin) of the pick list; candidates were appended after
-        }
-    }
+    for (uint32_t i = tid; i < nwin; i += kRowThreads)
+        S.bm[i] = S.win_s[i];   // slots [0, nwin) of the pick list; candidates were appended after
     __syncthreads();
 
     // ---- emit in ascending id order ----------------------------------------------------------
@@ -765,24 +753,28 @@ __device__ void row_finalize(const TopkDev& a, const RowState& S, int r, int64_t
             }
         }
     };
-    if (use_bm) {
-        emit_bitmap<kRowThreads>(S.bm, nwords, K, o, a.expand8, lim, S.wsum);
-        return;
-    }
-    int npick;
-    {
-        // winners occupy [0, nwin), candidates were appended from tot_s[0] = nwin_all on
-        npick = (int)min(many ? S.tot_s[0] : nwin, (uint32_t)K);
-        for (int i = tid; i < npick; i += kRowThreads) {
-            const uint32_t v = S.bm[i];
-            int rank = 0;
-            for (int j = 0; j < npick; ++j) {
-                const uint32_t u = S.bm[j];
-                rank += (u < v) | ((u == v) & (j < i));
+    // winners occupy [0, nwin), candidates were appended from tot_s[0] = nwin_all on: a
+    // bitonic sort of the (distinct) picks, padded to a power of two (at most kMaxK)
+    const int npick = (int)min(many ? S.tot_s[0] : nwin, (uint32_t)K);
+    int p2 = 1;
+    while (p2 < npick) p2 <<= 1;
+    for (int i = npick + tid; i < p2; i += kRowThreads) S.bm[i] = 0xFFFFFFFFu;
+    __syncthreads();
+    for (int k = 2; k <= p2; k <<= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < p2; i += kRowThreads) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const uint32_t x = S.bm[i], y = S.bm[l];
+                    if ((x > y) == ((i & k) == 0)) {
+                        S.bm[i] = y;
+                        S.bm[l] = x;
+                    }
+                }
             }
-            emit((uint32_t)rank, v);
+            __syncthreads();
         }
-    }
+    for (int i = tid; i < npick; i += kRowThreads) emit((uint32_t)i, S.bm[i]);
     const int mult = a.expand8 ? 8 : 1;
     for (int i = npick * mult + tid; i < K * mult; i += kRowThreads) o[i] = -1;
 }
@@ -810,8 +802,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_gather_kernel(const TopkD
     const int64_t n = row_len(a, r);
     const int K = a.K;
     const uint32_t id_lim = (uint32_t)max(0, ld_dep(a.id_limit + r));
-    const bool use_bm = a.bitmap_words > 0;
-    const int nwords = a.bitmap_words;
     if (tid == 0) {
         tot_s[0] = tot_s[1] = 0u;
         dig_s[0] = -1;
@@ -833,8 +823,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_gather_kernel(const TopkD
     };
     load(0);
     const uint4 h4 = reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kBinsT)[kRowThreads - 1 - tid];
-    if (use_bm)
-        for (int i = tid; i < nwords; i += kRowThreads) S.bm[i] = 0u;
     const uint32_t b4[4] = {h4.w, h4.z, h4.y, h4.x};
     row_threshold(S, b4, K, many, d0, above);
     for (int64_t base = 0; base < n; base += BATCH) {
@@ -1268,11 +1256,9 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
         return launch_bitmap<512, 1>(a, l.max_n, l.R, st);
     }
     if (l.ids && l.max_n <= kRowMaxN) {
-        // the bitmap of ids may cover up to 2^20 ids
-        a.bitmap_words = (l.id_bound > 0 && words * 4 <= 128 * 1024) ? (int)words : 0;
-        const size_t rsmem = kRowOffBm + (a.bitmap_words > 0 ? (size_t)a.bitmap_words * 4
-                                                              : (size_t)kMaxK * 4);
-        if (rsmem > 227 * 1024) return cudaErrorInvalidValue;
+        // the picks (at most K) are ordered by a bitonic sort: a bitmap over every possible
+        // id would be mostly empty, and zeroing and scanning it cost more than the sort
+        const size_t rsmem = kRowOffBm + (size_t)kMaxK * 4;
         e = cudaFuncSetAttribute(topk_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)rsmem);
         if (e != cudaSuccess) return e;
