@@ -631,8 +631,11 @@ size_t attention_stage_bytes(int Q, int rows) {
            (size_t)Q * rows * 4 + 4 * 256;
 }
 
-// Whether the decode splits of every query can run as clusters in one wave (the merge then
-// happens in distributed shared memory). Looked up once per (splits, shared memory) shape.
+// Whether the decode splits of a query can run as one thread-block cluster (the merge then
+// happens in distributed shared memory, with no partials in global memory and no merge
+// kernel). More queries than the clusters resident at once simply take several waves: at
+// 64 queries (two waves) this is 1% faster per step than partials plus the merge kernel.
+// Looked up once per (splits, shared memory) shape.
 static bool cluster_merge_fits(int Q, int nsplit, int dsmem) {
     if (nsplit < 2 || nsplit > 8) return false;
     static std::mutex mu;
@@ -661,7 +664,7 @@ static bool cluster_merge_fits(int Q, int nsplit, int dsmem) {
         cudaGetLastError();   // a refused query leaves no sticky error
         it = cache.emplace(key, n).first;
     }
-    return it->second >= Q;
+    return Q >= 1 && it->second >= 1;
 }
 
 int attention_decode_launches(int Q, int K, int W) {
