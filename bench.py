@@ -45,6 +45,9 @@ SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csr
 # DRAM traffic of one indexer-scan launch, from `ncu --metrics dram__bytes_read.sum,
 # dram__bytes_write.sum` (summary in profiles/), valid only for the indexer.cu it was taken
 # on: {workload: (sha1 of indexer.cu, bytes per launch)}.
+# device buffer sets of the end-to-end pipeline (step inputs and outputs)
+E2E_SETS = 3
+
 SCAN_TRAFFIC = {
     "decode_full_b32_ctx64k_r2": ("d4aec0c726679d57f6541074179e0477938198ac",
                                   134705152 + 3618048),
@@ -884,9 +887,9 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), pg, dev)
 
     # end-to-end: host inputs -> device -> step -> host output, through the public API.
-    # Steps are pipelined as a serving loop would run them: two sets of device inputs and
-    # outputs, so that the host->device copy of step k+1 and the device->host copy of step
-    # k-1 (copy streams) overlap step k (compute stream). Every step copies all of its
+    # Steps are pipelined as a serving loop would run them: E2E_SETS sets of device inputs
+    # and outputs, so that the host->device copies of the next steps and the device->host
+    # copies of the previous ones (copy streams) overlap step k (compute stream). Every step copies all of its
     # inputs in and its outputs back. L2 is not flushed inside this continuous region: each
     # step streams the 134 MB indexer-key cache (evict-first), more than the 126 MB L2.
     # Every step's inputs travel in one host->device copy and its outputs in one
@@ -901,7 +904,7 @@ def main():
     h_outbuf, _ = packed_like(outs0, "cpu")
     bi, bo = h_inbuf.numel(), h_outbuf.numel()
     io = []
-    for _ in range(2):
+    for _ in range(E2E_SETS):
         d_inbuf, d_in = packed_like(ins0, dev)
         d_outbuf, d_out = packed_like(outs0, dev)
         for d, x in zip(d_in, ins0):
@@ -920,20 +923,20 @@ def main():
             g_io.append(g)
         torch.cuda.synchronize()
     ev = lambda: torch.cuda.Event(enable_timing=False)
-    loaded, consumed, drained = [[ev(), ev()] for _ in range(3)]
+    loaded, consumed, drained = [[ev() for _ in range(E2E_SETS)] for _ in range(3)]
 
     def pipelined(n):
         for k in range(n):
-            s_ = k & 1
+            s_ = k % E2E_SETS
             inbuf, ins, outbuf, outs = io[s_]
             with torch.cuda.stream(h2d):
-                if k >= 2:
-                    h2d.wait_event(consumed[s_])      # step k-2 no longer reads set s_
+                if k >= E2E_SETS:
+                    h2d.wait_event(consumed[s_])      # the last step on set s_ no longer reads it
                 inbuf.copy_(h_inbuf, non_blocking=True)
                 loaded[s_].record(h2d)
             stream.wait_event(loaded[s_])
-            if k >= 2:
-                stream.wait_event(drained[s_])        # step k-2's outputs are on the host
+            if k >= E2E_SETS:
+                stream.wait_event(drained[s_])        # that step's outputs are on the host
             if g_io:
                 with torch.cuda.stream(stream):
                     g_io[s_].replay()
@@ -946,7 +949,7 @@ def main():
                 h_outbuf.copy_(outbuf, non_blocking=True)
                 drained[s_].record(d2h)
 
-    pipelined(2)                                      # warm the copy streams
+    pipelined(E2E_SETS)                               # warm the copy streams
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -1012,7 +1015,7 @@ def main():
             "e2e": {"value": queries / (e2e_ms / 1e3), "unit": "queries/s",
                     "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                     "schedule": "pipelined: step k+1's inputs in and step k-1's outputs out "
-                                "on copy streams while step k runs (two device buffer sets); "
+                                "on copy streams while step k runs (three device buffer sets); "
                                 "one packed copy each way per step"},
             "gpu_launches": state.launches_per_step() * args.steps,
             "clocks": clk,
