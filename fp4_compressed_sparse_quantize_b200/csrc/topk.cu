@@ -1246,9 +1246,12 @@ cudaError_t launch_topk(const TopkLaunch& l, cudaStream_t st) {
     cudaError_t e;
     if (!l.ids && l.max_n <= kBmMaxN) {
         // Few rows: a cluster per row spreads the reading over more SMs, within one wave:
-        // 1024-thread CTAs (one per SM) while four per row fit, else 512-thread CTAs (two
-        // per SM), with at least 4,096 elements per CTA.
+        // eight 512-thread CTAs per row for rows of 64K elements or more (the pool's 131,072
+        // block maxima at 1M context: 22.6 us against 26.3 us with four 1024-thread CTAs),
+        // else 1024-thread CTAs (one per SM) while four per row fit, else 512-thread CTAs
+        // (two per SM), with at least 4,096 elements per CTA.
         const int sms = device_sm_count();
+        if (l.max_n >= 65536 && l.R * 8 <= sms) return launch_bitmap<512, 8>(a, l.max_n, l.R, st);
         if (l.max_n >= 4 * 8192 && l.R * 4 <= sms) return launch_bitmap<1024, 4>(a, l.max_n, l.R, st);
         if (l.max_n >= 8 * 4096 && l.R * 8 <= 2 * sms) return launch_bitmap<512, 8>(a, l.max_n, l.R, st);
         if (l.max_n >= 4 * 4096 && l.R * 4 <= 2 * sms) return launch_bitmap<512, 4>(a, l.max_n, l.R, st);
