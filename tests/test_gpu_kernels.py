@@ -300,7 +300,9 @@ def _attn_case(B, H, K, W, n, seed, valid=None):
 @pytest.mark.parametrize("B,H,K,W,n", [(1, 16, 64, 128, 4096), (3, 64, 512, 128, 3000),
                                        (2, 64, 100, 5, 300), (2, 40, 512, 0, 700),
                                        (1, 64, 0, 128, 10), (2, 8, 7, 1, 20),
-                                       (24, 32, 512, 128, 2000)])
+                                       (24, 32, 512, 128, 2000),
+                                       # more than 8 splits: partials and the merge kernel
+                                       (2, 64, 2048, 128, 4000)])
 def test_attention_decode(B, H, K, W, n):
     kv, codes, scales, idx, q, swa = _attn_case(B, H, K, W, n, seed=B * 100 + K + W)
     out = torch.empty((B, H, 512), dtype=torch.float32, device=dev)
