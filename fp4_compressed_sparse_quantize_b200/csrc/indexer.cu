@@ -301,15 +301,26 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                                              (int32_t)(row + hh * kTileRows), policy);
                 }
             } else {
-                // pool rows of query row r0 (G == 1 in gather mode)
+                // pool rows of query row r0 (G == 1 in gather mode). The tile's 128 pool
+                // positions are loaded first, four per lane, so that no copy waits for its
+                // own index load; the rows then go 4 per pass, 8 lanes per row.
+                static_assert(!GATHER || kRowsT == 128, "gathered tiles are 128 keys");
                 const int32_t* pl = p.pool + (int64_t)r0 * p.P + jt * kRowsT;
                 const int n_vis = ld_dep(p.n_row + r0);
                 const uint32_t dst_u = smem_u32(dst);
+                int pv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int64_t slot = jt * kRowsT + 32 * k + lane;
+                    const int v = (slot < p.P) ? ld_dep(pl + 32 * k + lane) : -1;
+                    pv[k] = v >= n_vis ? -1 : v;
+                }
+#pragma unroll 4
                 for (int rr = 0; rr < kRowsT; rr += 4) {
                     const int rl = rr + (lane >> 3);       // 4 rows per pass, 8 lanes per row
-                    const int64_t slot = jt * kRowsT + rl;
-                    int pos = (slot < p.P) ? ld_dep(pl + rl) : -1;
-                    if (pos >= n_vis) pos = -1;
+                    const int q = rr >> 5;                 // the same for every lane
+                    const int pq = q == 0 ? pv[0] : q == 1 ? pv[1] : q == 2 ? pv[2] : pv[3];
+                    const int pos = __shfl_sync(0xffffffffu, pq, rl & 31);
                     if (pos >= 0 && KF4) {
                         // compact key: 16 codes (8 bytes) per 16-byte slot, the layout the
                         // unpacking TMA load gives the contiguous tiles; the other half is 0
