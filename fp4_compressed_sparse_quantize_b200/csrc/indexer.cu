@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
         cur.init(p.prefix, ngroups, t0);
         int qg = -1, qcount = 0;
         int64_t it = 0;
+        int gather_prev = -1;   // gather mode: the stage whose copies are still in flight
         const uint64_t policy = l2_policy_evict_first();
         for (int64_t t = t0; t < t1; ++t, ++it) {
             if (*abort_flag) break;
@@ -339,12 +340,23 @@ __global__ void __launch_bounds__(32 * kEpiWarp0 + 128 * EPI, 1)
                         }
                     }
                 }
+                // two tiles in flight: the previous tile's copies are waited for (and made
+                // visible to the tensor core) only now that this tile's are issued
                 cp_async_commit();
-                cp_async_wait<0>();
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[s]);
+                if (gather_prev >= 0) {
+                    cp_async_wait<1>();
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[gather_prev]);
+                }
+                gather_prev = s;
             }
+        }
+        if (GATHER && gather_prev >= 0) {
+            cp_async_wait<0>();
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[gather_prev]);
         }
         // Drain: every TMA issued into this CTA's shared memory must land before exit.
         if (!GATHER && lane == 0) {
