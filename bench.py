@@ -49,8 +49,8 @@ SCAN_KERNEL_SRC = os.path.join(ROOT, "fp4_compressed_sparse_quantize_b200", "csr
 E2E_SETS = 3
 
 SCAN_TRAFFIC = {
-    "decode_full_b32_ctx64k_r2": ("d4aec0c726679d57f6541074179e0477938198ac",
-                                  134705152 + 3618048),
+    "decode_full_b32_ctx64k_r2": ("000c6d6bf38b6d6fecd39db36f22a85ceb28acdd",
+                                  134714368 + 3515904),
 }
 
 
