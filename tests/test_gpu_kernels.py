@@ -176,6 +176,21 @@ def test_topk_long_rows_odd_stride():
         check_topk(idx[b, 0], s, np.arange(n), K, f"b={b} n={n}")
 
 
+def test_topk_rows_beyond_the_bitmap_kernel():
+    """Rows longer than 262,144 entries go to the chunked kernel (every CTA classifies a
+    chunk, the last one of the row finishes it); at 300,001 entries its picks are emitted
+    through a bitmap of positions."""
+    g = _gen(78)
+    n, K = 300001, 512
+    k_I = _keys(1, n, torch.float8_e4m3fn, g, dup=True)
+    q_I = torch.randn((1, 1, 16, 128), generator=g).to(torch.float8_e4m3fn)
+    w = torch.rand((1, 1, 16), generator=g)
+    idx, scores, _, st = _full_decode(q_I, w, k_I, [n], K)
+    assert st == 0
+    s = O.index_scores(raw_qk(q_I[0, 0]), w[0, 0].numpy(), raw_qk(k_I[0]), O.E4M3)
+    check_topk(idx[0, 0], s, np.arange(n), K, "n=300001")
+
+
 def test_topk_degenerate_all_equal_scores():
     """w = 0: every score is +0, the K lowest positions must win (slow exact path)."""
     g = _gen(7)
