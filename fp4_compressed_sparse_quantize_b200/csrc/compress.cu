@@ -11,18 +11,21 @@
 //   codes, scales = FP4 quantize-on-write of x[j] (as csa2_quantize_kv)
 //   k[j][e] = sum_d W[e][d] * x[j][d], stored as E4M3 (RNE, saturating) or bf16.
 //
-// One CTA per 32 entries (the MMA's M is 128; rows 32.. are computed and discarded, the
-// projection being tiny next to the pooling's loads), 8 warps:
-//  1. pooling: warp w takes entries w, w+8, w+16, w+24; lane l owns channels [16l, 16l+16), i.e.
+// One CTA per E entries, E = 8, 16 or 32: the fewest that still fill the SMs (the MMA's M is
+// 128; rows E.. are computed and discarded, the projection being tiny next to the pooling's
+// loads), 8 warps:
+//  1. pooling: warp w takes entries w, w+8, ...; lane l owns channels [16l, 16l+16), i.e.
 //     one FP4 scale block. Per token the warp reads the 1 KiB latent and logit rows in one
-//     coalesced sweep (for up to 4 tokens, all of an entry's rows in one batch of loads);
-//     the softmax (max, then exp-weighted sums) runs in fp32 per channel.
+//     coalesced sweep (up to 4 tokens: all of an entry's rows in one batch of loads, issued
+//     before the entry's cache offset is known); the softmax (max, then exp-weighted sums)
+//     runs in fp32 per channel. (Two entries' rows per batch was slower after an L2 flush.)
 //     The bf16 latent goes to the global FP4 cache (codes + scale, this lane's block) and
 //     into shared memory as the MMA's A operand (K-major, 128-byte swizzle, 8 slabs of
 //     64 channels);
 //  2. projection: one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
-//     M = 128 entries, N = 64 key channels, K = 512, twice (W's two halves are TMA-loaded
-//     in turn into one 64 KiB buffer);
+//     M = 128 entries, N = 64 key channels, K = 512, twice. Both halves of W are TMA-loaded
+//     at the start: the first into rows 64-127 of the A operand's slabs, which hold no
+//     entry (the MMA reads them as discarded rows), the second into its own 64 KiB;
 //  3. epilogue: warp 0 reads TMEM lanes 0-31 (one entry per thread), converts and stores
 //     the 128-channel key row.
 #include "csa2_common.cuh"
@@ -33,14 +36,16 @@ namespace csa2 {
 namespace {
 
 constexpr int kM = 128;                    // MMA rows (A operand rows in shared memory)
-constexpr int kE = 32;                     // entries per CTA (rows kE.. of the MMA unused)
+constexpr int kMaxE = 32;                  // entries per CTA at most (rows E.. of the MMA unused)
 constexpr int kD = 512;                    // latent channels
 constexpr int kDi = 128;                   // indexer-key channels
 constexpr int kThreads = 256;
 constexpr int kESlab = kM * 128;           // 128 entries x 64 bf16 channels = 16 KiB
 constexpr int kWSlab = 64 * 128;           // 64 key channels x 64 bf16 channels = 8 KiB
 constexpr int kOffE = 0;                   // 8 slabs: 128 KiB
-constexpr int kOffW = 8 * kESlab;          // 8 slabs of one half of W: 64 KiB
+constexpr int kWInE = 64 * 128;            // W's first half: rows 64.. of each A slab (8 KiB)
+constexpr int kOffW = 8 * kESlab;          // 8 slabs of W's second half: 64 KiB
+static_assert(kMaxE <= 64, "W's first half shares the A slabs above the entries' rows");
 constexpr int kOffRow = kOffW + 8 * kWSlab;   // int64 per entry: cache row or -1
 constexpr int kOffBar = kOffRow + kM * 8;
 constexpr int kDynBytes = kOffBar + 64 + 1024;   // + alignment slack
@@ -57,6 +62,7 @@ struct CompressDev {
     float* key_scales;            // compact keys: fp32 scale per key [B][cap]
     int key_bf16;
     int key_fp4;
+    int epc;                      // entries per CTA (8, 16 or 32)
     int64_t cap;
     __nv_bfloat16* latent;        // [B * n_new][512] or null
     int32_t* status;
@@ -71,6 +77,46 @@ __device__ __forceinline__ void bf16x16_to_float(const uint4& a, const uint4& b,
     }
 }
 
+// Per channel, the softmax over the entry's nt <= NT tokens of the logits zr weighting the
+// latents cr (rows already in registers), rounded to bf16: the maximum first, then the
+// exp-weighted sums in token order.
+template <int NT>
+__device__ __forceinline__ void pool_rows(const uint4 (&zr)[NT][2], const uint4 (&cr)[NT][2],
+                                          int nt, float (&x)[16]) {
+    float zmax[16], den[16], num[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        zmax[k] = -INFINITY;
+        den[k] = num[k] = 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (t < nt) {
+            float z[16];
+            bf16x16_to_float(zr[t][0], zr[t][1], z);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        if (t < nt) {
+            float z[16], c[16];
+            bf16x16_to_float(zr[t][0], zr[t][1], z);
+            bf16x16_to_float(cr[t][0], cr[t][1], c);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float e = expf(z[k] - zmax[k]);
+                den[k] += e;
+                num[k] = fmaf(e, c[k], num[k]);
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+        x[k] = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(num[k], den[k])));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     compress_kv_kernel(const __grid_constant__ CUtensorMap tmap_w, const CompressDev a) {
     extern __shared__ uint8_t dsm_raw[];
@@ -78,8 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~(uintptr_t)1023);
     int64_t* row_dst = reinterpret_cast<int64_t*>(sm + kOffRow);
     uint64_t* wfull = reinterpret_cast<uint64_t*>(sm + kOffBar);
-    uint64_t* mdone0 = wfull + 1;
-    uint64_t* mdone1 = wfull + 2;
+    uint64_t* mdone = wfull + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wfull + 3);
     volatile int* stuck = reinterpret_cast<volatile int*>(wfull + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -88,8 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_launch();
     if (threadIdx.x == 0) {
         mbar_init(wfull, 1);
-        mbar_init(mdone0, 1);
-        mbar_init(mdone1, 1);
+        mbar_init(mdone, 1);
         *stuck = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
@@ -101,102 +145,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_holder;
     grid_dep_wait();   // C, Z, W and the offsets come from earlier work on the stream
 
-    if (threadIdx.x == 0) {   // first half of W: key channels 0..63
-        mbar_arrive_expect_tx(wfull, 8 * kWSlab);
-        for (int s = 0; s < 8; ++s) tma_load_2d(sm + kOffW + s * kWSlab, &tmap_w, wfull, 64 * s, 0);
+    if (threadIdx.x == 0) {   // W: key channels 0..63 into the A slabs, 64..127 apart
+        mbar_arrive_expect_tx(wfull, 16 * kWSlab);
+        for (int s = 0; s < 8; ++s) {
+            tma_load_2d(sm + kOffE + s * kESlab + kWInE, &tmap_w, wfull, 64 * s, 0);
+            tma_load_2d(sm + kOffW + s * kWSlab, &tmap_w, wfull, 64 * s, 64);
+        }
     }
 
     // ---- 1. pooling, FP4 write and the A operand ----------------------------------------
     const int64_t total = (int64_t)a.B * a.n_new;
-    if (threadIdx.x >= kE && threadIdx.x < kM) row_dst[threadIdx.x] = -1;
-    for (int m = warp; m < kE; m += kThreads / 32) {
-        const int64_t g = (int64_t)blockIdx.x * kE + m;
+    const int epc = a.epc;
+    if (threadIdx.x >= epc && threadIdx.x < kM) row_dst[threadIdx.x] = -1;
+    // entry m of this CTA: its sequence b, index j and cache offset (the offset is used only
+    // by the writes, so the entry's rows are requested without waiting for it)
+    auto locate = [&](int m, int& b, int& j, int64_t& dst) -> bool {
+        const int64_t g = (int64_t)blockIdx.x * epc + m;
+        b = 0;
+        j = 0;
+        dst = -1;
+        if (m >= epc || g >= total) return false;
+        b = (int)(g / a.n_new);
+        j = (int)(g - (int64_t)b * a.n_new);
+        dst = (int64_t)ld_dep(a.dst_off + b) + j;
+        return true;
+    };
+    // this lane's 16 channels of token t of entry (b, j): logits and latents
+    auto zrow = [&](int b, int j, int t) {
+        return reinterpret_cast<const uint4*>(a.Z + (int64_t)b * a.bstride +
+                                              ((int64_t)j * a.r + t) * a.ld + lane * 16);
+    };
+    auto crow_src = [&](int b, int j, int t) {
+        return reinterpret_cast<const uint4*>(a.C + (int64_t)b * a.bstride +
+                                              ((int64_t)j * a.r + t) * a.ld + lane * 16);
+    };
+    // the writes of entry m: its bf16 latent into the A operand (and the optional latent
+    // output), its FP4 codes and scale into the cache
+    auto finish = [&](int m, bool have, int b, int64_t dst, const float (&x)[16]) {
         int64_t crow = -1;
-        int b = 0, j = 0;
-        if (g < total) {
-            b = (int)(g / a.n_new);
-            j = (int)(g - (int64_t)b * a.n_new);
-            const int64_t dst = (int64_t)ld_dep(a.dst_off + b) + j;
+        if (have) {
             if (dst >= 0 && dst < a.cap)
                 crow = (int64_t)b * a.cap + dst;
             else if (lane == 0)
                 set_status(a.status, CSA2_DEV_BAD_INDEX);
-        }
-        float x[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) x[k] = 0.f;
-        if (crow >= 0) {
-            const int64_t tok0 = (int64_t)j * a.r;
-            const __nv_bfloat16* zc = a.Z + (int64_t)b * a.bstride + lane * 16;
-            const __nv_bfloat16* cc = a.C + (int64_t)b * a.bstride + lane * 16;
-            float zmax[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) zmax[k] = -INFINITY;
-            float den[16], num[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) den[k] = num[k] = 0.f;
-            if (a.r <= 4) {
-                // up to 4 tokens: every latent and logit row of the entry in one batch of loads
-                uint4 zr[4][2], cr[4][2];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    if (t < a.r) {
-                        const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
-                        const uint4* cp = reinterpret_cast<const uint4*>(cc + (tok0 + t) * a.ld);
-                        zr[t][0] = ld_dep(zp);
-                        zr[t][1] = ld_dep(zp + 1);
-                        cr[t][0] = ld_dep(cp);
-                        cr[t][1] = ld_dep(cp + 1);
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    if (t < a.r) {
-                        float z[16];
-                        bf16x16_to_float(zr[t][0], zr[t][1], z);
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    if (t < a.r) {
-                        float z[16], c[16];
-                        bf16x16_to_float(zr[t][0], zr[t][1], z);
-                        bf16x16_to_float(cr[t][0], cr[t][1], c);
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const float e = expf(z[k] - zmax[k]);
-                            den[k] += e;
-                            num[k] = fmaf(e, c[k], num[k]);
-                        }
-                    }
-                }
-            } else {
-                for (int t = 0; t < a.r; ++t) {
-                    const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
-                    float z[16];
-                    bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
-                }
-                for (int t = 0; t < a.r; ++t) {
-                    const uint4* zp = reinterpret_cast<const uint4*>(zc + (tok0 + t) * a.ld);
-                    const uint4* cp = reinterpret_cast<const uint4*>(cc + (tok0 + t) * a.ld);
-                    float z[16], c[16];
-                    bf16x16_to_float(ld_dep(zp), ld_dep(zp + 1), z);
-                    bf16x16_to_float(ld_dep(cp), ld_dep(cp + 1), c);
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float e = expf(z[k] - zmax[k]);
-                        den[k] += e;
-                        num[k] = fmaf(e, c[k], num[k]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                x[k] = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(num[k], den[k])));
         }
         // bf16 latent: 16 channels = two 16-byte chunks of row m in slab lane/4
         uint32_t pk[8];
@@ -219,11 +210,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             reinterpret_cast<uint2*>(a.codes + crow * CSA2_ENTRY_CODE_BYTES)[lane] = packed;
             a.scales[crow * CSA2_ENTRY_SCALE_BYTES + lane] = sc;
             if (a.latent) {
+                const int64_t g = (int64_t)blockIdx.x * epc + m;
                 uint4* lp = reinterpret_cast<uint4*>(a.latent + g * kD + lane * 16);
                 lp[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 lp[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
         }
+    };
+
+    for (int m = warp; m < epc; m += kThreads / 32) {
+        int b, j;
+        int64_t dst;
+        const bool have = locate(m, b, j, dst);
+        float x[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[k] = 0.f;
+        if (have && a.r <= 4) {
+            // up to 4 tokens: every latent and logit row of the entry in one batch of loads
+            uint4 zr[4][2], cr[4][2];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if (t < a.r) {
+                    zr[t][0] = ld_dep(zrow(b, j, t));
+                    zr[t][1] = ld_dep(zrow(b, j, t) + 1);
+                    cr[t][0] = ld_dep(crow_src(b, j, t));
+                    cr[t][1] = ld_dep(crow_src(b, j, t) + 1);
+                }
+            }
+            pool_rows<4>(zr, cr, a.r, x);
+        } else if (have) {
+            float zmax[16], den[16], num[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                zmax[k] = -INFINITY;
+                den[k] = num[k] = 0.f;
+            }
+            for (int t = 0; t < a.r; ++t) {
+                float z[16];
+                bf16x16_to_float(ld_dep(zrow(b, j, t)), ld_dep(zrow(b, j, t) + 1), z);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) zmax[k] = fmaxf(zmax[k], z[k]);
+            }
+            for (int t = 0; t < a.r; ++t) {
+                float z[16], c[16];
+                bf16x16_to_float(ld_dep(zrow(b, j, t)), ld_dep(zrow(b, j, t) + 1), z);
+                bf16x16_to_float(ld_dep(crow_src(b, j, t)), ld_dep(crow_src(b, j, t) + 1), c);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float e = expf(z[k] - zmax[k]);
+                    den[k] += e;
+                    num[k] = fmaf(e, c[k], num[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                x[k] = __bfloat162float(__float2bfloat16_rn(__fdiv_rn(num[k], den[k])));
+        }
+        finish(m, have, b, dst, x);
     }
     // the A operand was written by plain stores: make it visible to the tensor core
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -234,34 +277,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- 2. projection ------------------------------------------------------------------
     if (threadIdx.x == 0) {
         constexpr uint32_t idesc = make_idesc(128, 64, 1u, 1u);   // bf16 x bf16 -> fp32
-        bool ok = mbar_wait(wfull, 0, a.status);
-        for (int half = 0; half < 2 && ok; ++half) {
-            if (half == 1) {
-                // the first half's MMAs have read the W buffer: load the second half
-                ok = mbar_wait(mdone0, 0, a.status);
-                if (!ok) break;
-                mbar_arrive_expect_tx(wfull, 8 * kWSlab);
-                for (int s = 0; s < 8; ++s)
-                    tma_load_2d(sm + kOffW + s * kWSlab, &tmap_w, wfull, 64 * s, 64);
-                ok = mbar_wait(wfull, 1, a.status);
-                if (!ok) break;
-            }
+        const bool ok = mbar_wait(wfull, 0, a.status);
+        if (ok) {
             tc_fence_after();
-#pragma unroll 1
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint64_t ad = sw128_desc(sE + (kk >> 2) * kESlab + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = sw128_desc(sW + (kk >> 2) * kWSlab + (kk & 3) * 32, 16, 1024);
-                mma_f16(tmem + 64 * half, ad, bd, idesc, kk > 0);
+            // fully unrolled: each descriptor is a base plus a constant (the start-address
+            // field counts 16-byte units and no address reaches 256 KiB), so the issuing
+            // thread spends a few instructions per MMA
+            const uint64_t a0 = sw128_desc(sE, 16, 1024);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint64_t b0 = sw128_desc(half == 0 ? sE + kWInE : sW, 16, 1024);
+                const uint32_t wstride = half == 0 ? (uint32_t)kESlab : (uint32_t)kWSlab;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t ad = a0 + (uint64_t)(((kk >> 2) * kESlab + (kk & 3) * 32) >> 4);
+                    const uint64_t bd = b0 + (uint64_t)(((kk >> 2) * wstride + (kk & 3) * 32) >> 4);
+                    mma_f16(tmem + 64 * half, ad, bd, idesc, kk > 0);
+                }
             }
-            mma_commit(half == 0 ? mdone0 : mdone1);
+            mma_commit(mdone);
         }
         if (!ok) *stuck = 1;   // an MMA or a load may still be in flight
     }
     __syncwarp();
 
     // ---- 3. epilogue: one entry per thread of warps 0-3 ------------------------------------
-    if (warp < (kE + 31) / 32) {
-        bool ok = !*stuck && mbar_wait(mdone1, 0, a.status);
+    if (warp < (epc + 31) / 32) {
+        bool ok = !*stuck && mbar_wait(mdone, 0, a.status);
         ok = __all_sync(0xffffffffu, ok);   // tcgen05.ld below is warp-collective
         if (!ok) *stuck = 1;
         tc_fence_after();
@@ -391,7 +433,16 @@ cudaError_t launch_compress_kv(const CompressLaunch& l, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(compress_kv_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kDynBytes);
     if (e != cudaSuccess) return e;
-    const int64_t grid = (entries + kE - 1) / kE;
+    // the fewest entries per CTA (8, 16, 32) whose grid still fits on the SMs: few entries
+    // (a decode step) spread over several CTAs, each with one short chain of loads per warp
+    const int sms = device_sm_count();
+    a.epc = kMaxE;
+    for (int e8 = 8; e8 < kMaxE; e8 *= 2)
+        if ((entries + e8 - 1) / e8 <= sms) {
+            a.epc = e8;
+            break;
+        }
+    const int64_t grid = (entries + a.epc - 1) / a.epc;
     return launch_pdl(compress_kv_kernel, dim3((unsigned)grid), dim3(kThreads), (size_t)kDynBytes,
                       st, mw, a);
 }

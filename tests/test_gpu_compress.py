@@ -179,6 +179,19 @@ def test_compress_decode_shape_and_prefill_chunk():
     assert flips <= 1e-3 * total
 
 
+def test_compress_sixteen_entries_per_cta():
+    # 1,800 entries: the launch takes 16 entries per CTA (113 CTAs), between the decode
+    # shape's 8 and a long chunk's 32
+    B, n_new, r, cap = 2, 900, 2, 1000
+    dst = [0, 100]
+    Cs, Zs, W, codes, scales, keys, latent, st = _case(B, n_new, r, cap, dst, torch.float8_e4m3fn, 37)
+    assert st == 0
+    flips, total = _check(Cs, Zs, r, W, dst, cap, codes, scales, keys, latent,
+                          torch.float8_e4m3fn, n_new)
+    assert flips <= 1e-3 * total
+    assert int(codes[1, :100].sum()) == 0 and int(codes[0, 900:].sum()) == 0
+
+
 def test_compress_writes_compact_keys():
     """With compact 68-byte keys the compressor stores csa2_quantize_keys_fp4's encoding of
     the bf16-rounded projection. The same call with bf16 keys yields that projection exactly
