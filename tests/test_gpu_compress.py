@@ -179,6 +179,20 @@ def test_compress_decode_shape_and_prefill_chunk():
     assert flips <= 1e-3 * total
 
 
+def test_compress_ratio_above_four():
+    # more than four source tokens per entry: the per-token loop instead of the single batch
+    # of loads, on a ragged count with strided inputs
+    B, n_new, r, cap = 2, 45, 6, 64
+    dst = [3, 19]
+    Cs, Zs, W, codes, scales, keys, latent, st = _case(B, n_new, r, cap, dst, torch.float8_e4m3fn,
+                                                       38, ld_pad=32)
+    assert st == 0
+    flips, total = _check(Cs, Zs, r, W, dst, cap, codes, scales, keys, latent,
+                          torch.float8_e4m3fn, n_new)
+    assert flips <= 1e-3 * total
+    assert int(codes[0, :3].sum()) == 0 and int(codes[0, 48:].sum()) == 0
+
+
 def test_compress_sixteen_entries_per_cta():
     # 1,800 entries: the launch takes 16 entries per CTA (113 CTAs), between the decode
     # shape's 8 and a long chunk's 32
