@@ -294,6 +294,54 @@ def test_pool_and_reindex_decode():
         check_topk(idx2[b, 0], s2, ids, K, f"reindex b={b}")
 
 
+def test_pool_and_reindex_with_bf16_keys():
+    """The candidate pool and the Reindex gather with bf16 indexer keys (two 128-byte halves
+    per key row): block selection, the rescored pool and its Top-K against the oracle."""
+    g = _gen(79)
+    B, n, H_I, K, nblk = 2, 6000, 16, 64, 128
+    k_I = _keys(B, n, torch.bfloat16, g)
+    q_I = torch.randn((B, 1, H_I, 128), generator=g).to(torch.bfloat16)
+    w = torch.rand((B, 1, H_I), generator=g)
+    n_list = [n, n - 11]
+    idx, scores, pool, st = _full_decode(q_I, w, k_I, n_list, K, pool_blocks=nblk)
+    assert st == 0
+    for b in range(B):
+        s = O.index_scores(raw_qk(q_I[b, 0]), w[b, 0].numpy(), raw_qk(k_I[b, :n_list[b]]), O.BF16)
+        check_topk(idx[b, 0], s, np.arange(n_list[b]), K, f"full b={b}")
+        nb = (n_list[b] + 7) // 8
+        bmax = np.array([s[8 * c:8 * c + 8].max() for c in range(nb)])
+        got_blocks = np.unique(pool[b, 0][pool[b, 0] >= 0] // 8)
+        gb = np.full(nblk, -1)
+        gb[: len(got_blocks)] = got_blocks
+        check_topk(gb, bmax, np.arange(nb), nblk, f"pool b={b}")
+    q2 = torch.randn((B, 1, H_I, 128), generator=g).to(torch.bfloat16)
+    w2 = torch.rand((B, 1, H_I), generator=g)
+    pool_o = np.stack([O.pool(O.index_scores(raw_qk(q_I[b, 0]), w[b, 0].numpy(),
+                                             raw_qk(k_I[b, :n_list[b]]), O.BF16), nblk)
+                       for b in range(B)])[:, None, :]
+    P = pool_o.shape[-1]
+    idx2 = torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+    sc2 = torch.zeros((B, 1, P), dtype=torch.float32, device=dev)
+    ws = C().new_workspace(C().workspace_bytes(0, B, 1, H_I, P, K))
+    C().index_score_topk("reindex", q2.to(dev), w2.to(dev), k_I.to(dev), K, idx2, ws,
+                         n_vis0=torch.tensor(n_list, dtype=torch.int32, device=dev),
+                         pool_in=torch.from_numpy(pool_o.astype(np.int32)).to(dev),
+                         scores_out=sc2)
+    torch.cuda.synchronize()
+    assert C().read_device_status(ws) == 0
+    idx2 = idx2.cpu().numpy()
+    sc2 = sc2.cpu().numpy()
+    for b in range(B):
+        slots = np.nonzero(pool_o[b, 0] >= 0)[0]
+        ids = pool_o[b, 0][slots]
+        s2 = O.index_scores(raw_qk(q2[b, 0]), w2[b, 0].numpy(), raw_qk(k_I[b]), O.BF16, rows=ids)
+        qd = O.bf16_array_to_f64(raw_qk(q2[b, 0]).ravel()).reshape(H_I, 128)
+        kd = O.bf16_array_to_f64(raw_qk(k_I[b]).ravel()).reshape(n, 128)[ids]
+        mag = np.abs(kd) @ np.abs(qd).T @ w2[b, 0].numpy().astype(np.float64)
+        np.testing.assert_array_less(np.abs(sc2[b, 0, slots] - s2), 2e-6 * mag + 1e-6)
+        check_topk(idx2[b, 0], s2, ids, K, f"reindex b={b}")
+
+
 # ---- attention ----------------------------------------------------------------------------
 
 def _attn_case(B, H, K, W, n, seed, valid=None):
