@@ -249,6 +249,26 @@ def test_topk_many_ties_mixed():
     np.testing.assert_array_equal(idx[0, 0], expect)
 
 
+@pytest.mark.parametrize("H_I,K,n_list", [(128, 256, [5000, 300, 40000]), (32, 512, [9000, 513])])
+def test_full_decode_other_head_counts(H_I, K, n_list):
+    """FP8 scans with 32 and 128 indexer heads: 128 heads take a single 384-column
+    accumulator and one epilogue group, 32 heads a query operand of 32 columns."""
+    g = _gen(H_I + 5)
+    B, cap = len(n_list), max(n_list)
+    k_I = _keys(B, cap, torch.float8_e4m3fn, g, dup=True)
+    q_I = torch.randn((B, 1, H_I, 128), generator=g).to(torch.float8_e4m3fn)
+    w = torch.rand((B, 1, H_I), generator=g)
+    idx, scores, _, st = _full_decode(q_I, w, k_I, n_list, K)
+    assert st == 0
+    for b, n in enumerate(n_list):
+        s = O.index_scores(raw_qk(q_I[b, 0]), w[b, 0].numpy(), raw_qk(k_I[b, :n]), O.E4M3)
+        qd = O.e4m3_array_to_f64(raw_qk(q_I[b, 0]).ravel()).reshape(H_I, 128)
+        kd = O.e4m3_array_to_f64(raw_qk(k_I[b, :n]).ravel()).reshape(n, 128)
+        mag = np.abs(kd) @ np.abs(qd).T @ w[b, 0].numpy().astype(np.float64)
+        np.testing.assert_array_less(np.abs(scores[b, 0, :n] - s), 2e-6 * mag + 1e-6)
+        check_topk(idx[b, 0], s, np.arange(n), K, f"H_I={H_I} b={b} n={n}")
+
+
 def test_pool_and_reindex_decode():
     g = _gen(9)
     B, n, H_I, K, nblk = 2, 20000, 64, 512, 512
