@@ -517,6 +517,47 @@ def test_prefill_indexer_and_attention_small():
             check_attention(out[b, t].cpu().numpy(), refs[b, t], f"b={b} t={t}")
 
 
+def test_prefill_attention_padded_heads_ragged_chunks_and_rescale():
+    """24 query heads (padded to the kernel's 64), 200 selected entries with 10 empty slots
+    plus the 128-row window (three chunks of rows, the last one partial), and one window row
+    aligned with head 0 whose logit exceeds every earlier one by far: the running maximum of
+    that head rises in the last chunk and its accumulator columns are rescaled."""
+    g = _gen(80)
+    B, T, H, K, W, r = 1, 6, 24, 200, 128, 2
+    q_pos0 = [600]
+    cap = (q_pos0[0] + T) // r
+    kv = torch.randn((B, cap, 512), generator=g).to(torch.bfloat16)
+    codes = torch.zeros((B, cap, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, cap, 32), dtype=torch.uint8, device=dev)
+    C().quantize_kv(kv.to(dev), torch.zeros(B, dtype=torch.int32, device=dev), codes, scales)
+    q = torch.randn((B, T, H, 512), generator=g).to(torch.bfloat16)
+    q[:, :, 0] = q[:, :1, 0]                       # head 0: one vector for every token
+    swa = torch.randn((B, W - 1 + T, 512), generator=g).to(torch.float8_e4m3fn)
+    swa[0, 100] = (torch.sign(q[0, 0, 0].float()) * 8).to(torch.float8_e4m3fn)
+    rng = np.random.default_rng(80)
+    oidx = np.full((B, T, K), -1, np.int32)
+    for t in range(T):
+        n = O.prefill_visible(q_pos0[0] + t, r)
+        oidx[0, t, :K - 10] = np.sort(rng.choice(n, K - 10, replace=False))
+    out = torch.empty((B, T, H, 512), dtype=torch.float32, device=dev)
+    wsa = C().new_workspace(C().workspace_bytes(2, B, T, H, cap, K))
+    C().sparse_attn_prefill(q.to(dev), codes, scales, torch.from_numpy(oidx).to(dev), swa.to(dev),
+                            out, wsa, W, q_pos0=torch.tensor(q_pos0, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    assert C().read_device_status(wsa) == 0
+    out = out.cpu().numpy()
+    for t in range(T):
+        _, ref = O.prefill_query(None, None, None, None, bits16(kv[0]), bits16(q[0, t]),
+                                 bits8(swa[0]), q_pos0[0], t, r, K, W, 512 ** -0.5,
+                                 idx_override=oidx[0, t])
+        # each against its own scale: head 0's output is the planted row (magnitude 8)
+        check_attention(out[0, t, :1], ref[:1], f"t={t} head 0")
+        check_attention(out[0, t, 1:], ref[1:], f"t={t} heads 1..")
+        # head 0 is the planted window row, as the oracle says
+        row = O.e4m3_array_to_f64(bits8(swa[0, 100]))
+        assert np.max(np.abs(ref[0] - row)) <= 1e-6 * np.max(np.abs(row))
+
+
 def test_prefill_indexer_back_to_back_calls():
     """Consecutive prefill index calls in one process, each launched while the previous
     kernel may still run: one workspace reused with a different tile prefix (other query
