@@ -469,6 +469,32 @@ def test_attention_swa_valid_prefix():
         check_attention(out[b].cpu().numpy(), ref, f"b={b}")
 
 
+def test_attention_decode_one_split_dominates():
+    """A window row aligned with head 5's query: the last of the four splits holds a logit
+    far above every other split's, so the cluster merge weighs the others by ~2^-200."""
+    B, H, K, W, n = 2, 64, 512, 128, 3000
+    kv, codes, scales, idx, q, swa = _attn_case(B, H, K, W, n, seed=81)
+    for b in range(B):
+        swa[b, 120] = (torch.sign(q[b, 5].float()) * 8).to(torch.float8_e4m3fn)
+    out = torch.empty((B, H, 512), dtype=torch.float32, device=dev)
+    ws = C().new_workspace(C().workspace_bytes(1, B, 1, H, n, K))
+    tau = 1 / math.sqrt(512)
+    C().sparse_attn_decode("full", q.to(dev), codes, scales, torch.from_numpy(idx).to(dev),
+                           swa.to(dev), out, ws, scale=tau)
+    torch.cuda.synchronize()
+    assert C().read_device_status(ws) == 0
+    out = out.cpu().numpy()
+    for b in range(B):
+        rows = np.concatenate([oracle_main_rows(bits16(kv[b, idx[b]])),
+                               O.e4m3_array_to_f64(bits8(swa[b])).reshape(W, 512)])
+        ref = O.attention(O.bf16_array_to_f64(bits16(q[b])).reshape(H, 512), rows, tau)
+        others = [h for h in range(H) if h != 5]
+        check_attention(out[b, 5:6], ref[5:6], f"b={b} head 5")
+        check_attention(out[b, others], ref[others], f"b={b} other heads")
+        planted = O.e4m3_array_to_f64(bits8(swa[b, 120]))
+        assert np.max(np.abs(ref[5] - planted)) <= 1e-6 * np.max(np.abs(planted))
+
+
 # ---- prefill ---------------------------------------------------------------------------------
 
 def test_prefill_indexer_and_attention_small():
