@@ -13,12 +13,14 @@
 //
 // One CTA per E entries, E = 8, 16 or 32: the fewest that still fill the SMs (the MMA's M is
 // 128; rows E.. are computed and discarded, the projection being tiny next to the pooling's
-// loads), 8 warps:
-//  1. pooling: warp w takes entries w, w+8, ...; lane l owns channels [16l, 16l+16), i.e.
+// loads), 16 warps (128 registers a thread; each warp's entries are pooled one after the
+// other, so more warps mean shorter chains of dependent loads):
+//  1. pooling: warp w takes entries w, w+16, ...; lane l owns channels [16l, 16l+16), i.e.
 //     one FP4 scale block. Per token the warp reads the 1 KiB latent and logit rows in one
-//     coalesced sweep (up to 4 tokens: all of an entry's rows in one batch of loads, issued
-//     before the entry's cache offset is known); the softmax (max, then exp-weighted sums)
-//     runs in fp32 per channel. (Two entries' rows per batch was slower after an L2 flush.)
+//     coalesced sweep (up to 2 tokens: all of an entry's rows in one batch of loads, issued
+//     before the entry's cache offset is known; more tokens: a pass for the maxima, then one
+//     for the sums); the softmax (max, then exp-weighted sums) runs in fp32 per channel.
+//     (Two entries' rows per batch was slower after an L2 flush.)
 //     The bf16 latent goes to the global FP4 cache (codes + scale, this lane's block) and
 //     into shared memory as the MMA's A operand (K-major, 128-byte swizzle, 8 slabs of
 //     64 channels);
@@ -39,7 +41,7 @@ constexpr int kM = 128;                    // MMA rows (A operand rows in shared
 constexpr int kMaxE = 32;                  // entries per CTA at most (rows E.. of the MMA unused)
 constexpr int kD = 512;                    // latent channels
 constexpr int kDi = 128;                   // indexer-key channels
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kESlab = kM * 128;           // 128 entries x 64 bf16 channels = 16 KiB
 constexpr int kWSlab = 64 * 128;           // 64 key channels x 64 bf16 channels = 8 KiB
 constexpr int kOffE = 0;                   // 8 slabs: 128 KiB
@@ -225,11 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) x[k] = 0.f;
-        if (have && a.r <= 4) {
-            // up to 4 tokens: every latent and logit row of the entry in one batch of loads
-            uint4 zr[4][2], cr[4][2];
+        if (have && a.r <= 2) {
+            // up to 2 tokens: every latent and logit row of the entry in one batch of loads
+            // (a batch of 4 spilled registers at 512 threads)
+            uint4 zr[2][2], cr[2][2];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
+            for (int t = 0; t < 2; ++t) {
                 if (t < a.r) {
                     zr[t][0] = ld_dep(zrow(b, j, t));
                     zr[t][1] = ld_dep(zrow(b, j, t) + 1);
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cr[t][1] = ld_dep(crow_src(b, j, t) + 1);
                 }
             }
-            pool_rows<4>(zr, cr, a.r, x);
+            pool_rows<2>(zr, cr, a.r, x);
         } else if (have) {
             float zmax[16], den[16], num[16];
 #pragma unroll
