@@ -875,6 +875,8 @@ def main():
                     help="context-parallel Full layer of the 1M-context workload over the ranks")
     ap.add_argument("--eager", action="store_true",
                     help="launch every call from Python instead of replaying CUDA graphs")
+    ap.add_argument("--compress-only", action="store_true",
+                    help="time only the KV compressor cases (one GPU; one JSON line each)")
     args = ap.parse_args()
 
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
@@ -889,6 +891,13 @@ def main():
         return reference_arm(args, rank, world, local)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.compress_only:
+        if world != 1:
+            sys.exit("bench.py: --compress-only runs on one GPU")
+        for name, B, n_new, r, cap in COMPRESS_CASES:
+            m = measure_compress(name, B, n_new, r, cap, args.seed, args.steps, dev)
+            print(json.dumps({"workload": name, **m}), flush=True)
+        return
     pg = None
     if world > 1:
         import datetime
